@@ -1,0 +1,398 @@
+"""Pins of the fp64 oracle to things other than itself: values written out by hand from the
+pages (tests/golden), closed forms, library routines that the definition reduces to in special
+cases, invariants, and brute force on tiny inputs.  CPU only."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import wam_oracle as O
+from tests.golden import load
+
+RNG = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------------------- schedules
+
+def test_video_schedule_lands_exactly_on_sigma_star():
+    meta, _ = load("schedules.txt")
+    n, end, *want = meta["video"]
+    s = O.flow_schedule(n, end)
+    assert s[0] == 1.0 and s[-1] == 0.9          # bit-exact endpoints
+    assert np.all(np.diff(s) < 0)
+    np.testing.assert_allclose(s, want, rtol=0, atol=1e-15)
+
+
+def test_action_schedule_runs_one_to_zero():
+    meta, _ = load("schedules.txt")
+    n, end, *want = meta["action"]
+    s = O.flow_schedule(n, end)
+    assert s[0] == 1.0 and s[-1] == 0.0
+    np.testing.assert_allclose(s, want, rtol=0, atol=1e-15)
+
+
+def test_time_shift_closed_form():
+    # s*u/(1+(s-1)u): endpoints fixed, u=1/2 -> s/(s+1)
+    for s in (0.5, 3.0, 5.0):
+        v = O.time_shift([0.0, 0.5, 1.0], s)
+        assert v[0] == 0.0 and v[2] == 1.0
+        assert abs(v[1] - s / (s + 1)) < 1e-15
+    sched = O.flow_schedule(4, 0.9, shift=3.0)
+    assert sched[0] == 1.0 and sched[-1] == 0.9
+
+
+def test_schedule_rejects_zero_steps():
+    with pytest.raises(ValueError):
+        O.flow_schedule(0)
+
+
+# ----------------------------------------------------------------------------- Euler
+
+def test_euler_with_true_target_recovers_x0():
+    # x_sigma = (1 - sigma) x0 + sigma eps, u = eps - x0: from x = eps at sigma = 1 the
+    # full schedule must return x0 and the partial one the path point at sigma* = 0.9.
+    x0, eps = RNG.standard_normal((5, 7)), RNG.standard_normal((5, 7))
+    for n, end in ((10, 0.0), (4, 0.9), (2, 0.9), (3, 0.5)):
+        s = O.flow_schedule(n, end)
+        x = eps.copy()
+        for i in range(n):
+            x = O.euler_step(x, eps - x0, s[i + 1] - s[i])
+        np.testing.assert_allclose(x, (1 - end) * x0 + end * eps, rtol=0, atol=1e-13)
+
+
+def test_euler_with_state_dependent_field_is_exact_on_a_line():
+    # For a single data point x0 the ideal velocity at x_sigma is (x_sigma - x0) / sigma;
+    # trajectories are straight lines in sigma, so Euler is exact at every step.
+    x0, eps = RNG.standard_normal(9), RNG.standard_normal(9)
+    s = O.flow_schedule(10, 0.0)
+    x = eps.copy()
+    for i in range(10):
+        x = O.euler_step(x, (x - x0) / s[i], s[i + 1] - s[i])
+        np.testing.assert_allclose(x, (1 - s[i + 1]) * x0 + s[i + 1] * eps, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- masks
+
+@pytest.mark.parametrize("name", ["video_mask_F3_T2_pad100.txt",
+                                  "video_mask_F3_T2_pad100_blocks011.txt",
+                                  "video_mask_F4_T1_pad0100_call23.txt"])
+def test_video_mask_matches_hand_written(name):
+    meta, want = load(name)
+    pad = np.array([meta["pad"]], dtype=np.uint8)
+    F = pad.shape[1]
+    T = want.shape[1] // F
+    got = O.video_allowed(pad, meta["blocks"], T, meta["f_begin"][0], meta["f_end"][0])
+    assert got.shape == (1,) + want.shape
+    np.testing.assert_array_equal(got[0].astype(int), want)
+
+
+def test_action_mask_matches_hand_written():
+    meta, want = load("action_mask_F3_T2_pad100_nact2.txt")
+    pad = np.array([meta["pad"]], dtype=np.uint8)
+    got = O.action_key_allowed(pad, 2, meta["n_act"][0])
+    np.testing.assert_array_equal(got.astype(int), want)
+    assert O.action_key_allowed(pad, 2, 3, with_video=False).all()
+
+
+@pytest.mark.parametrize("F,T,P", [(5, 3, 0), (6, 2, 2), (4, 4, 3)])
+def test_video_mask_pair_counts(F, T, P):
+    pad = np.zeros((2, F), np.uint8)
+    pad[:, :P] = 1
+    v = F - P
+    m = O.video_allowed(pad, None, T, 0, F)
+    assert m.sum() == 2 * T * T * v * (v + 1) // 2           # block lower triangle
+    m1 = O.video_allowed(pad, [0] * F, T, 0, F)
+    assert m1.sum() == 2 * (v * T) ** 2                      # one block: all valid pairs
+
+
+def test_video_mask_call_slice_is_rows_of_full_call():
+    pad = np.array([[1, 0, 0, 1, 0, 0]], np.uint8)
+    full = O.video_allowed(pad, None, 3, 0, 6)
+    part = O.video_allowed(pad, None, 3, 2, 5)
+    np.testing.assert_array_equal(part[0], full[0, 6:15, :15])
+
+
+def test_block_ids_validation():
+    with pytest.raises(ValueError):
+        O.block_ids([0, 2, 1], 3)
+    with pytest.raises(ValueError):
+        O.block_ids([0, 1], 3)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _sdpa(q, k, v, **kw):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), **kw)[0, 0].numpy()
+
+
+def test_single_frame_is_textbook_attention():
+    T, D = 12, 16
+    q, k, v = (RNG.standard_normal((1, T, 1, D)) for _ in range(3))
+    o = O.video_prefill(q, k, v, None, None, np.zeros((1, 1), np.uint8), None, T, 0, 1)
+    np.testing.assert_allclose(o[0, :, 0], _sdpa(q[0, :, 0], k[0, :, 0], v[0, :, 0]),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_one_token_frames_are_causal_attention():
+    F, D = 9, 8
+    q, k, v = (RNG.standard_normal((1, F, 1, D)) for _ in range(3))
+    o = O.video_prefill(q, k, v, None, None, np.zeros((1, F), np.uint8), None, 1, 0, F)
+    np.testing.assert_allclose(o[0, :, 0], _sdpa(q[0, :, 0], k[0, :, 0], v[0, :, 0],
+                                                 is_causal=True), rtol=1e-12, atol=1e-12)
+
+
+def test_brute_force_tiny_with_padding_and_cache():
+    # Pure-Python loops with math.exp over the predicate stated in words.
+    B, H, D, T, F, fb = 2, 2, 4, 2, 4, 1
+    pad = np.array([[0, 1, 0, 0], [1, 0, 0, 0]], np.uint8)
+    q = RNG.standard_normal((B, (F - fb) * T, H, D))
+    kn, vn = RNG.standard_normal((2, B, (F - fb) * T, H, D))
+    kc, vc = RNG.standard_normal((2, B, F * T, H, D))
+    got = O.video_prefill(q, kn, vn, kc, vc, pad, None, T, fb, F)
+    for b in range(B):
+        for h in range(H):
+            for i in range(q.shape[1]):
+                fq = fb + i // T
+                num, den = np.zeros(D), 0.0
+                for kt in range(F * T):
+                    fk = kt // T
+                    if pad[b, fq] or pad[b, fk] or fk > fq:
+                        continue
+                    kk = kc[b, kt, h] if fk < fb else kn[b, kt - fb * T, h]
+                    vv = vc[b, kt, h] if fk < fb else vn[b, kt - fb * T, h]
+                    w = math.exp(sum(q[b, i, h, d] * kk[d] for d in range(D)) / math.sqrt(D))
+                    num, den = num + w * vv, den + w
+                want = num / den if den else np.zeros(D)
+                np.testing.assert_allclose(got[b, i, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_two_key_closed_form_pins_the_scale():
+    # q = a e1, keys +e1 and -e1, values 1 and 0: O = sigmoid(2 a / sqrt(D)).
+    D, a = 16, 3.0
+    q = np.zeros((1, D)); q[0, 0] = a
+    k = np.zeros((2, D)); k[0, 0], k[1, 0] = 1.0, -1.0
+    v = np.array([[1.0], [0.0]])
+    o = O.masked_attention(q, k, v, np.ones((1, 2), bool), 1 / math.sqrt(D))
+    assert abs(o[0, 0] - 1 / (1 + math.exp(-2 * a / math.sqrt(D)))) < 1e-15
+
+
+def test_constant_values_and_padded_rows():
+    B, H, D, T, F = 1, 1, 8, 3, 4
+    pad = np.array([[1, 1, 0, 0]], np.uint8)
+    q, k = RNG.standard_normal((2, B, F * T, H, D))
+    v = np.full((B, F * T, H, D), 2.5)
+    o = O.video_prefill(q, k, v, None, None, pad, None, T, 0, F)
+    assert np.all(o[0, :2 * T] == 0.0)
+    np.testing.assert_allclose(o[0, 2 * T:], 2.5, rtol=1e-14)
+
+
+def test_padded_keys_and_later_frames_do_not_matter():
+    B, H, D, T, F = 1, 2, 8, 2, 5
+    pad = np.array([[1, 0, 1, 0, 0]], np.uint8)
+    q, k, v = RNG.standard_normal((3, B, F * T, H, D))
+    base = O.video_prefill(q, k, v, None, None, pad, None, T, 0, F)
+    k2, v2 = k.copy(), v.copy()
+    for f in (0, 2):
+        k2[0, f * T:(f + 1) * T] = 1e3 * RNG.standard_normal((T, H, D))
+        v2[0, f * T:(f + 1) * T] = -7.0
+    np.testing.assert_array_equal(base, O.video_prefill(q, k2, v2, None, None, pad, None, T, 0, F))
+    k3 = k.copy(); k3[0, 4 * T:] += 5.0
+    o3 = O.video_prefill(q, k3, v, None, None, pad, None, T, 0, F)
+    np.testing.assert_array_equal(base[0, :4 * T], o3[0, :4 * T])
+
+
+def test_two_calls_through_the_cache_equal_one_call():
+    B, H, D, T, F, Fh = 2, 2, 8, 3, 5, 3
+    pad = np.array([[1, 0, 0, 0, 0], [0, 0, 0, 0, 0]], np.uint8)
+    q, k, v = RNG.standard_normal((3, B, F * T, H, D))
+    whole = O.video_prefill(q, k, v, None, None, pad, None, T, 0, F)
+    kc = O.cache_store(np.zeros((B, F * T, H, D)), k[:, :Fh * T], pad, T, 0, Fh)
+    vc = O.cache_store(np.zeros((B, F * T, H, D)), v[:, :Fh * T], pad, T, 0, Fh)
+    fut = O.video_prefill(q[:, Fh * T:], k[:, Fh * T:], v[:, Fh * T:], kc, vc, pad, None, T, Fh, F)
+    np.testing.assert_allclose(fut, whole[:, Fh * T:], rtol=1e-13, atol=1e-13)
+
+
+def test_cache_store_skips_padding_only():
+    pad = np.array([[1, 0, 0]], np.uint8)
+    old = np.full((1, 6, 1, 1), -1.0)
+    new = np.arange(6.0).reshape(1, 6, 1, 1)
+    got = O.cache_store(old, new, pad, 2, 0, 3)
+    np.testing.assert_array_equal(got.ravel(), [-1, -1, 2, 3, 4, 5])
+
+
+# ----------------------------------------------------------------------------- fusion
+
+def test_partition_of_thirty_layers_by_four():
+    parts = O.interval_partition(30, 4)
+    assert len(parts) == 8 and parts[0] == [0, 1, 2, 3] and parts[-1] == [28, 29]
+    assert sum(len(p) for p in parts) == 30
+    assert O.interaction_layers(30, 4) == [3, 7, 11, 15, 19, 23, 27, 29]
+    assert O.interval_partition(4, 2) == [[0, 1], [2, 3]]
+    assert O.interaction_layers(30, 1) == list(range(30))
+
+
+def test_fuse_weights_closed_forms():
+    w = O.fuse_weights([0.0, math.log(3.0)])
+    np.testing.assert_allclose(w, [0.25, 0.75], rtol=1e-15)
+    np.testing.assert_array_equal(O.fuse_weights([0.0, -np.inf, -np.inf]), [1.0, 0.0, 0.0])
+    np.testing.assert_allclose(O.fuse_weights([2.0] * 4), [0.25] * 4, rtol=1e-15)
+    x = RNG.standard_normal(4)
+    assert abs(O.fuse_weights(x).sum() - 1.0) < 1e-15
+    np.testing.assert_allclose(O.fuse_weights(x + 100.0), O.fuse_weights(x), rtol=1e-14)
+
+
+def test_fusion_one_hot_reproduces_a_layer_exactly():
+    layers = [RNG.standard_normal((1, 6, 2, 4)) for _ in range(4)]
+    for j in range(4):
+        w = np.zeros(4); w[j] = 1.0
+        np.testing.assert_array_equal(O.fuse_interval(layers, w), layers[j])
+
+
+def test_fusion_closed_form_and_mean():
+    layers = [np.full((2, 3), float(j + 1)) for j in range(4)]
+    w = np.array([0.1, 0.2, 0.3, 0.4])
+    np.testing.assert_allclose(O.fuse_interval(layers, w), 3.0, rtol=1e-15)  # sum_j w_j (j+1)
+    eq = O.fuse_interval(layers, O.fuse_weights([0.0] * 4))
+    np.testing.assert_allclose(eq, 2.5, rtol=1e-15)
+    assert O.fuse_interval(layers, w).shape == layers[0].shape       # one layer's length
+
+
+# ----------------------------------------------------------------------------- action attention
+
+def test_action_self_only_is_bidirectional_attention():
+    B, n, H, D = 1, 6, 2, 8
+    qa, ka, va = RNG.standard_normal((3, B, n, H, D))
+    o = O.action_attention(qa, ka, va, None, None, np.zeros((1, 1), np.uint8), 4)
+    for h in range(H):
+        np.testing.assert_allclose(o[0, :, h], _sdpa(qa[0, :, h], ka[0, :, h], va[0, :, h]),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_action_attention_equals_masked_library_attention():
+    B, n, H, D, T, F = 2, 4, 2, 8, 3, 4
+    pad = np.array([[1, 1, 0, 0], [0, 0, 1, 0]], np.uint8)
+    qa, ka, va = RNG.standard_normal((3, B, n, H, D))
+    fk, fv = RNG.standard_normal((2, B, F * T, H, D))
+    o = O.action_attention(qa, ka, va, fk, fv, pad, T)
+    for b in range(B):
+        keep = np.concatenate([np.repeat(pad[b] == 0, T), np.ones(n, bool)])
+        mask = torch.from_numpy(np.repeat(keep[None], n, axis=0))[None, None]
+        for h in range(H):
+            K = np.concatenate([fk[b, :, h], ka[b, :, h]])
+            V = np.concatenate([fv[b, :, h], va[b, :, h]])
+            want = _sdpa(qa[b, :, h], K, V, attn_mask=mask[0, 0])
+            np.testing.assert_allclose(o[b, :, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_action_two_buffer_merge_equals_concatenation():
+    # One softmax over [video; action] equals two per-buffer softmaxes merged by their
+    # log-sum-exp (the shared normalisation of Long-WAM Summary §4.2).
+    n, D, Nv = 5, 8, 11
+    q, ka, va = RNG.standard_normal((3, n, D))
+    kv, vv = RNG.standard_normal((2, Nv, D))
+    s = 1 / math.sqrt(D)
+    whole = O.masked_attention(q, np.concatenate([kv, ka]), np.concatenate([vv, va]),
+                               np.ones((n, Nv + n), bool), s)
+    def part(k, v):
+        z = s * q @ k.T
+        m = z.max(1, keepdims=True)
+        p = np.exp(z - m)
+        return p @ v, p.sum(1, keepdims=True), m
+    o1, l1, m1 = part(kv, vv)
+    o2, l2, m2 = part(ka, va)
+    m = np.maximum(m1, m2)
+    merged = (o1 * np.exp(m1 - m) + o2 * np.exp(m2 - m)) / (l1 * np.exp(m1 - m) + l2 * np.exp(m2 - m))
+    np.testing.assert_allclose(whole, merged, rtol=1e-12, atol=1e-12)
+
+
+def test_action_all_video_padded_equals_self_only():
+    B, n, H, D, T, F = 1, 4, 1, 8, 2, 3
+    qa, ka, va = RNG.standard_normal((3, B, n, H, D))
+    fk, fv = RNG.standard_normal((2, B, F * T, H, D))
+    pad = np.ones((1, F), np.uint8)
+    np.testing.assert_allclose(O.action_attention(qa, ka, va, fk, fv, pad, T),
+                               O.action_attention(qa, ka, va, None, None, pad, T), rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------- chunk
+
+def _tiny_inputs(B=1, L=4, S=2, H=2, D=4, T=2, Fh=2, Ff=2, n=3, Nv=2, Ne=3, C=3, A=2):
+    r = np.random.default_rng(7)
+    g = lambda *s: r.standard_normal(s)
+    M = -(-L // S)
+    inp = {
+        "hist_q": [g(B, Fh * T, H, D) for _ in range(L)],
+        "hist_k": [g(B, Fh * T, H, D) for _ in range(L)],
+        "hist_v": [g(B, Fh * T, H, D) for _ in range(L)],
+        "imag_q": [[g(B, Ff * T, H, D) for _ in range(L)] for _ in range(Nv)],
+        "imag_k": [[g(B, Ff * T, H, D) for _ in range(L)] for _ in range(Nv)],
+        "imag_v": [[g(B, Ff * T, H, D) for _ in range(L)] for _ in range(Nv)],
+        "final_q": [g(B, Ff * T, H, D) for _ in range(L)],
+        "final_k": [g(B, Ff * T, H, D) for _ in range(L)],
+        "final_v": [g(B, Ff * T, H, D) for _ in range(L)],
+        "fuse_weights": [O.fuse_weights(g(len(I))) for I in O.interval_partition(L, S)],
+        "act_q": [[g(B, n, H, D) for _ in range(L)] for _ in range(Ne)],
+        "act_k": [[g(B, n, H, D) for _ in range(L)] for _ in range(Ne)],
+        "act_v": [[g(B, n, H, D) for _ in range(L)] for _ in range(Ne)],
+        "x_future": g(B, Ff * T, C), "v_future": [g(B, Ff * T, C) for _ in range(Nv)],
+        "x_act": g(B, n, A), "v_act": [g(B, n, A) for _ in range(Ne)],
+    }
+    kw = dict(L=L, S=S, T=T, F_h=Fh, F_f=Ff, n_video_steps=Nv, n_euler_steps=Ne, sigma_star=0.9)
+    return inp, kw, M
+
+
+def test_chunk_composes_the_stage_definitions():
+    inp, kw, M = _tiny_inputs()
+    pad = np.array([[1, 0, 0, 0]], np.uint8)
+    out = O.chunk(inp, pad=pad, **kw)
+    L, T, Fh, Ff = kw["L"], kw["T"], kw["F_h"], kw["F_f"]
+    # Euler chains close in one sum of dsigma * v
+    s_a = O.flow_schedule(kw["n_euler_steps"])
+    want = inp["x_act"] + sum((s_a[i + 1] - s_a[i]) * inp["v_act"][i]
+                              for i in range(kw["n_euler_steps"]))
+    np.testing.assert_allclose(out["x_act"], want, atol=1e-13)
+    s_v = O.flow_schedule(kw["n_video_steps"], 0.9)
+    want = inp["x_future"] - 0.1 * sum(inp["v_future"]) / kw["n_video_steps"]
+    np.testing.assert_allclose(out["x_future"], want, atol=1e-13)
+    assert abs(s_v[-1] - s_v[0] + 0.1) < 1e-15
+    # per-layer cache of valid frames = that layer's history / final-pass K
+    for l in range(L):
+        np.testing.assert_array_equal(out["k_cache"][l][:, T:Fh * T], inp["hist_k"][l][:, T:])
+        np.testing.assert_array_equal(out["v_cache"][l][:, Fh * T:], inp["final_v"][l])
+    # fused pair m = weighted sum of its interval's caches
+    for m, I in enumerate(O.interval_partition(L, kw["S"])):
+        fk = sum(w * out["k_cache"][j] for w, j in zip(inp["fuse_weights"][m], I))
+        np.testing.assert_allclose(out["fused_k"][m], fk, atol=1e-14)
+    # layers outside the interaction set never read video
+    for i in range(kw["n_euler_steps"]):
+        for l in range(L):
+            if l in O.interaction_layers(L, kw["S"]):
+                continue
+            so = O.action_attention(inp["act_q"][i][l], inp["act_k"][i][l], inp["act_v"][i][l],
+                                    None, None, pad, T)
+            np.testing.assert_array_equal(out["act_o"][i][l], so)
+    # imagination outputs read the history cache of their own layer
+    l = 1
+    whole_q = np.concatenate([inp["hist_q"][l], inp["imag_q"][0][l]], axis=1)
+    whole_k = np.concatenate([inp["hist_k"][l], inp["imag_k"][0][l]], axis=1)
+    whole_v = np.concatenate([inp["hist_v"][l], inp["imag_v"][0][l]], axis=1)
+    one = O.video_prefill(whole_q, whole_k, whole_v, None, None, pad, None, T, 0, Fh + Ff)
+    np.testing.assert_allclose(out["imag_o"][0][l], one[:, Fh * T:], atol=1e-13)
+
+
+def test_action_never_changes_video_outputs():
+    inp, kw, _ = _tiny_inputs()
+    pad = np.zeros((1, 4), np.uint8)
+    a = O.chunk(inp, pad=pad, **kw)
+    inp2 = dict(inp)
+    inp2["act_k"] = [[x + 3.0 for x in row] for row in inp["act_k"]]
+    inp2["act_v"] = [[x - 2.0 for x in row] for row in inp["act_v"]]
+    b = O.chunk(inp2, pad=pad, **kw)
+    for key in ("hist_o", "final_o"):
+        for x, y in zip(a[key], b[key]):
+            np.testing.assert_array_equal(x, y)
+    for m in range(len(a["fused_k"])):
+        np.testing.assert_array_equal(a["fused_k"][m], b["fused_k"][m])

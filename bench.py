@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark: action chunks/s of the WAM attention stack at 19.2 s of context on B200.
+
+One step = one whole action chunk (every stage a3-a8) over one synthetic episode:
+30-layer history prefill with the cache store and fusion epilogue, 4 imagination passes x 30
+layers, the final cache pass, 10 Euler steps x 30 action layers (8 reading a fused pair).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs its own episode
+(independent replicas, no collective on the data path; weak scaling); the timed region is
+bracketed by a barrier + synchronize and the reported time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this path has) on the
+host cores, on a bounded sample of the same workload, extrapolated to a whole chunk.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import signal
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from cached_kv_attention_b200 import synth  # noqa: E402
+
+METRIC = "action chunks/s at 19.2 s context (1 B200); % HBM / tensor-core roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="ctx19.2s_bf16", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--fusion", default="epilogue", choices=["epilogue", "standalone"])
+    ap.add_argument("--no-graph", action="store_true", help="issue the chunk eagerly")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------ work model
+
+def algorithmic_work(w: synth.Workload, pad: np.ndarray) -> dict:
+    """Allowed work of one chunk, counting only allowed (query, key) pairs and valid keys.
+
+    prefill FLOPs = 4 D H T^2 x sum over calls and valid query frames of the valid key
+    frames it reads; action bytes = fused valid keys x H x D x 2 (K, V) x 2 B per interaction
+    read plus Q/K/V (bf16) and O (fp32) of every action call."""
+    T, D, H = w.T, w.D, w.H
+    pair = 4.0 * D * H * T * T
+    hist_pairs = fut_pairs = 0
+    valid_keys = 0
+    for b in range(w.B):
+        valid = [f for f in range(w.F) if not pad[b, f]]
+        valid_keys += len(valid) * T
+        for f in range(w.F_h):
+            if not pad[b, f]:
+                hist_pairs += sum(1 for g in valid if g <= f)
+        for f in range(w.F_h, w.F):
+            fut_pairs += sum(1 for g in valid if g <= f)
+    n_pass_fut = w.n_video_steps + 1
+    flops_hist = pair * hist_pairs * w.L
+    flops_fut = pair * fut_pairs * w.L * n_pass_fut
+    act_qkvo = w.n_act * H * D * (3 * 2 + 4) * w.B
+    reads = w.M * w.n_euler_steps
+    calls = w.L * w.n_euler_steps
+    action_bytes = valid_keys * H * D * 2 * 2 * reads + act_qkvo * calls
+    fused_read_bytes = valid_keys * H * D * 2 * 2  # one fused pair read
+    return {
+        "prefill_flops": flops_hist + flops_fut,
+        "prefill_launches": w.L * (1 + n_pass_fut),
+        "action_bytes": action_bytes,
+        "action_launches": calls,
+        "action_reads": reads,
+        "fused_read_bytes": fused_read_bytes,
+        "valid_keys": valid_keys,
+    }
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) taken while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.path = index, None, None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.send_signal(signal.SIGTERM)
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) >= 9:
+                rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------------------------ distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample_seconds(w: synth.Workload, pad: np.ndarray, n_heads: int, n_layers: int,
+                          seed: int, row_stride: int = 1) -> float:
+    """Time the oracle (as it stands) over every stage of one chunk for n_heads heads and
+    n_layers layers (inputs drawn per head, same distributions), computing every
+    row_stride-th video query row (rows are independent).  Returns seconds."""
+    from oracle import wam_oracle as O
+    T, D = w.T, w.D
+    hist, fut = w.F_h * T, w.F_f * T
+    g = lambda name, tok, *i: synth.normal((w.B, tok, n_heads, D), seed, "cpu_" + name, *i,
+                                           std=w.qkv_std, dtype=torch.bfloat16).double().numpy()
+    layers = list(range(n_layers))
+    hq = [g("hq", hist, l) for l in layers]
+    hk = [g("hk", hist, l) for l in layers]
+    hv = [g("hv", hist, l) for l in layers]
+    iq = [[g("iq", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
+    ik = [[g("ik", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
+    iv = [[g("iv", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
+    aq = [[g("aq", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
+    ak = [[g("ak", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
+    av = [[g("av", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
+    xf = np.zeros((w.B, fut, w.C))
+    vf = np.ones((w.B, fut, w.C))
+    xa = np.zeros((w.B, w.n_act, w.A))
+    va = np.ones((w.B, w.n_act, w.A))
+    N = w.F * T
+    t0 = time.perf_counter()
+    kc = [O.cache_store(np.zeros((w.B, N, n_heads, D)), hk[l], pad, T, 0, w.F_h) for l in layers]
+    vc = [O.cache_store(np.zeros((w.B, N, n_heads, D)), hv[l], pad, T, 0, w.F_h) for l in layers]
+    rows_h = np.arange(0, hist, row_stride)
+    rows_f = np.arange(0, fut, row_stride)
+    for l in layers:
+        O.video_prefill(hq[l], hk[l], hv[l], None, None, pad, None, T, 0, w.F_h, rows=rows_h)
+    sv = O.flow_schedule(w.n_video_steps, w.sigma_star)
+    for s in range(w.n_video_steps + 1):
+        for l in layers:
+            O.video_prefill(iq[s][l], ik[s][l], iv[s][l], kc[l], vc[l], pad, None, T, w.F_h, w.F,
+                            rows=rows_f)
+        if s < w.n_video_steps:
+            xf = O.euler_step(xf, vf, sv[s + 1] - sv[s])
+    for l in layers:
+        kc[l] = O.cache_store(kc[l], ik[-1][l], pad, T, w.F_h, w.F)
+        vc[l] = O.cache_store(vc[l], iv[-1][l], pad, T, w.F_h, w.F)
+    wts = O.fuse_weights(np.zeros(n_layers))
+    fk = O.fuse_interval(kc, wts)
+    fv = O.fuse_interval(vc, wts)
+    sa = O.flow_schedule(w.n_euler_steps)
+    interaction = max(1, round(n_layers * w.M / w.L))
+    for i in range(w.n_euler_steps):
+        for j, l in enumerate(layers):
+            video = j < interaction
+            O.action_attention(aq[i][l], ak[i][l], av[i][l], fk if video else None,
+                               fv if video else None, pad, T)
+        xa = O.euler_step(xa, va, sa[i + 1] - sa[i])
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w: synth.Workload, pad: np.ndarray, seed: int) -> dict:
+    n_heads, n_layers = 1, 4
+    sec = oracle_sample_seconds(w, pad, n_heads, n_layers, seed)
+    scale = (w.H / n_heads) * (w.L / n_layers)
+    chunk_s = sec * scale
+    return {"value": 1.0 / chunk_s, "unit": "chunks/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"all stages of one chunk for {n_heads}/{w.H} heads x {n_layers}/{w.L} layers "
+                      f"({sec:.1f} s of fp64 CPU work), extrapolated x{scale:.0f} to a whole chunk"}
+
+
+# ------------------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    pad = synth.pad_mask(w).numpy()
+    n_heads, n_layers, stride = 1, 1, 4
+    scale = (w.H / n_heads) * (w.L / n_layers)
+    for i in range(args.warmup):
+        oracle_sample_seconds(w, pad, n_heads, n_layers, seed=1000 + i, row_stride=stride)
+    times = [oracle_sample_seconds(w, pad, n_heads, n_layers, seed=2000 + i, row_stride=stride)
+             for i in range(args.steps)]
+    # the video stages were sampled on 1/stride of their query rows: time them at full rows
+    full = oracle_sample_seconds(w, pad, n_heads, n_layers, seed=3000, row_stride=1)
+    part = oracle_sample_seconds(w, pad, n_heads, n_layers, seed=3000, row_stride=stride)
+    chunk_s = sum(times) / len(times) * (full / part) * scale
+    value = 1.0 / chunk_s
+    sample = (f"each step: all stages of one chunk for {n_heads}/{w.H} heads x {n_layers}/{w.L} "
+              f"layers on every {stride}th video query row, scaled to all rows by one full-row "
+              f"step (x{full / part:.2f}) and x{scale:.0f} to a whole chunk")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": chunk_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "T": w.T,
+                   "F_h": w.F_h, "F_f": w.F_f, "pad_frames": int(pad.sum()), "n_act": w.n_act,
+                   "n_video_steps": w.n_video_steps, "n_euler_steps": w.n_euler_steps},
+        "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ this library
+
+def run_mine(args, world, rank, local):
+    from cached_kv_attention_b200 import chunk as C
+    from cached_kv_attention_b200 import wam
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w0 = synth.WORKLOADS[args.workload]
+    w = w0.replace(seed=w0.seed + 1000 * rank)  # each rank: its own episode
+    pad = synth.pad_mask(w0).numpy()
+    work = algorithmic_work(w, pad)
+
+    inp = C.make_inputs(w, device="cuda")
+    stream = torch.cuda.current_stream()
+    runner = C.ChunkRunner(w, inp, pad=pad, distinct_out=False, fusion=args.fusion).prepare(stream)
+    launches = runner.launches_per_chunk()
+
+    ev = {name: (torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for name in ("video", "action")}
+    runner.run()  # first call: one-time per-device set-up outside any capture
+    torch.cuda.synchronize()
+    wam.device_error()
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            runner.run(events=ev)
+        step = graph.replay
+    else:
+        step = lambda: runner.run(events=ev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stage_ms = {k: [] for k in ev}
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t_start.elapsed_time(t_end)
+    # Stage events are re-recorded by every step: read the last timed step's stage times,
+    # then time up to 10 more steps one by one for the stage averages.
+    for k, (a, b) in ev.items():
+        stage_ms[k].append(a.elapsed_time(b))
+    for _ in range(min(args.steps, 10)):
+        step()
+        torch.cuda.synchronize()
+        for k, (a, b) in ev.items():
+            stage_ms[k].append(a.elapsed_time(b))
+    wam.device_error()
+    ms = max_over_ranks(total_ms / args.steps, world)
+    video_ms = statistics.mean(stage_ms["video"])
+    action_ms = statistics.mean(stage_ms["action"])
+
+    peaks = {}
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        peaks = json.load(open(pk))
+    tflops_peak = peaks.get("bf16_tflops_sustained")
+    hbm_peak = peaks.get("hbm_gbs")
+    peak_src = "measured" if peaks else "fallback"
+    if tflops_peak is None:
+        tflops_peak = 1400.0
+    if hbm_peak is None:
+        hbm_peak = 6650.0
+
+    prefill_tflops = work["prefill_flops"] / (video_ms * 1e-3) / 1e12
+    action_gbs = work["action_bytes"] / (action_ms * 1e-3) / 1e9
+    roofline = {"bound": "tensor", "achieved": prefill_tflops, "peak": tflops_peak,
+                "unit": "TFLOP/s", "frac": prefill_tflops / tflops_peak, "traffic": None,
+                "kernel": "wam_video_prefill_kv (tensor-core prefill)",
+                "peak_kind": f"{peak_src} bf16 sustained",
+                "flops_per_launch": work["prefill_flops"] / work["prefill_launches"],
+                "ms_per_launch": video_ms / work["prefill_launches"]}
+    roofline_action = {"bound": "hbm", "achieved": action_gbs, "peak": hbm_peak, "unit": "GB/s",
+                       "frac": action_gbs / hbm_peak, "frac_of_8tbs": action_gbs / 8000.0,
+                       "kernel": "wam_action_attn (all 300 calls of the chunk, 80 fused reads)",
+                       "peak_kind": f"{peak_src} copy bandwidth",
+                       "bytes_per_chunk": work["action_bytes"]}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, w, runner, inp, step, pad, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, pad, seed=7)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * 1000.0 / ms, "unit": "chunks/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "T": w.T,
+                       "F_h": w.F_h, "F_f": w.F_f, "pad_frames": int(pad.sum()),
+                       "valid_keys": work["valid_keys"], "n_act": w.n_act,
+                       "n_video_steps": w.n_video_steps, "n_euler_steps": w.n_euler_steps,
+                       "fusion_stride": w.S, "fusion": args.fusion,
+                       "launch": "cuda graph" if graph is not None else "eager",
+                       "l2": "inputs larger than L2: ~25 GB of distinct per-layer buffers per chunk",
+                       "parallelism": f"replicas x{world}"},
+            "stage_ms": {"video": video_ms, "action": action_ms},
+            "roofline": roofline,
+            "roofline_action": roofline_action,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+
+
+def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
+    """Chunks/s through the public API with the chunk's inputs in pinned HOST memory: every
+    step copies the inputs it reads (the non-padding frames of every Q/K/V tensor, the
+    velocities and initial noise) host -> device, runs the chunk and reads x_act back."""
+    stream = torch.cuda.current_stream()
+    valid = [f for f in range(w.F) if not pad[0, f]] if w.B == 1 else None
+    copies = []  # (device tensor view, host tensor view)
+    pools = {}
+
+    def host_like(key, t, slot):
+        k = (key, slot)
+        if k not in pools:
+            pools[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            pools[k].copy_(t.cpu() if t.numel() < (1 << 26) else torch.ones(t.shape, dtype=t.dtype))
+        return pools[k]
+
+    def add(key, t, slot, frame_rows=None):
+        h = host_like(key, t, slot)
+        if frame_rows is None:
+            copies.append((t, h))
+        else:
+            for r0, r1 in frame_rows:
+                copies.append((t[:, r0:r1], h[:, r0:r1]))
+
+    T = w.T
+    runs = []
+    if valid is not None:
+        hv = [f for f in valid if f < w.F_h]
+        if hv:
+            s0 = hv[0]
+            prev = s0
+            for f in hv[1:] + [None]:
+                if f is None or f != prev + 1:
+                    runs.append((s0 * T, (prev + 1) * T))
+                    if f is not None:
+                        s0 = f
+                if f is not None:
+                    prev = f
+    else:
+        runs = None
+    for name in ("hist_q", "hist_k", "hist_v"):
+        for l, t in enumerate(inp[name]):
+            add(name, t, l % 2, runs)
+    for name in ("imag_q", "imag_k", "imag_v", "act_q", "act_k", "act_v"):
+        for i, row in enumerate(inp[name]):
+            for l, t in enumerate(row):
+                add(name, t, (i + l) % 2)
+    for name in ("final_q", "final_k", "final_v"):
+        for l, t in enumerate(inp[name]):
+            add(name, t, l % 2)
+    for name in ("v_future", "v_act"):
+        for i, t in enumerate(inp[name]):
+            add(name, t, i % 2)
+    add("x_future", runner.x_future, 0)
+    add("x_act", runner.x_act, 0)
+    h2d = sum(d.numel() * d.element_size() for d, _ in copies)
+    out_host = torch.empty(runner.x_act.shape, dtype=torch.float32, pin_memory=True)
+    d2h = out_host.numel() * 4
+
+    def one():
+        for d, h in copies:
+            d.copy_(h, non_blocking=True)
+        step()
+        out_host.copy_(runner.x_act, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
+    return {"value": world * 1000.0 / ms, "unit": "chunks/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "inputs in pinned host memory; non-padding frames of every Q/K/V tensor "
+                    "copied host->device each step, x_act read back"}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("bench.py: this implementation needs a CUDA GPU (B200)")
+            run_mine(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

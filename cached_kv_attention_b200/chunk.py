@@ -1,0 +1,235 @@
+"""One action chunk of the WAM attention stack, issued through the C ABI.
+
+Stage order (one chunk):
+  a3  history prefill, one call per layer, with the cache store and the fusion epilogue
+  a4  N_v imagination passes (future queries over cached history + current future K/V),
+      each followed by an Euler step of the future latents (sigma 1 -> sigma*)
+  a5  final pass at sigma*, storing the future K/V and completing the fused pairs
+  a6  Interval KV-Fusion (in the a3/a5 epilogues, or as standalone calls)
+  a7  N_e Euler steps x L action layers: the M interaction layers read their fused pair,
+      the others attend to the action chunk only
+  a8  one Euler step of the action latents per step
+("Long-WAM 源码精读" §04; "世界模型之Faster-WAM详解" §3.1-3.4; "Fast-WAM 精读" SECTION 07.)
+
+Projections, MLPs and RoPE need trained weights, so every pass takes fresh seeded Q/K/V and
+every Euler step a seeded velocity.  The chunk's arguments are marshalled once in
+``prepare``; ``run`` then only issues the C calls on one stream, which also lets a CUDA graph
+capture the whole chunk.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, List, Optional
+
+import numpy as np
+import torch
+
+from . import synth
+from . import wam
+from .synth import Workload
+
+__all__ = ["make_inputs", "ChunkRunner", "interval_partition", "interaction_layers"]
+
+
+def interval_partition(L: int, S: int) -> List[List[int]]:
+    """Layers of each fusion interval: {S*m, ..., min(S*m + S, L) - 1}."""
+    return [list(range(S * m, min(S * m + S, L))) for m in range(-(-L // S))]
+
+
+def interaction_layers(L: int, S: int) -> List[int]:
+    """The action layer that reads interval m is the last layer of the interval."""
+    return [I[-1] for I in interval_partition(L, S)]
+
+
+def make_inputs(w: Workload, device: str = "cpu") -> Dict:
+    """Seeded inputs of one chunk (see ``synth``); drawn on ``device``."""
+    dt = synth.torch_dtype(w)
+    B, H, D, T = w.B, w.H, w.D, w.T
+    hist, fut = w.F_h * T, w.F_f * T
+
+    def qkv(name, tokens, *idx):
+        return synth.normal((B, tokens, H, D), w.seed, name, *idx, std=w.qkv_std, dtype=dt,
+                            device=device)
+
+    inp = {
+        "hist_q": [qkv("hist_q", hist, l) for l in range(w.L)],
+        "hist_k": [qkv("hist_k", hist, l) for l in range(w.L)],
+        "hist_v": [qkv("hist_v", hist, l) for l in range(w.L)],
+        "imag_q": [[qkv("imag_q", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
+        "imag_k": [[qkv("imag_k", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
+        "imag_v": [[qkv("imag_v", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
+        "final_q": [qkv("final_q", fut, l) for l in range(w.L)],
+        "final_k": [qkv("final_k", fut, l) for l in range(w.L)],
+        "final_v": [qkv("final_v", fut, l) for l in range(w.L)],
+        "fuse_logits": [synth.normal((len(I),), w.seed, "fuse_logits", m)
+                        for m, I in enumerate(interval_partition(w.L, w.S))],
+        "act_q": [[qkv("act_q", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
+        "act_k": [[qkv("act_k", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
+        "act_v": [[qkv("act_v", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
+        "x_future": synth.normal((B, fut, w.C), w.seed, "x_future", device=device),
+        "v_future": [synth.normal((B, fut, w.C), w.seed, "v_future", s, device=device)
+                     for s in range(w.n_video_steps)],
+        "x_act": synth.normal((B, w.n_act, w.A), w.seed, "x_act", device=device),
+        "v_act": [synth.normal((B, w.n_act, w.A), w.seed, "v_act", i, device=device)
+                  for i in range(w.n_euler_steps)],
+    }
+    return inp
+
+
+def _vp(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class ChunkRunner:
+    """Device buffers and the prepared C calls of one chunk.
+
+    inputs        dict from ``make_inputs`` (tensors already on the device)
+    distinct_out  keep one output buffer per pass (tests) or reuse one per pass kind (bench)
+    fusion        "epilogue" (fold in the cache store) or "standalone" (wam_fuse_interval_kv)
+    """
+
+    def __init__(self, w: Workload, inputs: Dict, pad=None, frame_block=None,
+                 distinct_out: bool = True, fusion: str = "epilogue", o_dtype=torch.float32,
+                 device: str = "cuda"):
+        self.w, self.inp, self.fusion = w, inputs, fusion
+        dt = synth.torch_dtype(w)
+        B, H, D, T, F, N = w.B, w.H, w.D, w.T, w.F, w.N
+        pad = synth.pad_mask(w) if pad is None else pad
+        self.pad = np.asarray(pad, dtype=np.uint8)
+        self.layout = wam.VideoLayout(B, H, D, T, F, self.pad, frame_block)
+        dev = torch.device(device)
+        z = lambda *s, dtype=dt: torch.zeros(s, dtype=dtype, device=dev)
+        self.k_cache = [z(B, N, H, D) for _ in range(w.L)]
+        self.v_cache = [z(B, N, H, D) for _ in range(w.L)]
+        self.fused_k = [z(B, N, H, D) for _ in range(w.M)]
+        self.fused_v = [z(B, N, H, D) for _ in range(w.M)]
+        self.acc_k = z(B, N, H, D, dtype=torch.float32)
+        self.acc_v = z(B, N, H, D, dtype=torch.float32)
+        hist, fut = w.F_h * T, w.F_f * T
+        n_h = w.L if distinct_out else 1
+        n_i = w.L * w.n_video_steps if distinct_out else 1
+        n_a = w.L * w.n_euler_steps if distinct_out else 1
+        self.hist_o = [z(B, hist, H, D, dtype=o_dtype) for _ in range(n_h)]
+        self.final_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_h)]
+        self.imag_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_i)]
+        self.act_o = [z(B, w.n_act, H, D, dtype=o_dtype) for _ in range(n_a)]
+        self.x_future = inputs["x_future"].clone()
+        self.x_act = inputs["x_act"].clone()
+        self.sig_v = wam.flow_schedule(w.n_video_steps, w.sigma_star)
+        self.sig_a = wam.flow_schedule(w.n_euler_steps, 0.0)
+        self.parts = interval_partition(w.L, w.S)
+        self.fw = [wam.fuse_weights(lg.cpu().numpy()) for lg in inputs["fuse_logits"]]
+        self.calls: List = []
+        self._keep: List = []
+
+    # ------------------------------------------------------------------ preparation
+    def _epilogue(self, l: int):
+        if self.fusion != "epilogue":
+            return None
+        m, j = l // self.w.S, l % self.w.S
+        I = self.parts[m]
+        e = wam.FuseEpilogue(self.fw[m][j], j == 0, l == I[-1], self.acc_k, self.acc_v,
+                             self.fused_k[m], self.fused_v[m])
+        self._keep.append(e)
+        return e.ref
+
+    def prepare(self, stream=None) -> "ChunkRunner":
+        w, L = self.w, wam.lib
+        s = ctypes.c_void_p(wam._stream(stream))
+        lay = self.layout.ref
+        dt = wam.BF16 if w.dtype == "bf16" else wam.F32
+        o_dt = wam.F32 if self.hist_o[0].dtype == torch.float32 else dt
+        inp, F_h, F = self.inp, w.F_h, w.F
+        calls = []
+
+        def o_of(lst, idx):
+            return _vp(lst[idx % len(lst)])
+
+        # a3: history prefill with the cache store (+ fusion epilogue)
+        for l in range(w.L):
+            calls.append((L.wam_video_prefill_kv,
+                          (lay, dt, 0, F_h, _vp(inp["hist_q"][l]), _vp(inp["hist_k"][l]),
+                           _vp(inp["hist_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
+                           o_of(self.hist_o, l), o_dt, self._epilogue(l), s)))
+        # a4: imagination passes + Euler on the future latents
+        nf = self.x_future.numel()
+        for st in range(w.n_video_steps):
+            for l in range(w.L):
+                calls.append((L.wam_video_prefill_kv,
+                              (lay, dt, F_h, F, _vp(inp["imag_q"][st][l]),
+                               _vp(inp["imag_k"][st][l]), _vp(inp["imag_v"][st][l]),
+                               _vp(self.k_cache[l]), _vp(self.v_cache[l]), 0,
+                               o_of(self.imag_o, st * w.L + l), o_dt, None, s)))
+            ds = float(self.sig_v[st + 1] - self.sig_v[st])
+            calls.append((L.wam_flow_euler_step, (nf, _vp(self.x_future),
+                                                  _vp(inp["v_future"][st]), ds, s)))
+        # a5: final pass at sigma*, store future K/V (+ complete the fused pairs)
+        for l in range(w.L):
+            calls.append((L.wam_video_prefill_kv,
+                          (lay, dt, F_h, F, _vp(inp["final_q"][l]), _vp(inp["final_k"][l]),
+                           _vp(inp["final_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
+                           o_of(self.final_o, l), o_dt, self._epilogue(l), s)))
+        # a6 standalone: fuse each interval over all frames once the caches are complete
+        if self.fusion == "standalone":
+            for m, I in enumerate(self.parts):
+                kp = (ctypes.c_void_p * len(I))(*[self.k_cache[j].data_ptr() for j in I])
+                vp = (ctypes.c_void_p * len(I))(*[self.v_cache[j].data_ptr() for j in I])
+                wt = (ctypes.c_float * len(I))(*[float(x) for x in self.fw[m]])
+                self._keep += [kp, vp, wt]
+                calls.append((L.wam_fuse_interval_kv,
+                              (lay, dt, len(I), kp, vp, wt, 0, F, _vp(self.fused_k[m]),
+                               _vp(self.fused_v[m]), s)))
+        video_end = len(calls)
+        # a7 + a8: action denoising
+        reader = {j: m for m, j in enumerate(interaction_layers(w.L, w.S))}
+        na = self.x_act.numel()
+        for i in range(w.n_euler_steps):
+            for l in range(w.L):
+                m = reader.get(l)
+                fk = _vp(self.fused_k[m]) if m is not None else None
+                fv = _vp(self.fused_v[m]) if m is not None else None
+                calls.append((L.wam_action_attn,
+                              (lay, dt, fk, fv, w.n_act, _vp(inp["act_q"][i][l]),
+                               _vp(inp["act_k"][i][l]), _vp(inp["act_v"][i][l]),
+                               o_of(self.act_o, i * w.L + l), o_dt, s)))
+            ds = float(self.sig_a[i + 1] - self.sig_a[i])
+            calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
+        self.calls = calls
+        # stage boundaries (call indices): the video stages a3-a6 (prefill kernels plus four
+        # small Euler steps), then the action stages a7-a8
+        self.stages = [("video", 0, video_end), ("action", video_end, len(calls))]
+        return self
+
+    def reset_latents(self) -> None:
+        """Restore the Euler states to the chunk's initial noise (device copies)."""
+        self.x_future.copy_(self.inp["x_future"])
+        self.x_act.copy_(self.inp["x_act"])
+
+    def run(self, events: Optional[Dict] = None, stream=None) -> None:
+        """Issue the chunk.  ``events`` maps a stage name to (start, end) CUDA events that are
+        recorded on ``stream`` around that stage (also inside a graph capture when the events
+        are external)."""
+        if not events:
+            for fn, args in self.calls:
+                st = fn(*args)
+                if st:
+                    wam.check(st)
+            return
+        stream = torch.cuda.current_stream() if stream is None else stream
+        for name, i0, i1 in self.stages:
+            ev = events.get(name)
+            if ev:
+                ev[0].record(stream)
+            for fn, args in self.calls[i0:i1]:
+                st = fn(*args)
+                if st:
+                    wam.check(st)
+            if ev:
+                ev[1].record(stream)
+
+    # ------------------------------------------------------------------ counts
+    def launches_per_chunk(self) -> int:
+        """Kernels this chunk launches (the library launches one kernel per call, except the
+        CUDA-core prefill path, which adds a store kernel)."""
+        return len(self.calls)

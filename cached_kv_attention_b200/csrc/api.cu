@@ -1,0 +1,414 @@
+// C-ABI entry points: argument validation (before any CUDA call), construction of the
+// per-launch work lists from the host padding mask and attention blocks, and dispatch to the
+// tensor-core or CUDA-core kernels.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+
+// The device error word: kernels whose bounded waits give up write WAM_ERR_TIMEOUT here.
+__device__ int g_wam_device_error = 0;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// Address of the error word on the current device (looked up once per device).
+int* device_error_word() {
+  static int* addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wam_device_error) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+wam_status fail(wam_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+wam_status ok() {
+  g_last_error.clear();
+  return WAM_OK;
+}
+
+wam_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(WAM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validated geometry with the derived per-episode valid-frame lists.
+struct Geo {
+  int B, H, D, T, F;
+  std::vector<uint8_t> pad;     // [B*F]
+  std::vector<int32_t> block;   // [F]
+  std::vector<int> kf_end;      // [F]: first frame after the block of f
+};
+
+wam_status check_layout(const wam_video_layout* L, Geo& g) {
+  if (!L) return fail(WAM_ERR_INVALID_ARGUMENT, "layout is NULL");
+  if (L->B < 1 || L->H < 1 || L->T < 1 || L->F < 1)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "B, H, T, F must be >= 1 (got %d, %d, %d, %d)", L->B,
+                L->H, L->T, L->F);
+  if (L->D != 64 && L->D != 128)
+    return fail(WAM_ERR_UNSUPPORTED, "head dim D must be 64 or 128 (got %d)", L->D);
+  if (L->F > WAM_MAX_FRAMES)
+    return fail(WAM_ERR_UNSUPPORTED, "F = %d exceeds WAM_MAX_FRAMES = %d", L->F, WAM_MAX_FRAMES);
+  if (int64_t(L->B) * L->F > WAM_MAX_EPISODE_FRAMES)
+    return fail(WAM_ERR_UNSUPPORTED, "B * F = %lld exceeds WAM_MAX_EPISODE_FRAMES = %d",
+                (long long)L->B * L->F, WAM_MAX_EPISODE_FRAMES);
+  if (int64_t(L->T) * L->F > (int64_t(1) << 24) || L->H > 4096)
+    return fail(WAM_ERR_UNSUPPORTED, "F * T or H too large");
+  g.B = L->B, g.H = L->H, g.D = L->D, g.T = L->T, g.F = L->F;
+  g.pad.assign(size_t(g.B) * g.F, 0);
+  if (L->frame_pad)
+    for (size_t i = 0; i < g.pad.size(); ++i) {
+      if (L->frame_pad[i] > 1)
+        return fail(WAM_ERR_INVALID_ARGUMENT, "frame_pad[%zu] = %u is not 0 or 1", i,
+                    unsigned(L->frame_pad[i]));
+      g.pad[i] = L->frame_pad[i];
+    }
+  g.block.resize(g.F);
+  for (int f = 0; f < g.F; ++f) {
+    g.block[f] = L->frame_block ? L->frame_block[f] : f;
+    if (f && g.block[f] < g.block[f - 1])
+      return fail(WAM_ERR_INVALID_ARGUMENT, "frame_block must be nondecreasing (frame %d)", f);
+  }
+  g.kf_end.resize(g.F);
+  for (int f = g.F - 1; f >= 0; --f)
+    g.kf_end[f] = (f + 1 < g.F && g.block[f + 1] == g.block[f]) ? g.kf_end[f + 1] : f + 1;
+  return WAM_OK;
+}
+
+wam_status check_dtype(wam_dtype dt, const char* name) {
+  if (dt != WAM_F32 && dt != WAM_BF16)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, int(dt));
+  return WAM_OK;
+}
+
+// Valid-frame lists of every episode.
+void fill_vlists(const Geo& g, wam::FrameLists& fl) {
+  for (int b = 0; b < g.B; ++b) {
+    int n = 0;
+    for (int f = 0; f < g.F; ++f)
+      if (!g.pad[size_t(b) * g.F + f]) fl.vlist[b * g.F + n++] = uint16_t(f);
+    fl.nvalid[b] = uint16_t(n);
+  }
+}
+
+// Work items of a prefill call: every valid query frame in [f_begin, f_end), with the number
+// of valid key frames it reads (those of blocks up to its own), longest first.
+void fill_items(const Geo& g, int f_begin, int f_end, wam::FrameLists& fl) {
+  std::vector<uint32_t> items;
+  for (int b = 0; b < g.B; ++b)
+    for (int f = f_begin; f < f_end; ++f) {
+      if (g.pad[size_t(b) * g.F + f]) continue;
+      int nk = 0;
+      for (int u = 0; u < fl.nvalid[b]; ++u)
+        if (fl.vlist[b * g.F + u] < g.kf_end[f]) ++nk;
+      items.push_back(wam::pack_item(b, f, nk));
+    }
+  std::stable_sort(items.begin(), items.end(), [](uint32_t x, uint32_t y) {
+    return wam::item_nk(x) > wam::item_nk(y);
+  });
+  fl.n_items = int32_t(items.size());
+  std::copy(items.begin(), items.end(), fl.item);
+}
+
+wam_status check_range(const Geo& g, int f_begin, int f_end) {
+  if (f_begin < 0 || f_end > g.F || f_begin >= f_end)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "frame range [%d, %d) is not inside [0, %d)", f_begin,
+                f_end, g.F);
+  if (f_begin > 0 && g.block[f_begin - 1] == g.block[f_begin])
+    return fail(WAM_ERR_INVALID_ARGUMENT, "f_begin = %d splits an attention block", f_begin);
+  if (f_end < g.F && g.block[f_end - 1] == g.block[f_end])
+    return fail(WAM_ERR_INVALID_ARGUMENT, "f_end = %d splits an attention block", f_end);
+  return WAM_OK;
+}
+
+#define WAM_CHECK(expr)            \
+  do {                             \
+    wam_status st_ = (expr);       \
+    if (st_ != WAM_OK) return st_; \
+  } while (0)
+
+#define WAM_NONNULL_ALIGNED(p)                                                             \
+  do {                                                                                     \
+    if (!(p)) return fail(WAM_ERR_INVALID_ARGUMENT, "%s is NULL", #p);                    \
+    if (!aligned16(p)) return fail(WAM_ERR_INVALID_ARGUMENT, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+// Tensor-core eligibility of a bf16 video/action call.
+bool tc_video_ok(const Geo& g, wam_dtype dt) { return dt == WAM_BF16 && g.D == 128 && g.T % 128 == 0; }
+bool tc_action_ok(const Geo& g, wam_dtype dt, int n_act) {
+  return dt == WAM_BF16 && g.D == 128 && g.T % 64 == 0 && n_act <= 32;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+// tensor maps (driver entry point fetched through the runtime; no -lcuda)
+// ---------------------------------------------------------------------------------------
+namespace wam {
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int B, int ntok, int H, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return false;
+  const cuuint64_t dims[4] = {128, cuuint64_t(H), cuuint64_t(ntok), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(128) * 2, cuuint64_t(H) * 128 * 2,
+                                 cuuint64_t(ntok) * H * 128 * 2};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+}  // namespace wam
+
+// ---------------------------------------------------------------------------------------
+// entry points
+// ---------------------------------------------------------------------------------------
+extern "C" {
+
+int32_t wam_version(void) { return 100; }
+
+const char* wam_last_error(void) { return g_last_error.c_str(); }
+
+wam_status wam_flow_schedule(int32_t n_steps, double sigma_end, double shift, double* sigmas) {
+  if (n_steps < 1) return fail(WAM_ERR_INVALID_ARGUMENT, "n_steps must be >= 1");
+  if (!sigmas) return fail(WAM_ERR_INVALID_ARGUMENT, "sigmas is NULL");
+  if (!(shift > 0.0) || !std::isfinite(sigma_end) || sigma_end < 0.0 || sigma_end >= 1.0)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "need shift > 0 and 0 <= sigma_end < 1");
+  for (int i = 0; i <= n_steps; ++i) {
+    const double u = double(n_steps - i) / double(n_steps);
+    const double phi = shift == 1.0 ? u : shift * u / (1.0 + (shift - 1.0) * u);
+    sigmas[i] = sigma_end + (1.0 - sigma_end) * phi;
+  }
+  return ok();
+}
+
+wam_status wam_fuse_weights(int32_t n, const float* logits, float* weights) {
+  if (n < 1 || n > WAM_MAX_FUSE_LAYERS)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n must be in [1, %d]", WAM_MAX_FUSE_LAYERS);
+  if (!logits || !weights) return fail(WAM_ERR_INVALID_ARGUMENT, "NULL pointer");
+  double mx = -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    if (std::isnan(logits[i]) || logits[i] == INFINITY)
+      return fail(WAM_ERR_INVALID_ARGUMENT, "logit %d is not finite or -inf", i);
+    mx = std::max(mx, double(logits[i]));
+  }
+  if (mx == -INFINITY) return fail(WAM_ERR_INVALID_ARGUMENT, "all logits are -inf");
+  double e[WAM_MAX_FUSE_LAYERS], s = 0.0;
+  for (int i = 0; i < n; ++i) s += (e[i] = std::exp(double(logits[i]) - mx));
+  for (int i = 0; i < n; ++i) weights[i] = float(e[i] / s);
+  return ok();
+}
+
+wam_status wam_flow_euler_step(int64_t n, float* x, const float* v, float dsigma,
+                               wam_stream_t stream) {
+  if (n < 0) return fail(WAM_ERR_INVALID_ARGUMENT, "n must be >= 0");
+  if (n == 0) return ok();
+  WAM_NONNULL_ALIGNED(x);
+  WAM_NONNULL_ALIGNED(v);
+  if (!std::isfinite(dsigma)) return fail(WAM_ERR_INVALID_ARGUMENT, "dsigma is not finite");
+  return cuda_status(wam::launch_euler(n, x, v, dsigma, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_flow_euler_step");
+}
+
+wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt, int32_t f_begin,
+                                int32_t f_end, const void* q, const void* k_new,
+                                const void* v_new, void* k_cache, void* v_cache,
+                                int32_t store_kv, void* o, wam_dtype o_dt,
+                                const wam_fuse_epilogue* fuse, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(dt, "dt"));
+  WAM_CHECK(check_dtype(o_dt, "o_dt"));
+  if (o_dt != WAM_F32 && o_dt != dt)
+    return fail(WAM_ERR_UNSUPPORTED, "o_dt must be WAM_F32 or the input dtype");
+  WAM_CHECK(check_range(g, f_begin, f_end));
+  WAM_NONNULL_ALIGNED(q);
+  WAM_NONNULL_ALIGNED(k_new);
+  WAM_NONNULL_ALIGNED(v_new);
+  WAM_NONNULL_ALIGNED(o);
+  if (f_begin > 0 || store_kv) {
+    WAM_NONNULL_ALIGNED(k_cache);
+    WAM_NONNULL_ALIGNED(v_cache);
+  }
+  if (fuse) {
+    if (!std::isfinite(fuse->weight))
+      return fail(WAM_ERR_INVALID_ARGUMENT, "fuse->weight is not finite");
+    if (!(fuse->first_in_interval && fuse->last_in_interval)) {
+      WAM_NONNULL_ALIGNED(fuse->acc_k);
+      WAM_NONNULL_ALIGNED(fuse->acc_v);
+    }
+    if (fuse->last_in_interval) {
+      WAM_NONNULL_ALIGNED(fuse->fused_k);
+      WAM_NONNULL_ALIGNED(fuse->fused_v);
+    }
+  }
+  static thread_local wam::PrefillArgs a;  // large; built on the host per call
+  std::memset(&a, 0, sizeof(a));
+  a.q = q, a.k_new = k_new, a.v_new = v_new, a.k_cache = k_cache, a.v_cache = v_cache;
+  a.k_store = store_kv ? k_cache : nullptr;
+  a.v_store = store_kv ? v_cache : nullptr;
+  a.o = o;
+  if (fuse) {
+    a.fuse_on = 1, a.fuse_first = fuse->first_in_interval ? 1 : 0;
+    a.fuse_last = fuse->last_in_interval ? 1 : 0, a.fuse_w = fuse->weight;
+    a.acc_k = fuse->acc_k, a.acc_v = fuse->acc_v, a.fused_k = fuse->fused_k, a.fused_v = fuse->fused_v;
+  }
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.f_begin = f_begin, a.f_end = f_end;
+  a.o_f32 = o_dt == WAM_F32;
+  a.scale_log2 = float(wam::kLog2e / std::sqrt(double(g.D)));
+  a.err = device_error_word();
+  fill_vlists(g, a.fl);
+  fill_items(g, f_begin, f_end, a.fl);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dt == WAM_BF16;
+  if (tc_video_ok(g, dt)) {
+    cudaError_t e = wam::launch_prefill_tc(a, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e, "wam_video_prefill_kv (tensor cores)");
+  }
+  cudaError_t e = wam::launch_prefill_simt(a, g.D, bf16, s);
+  if (e == cudaSuccess) e = wam::launch_store_fuse(a, g.D, bf16, s);
+  return cuda_status(e, "wam_video_prefill_kv");
+}
+
+wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, int32_t n_layers,
+                                const void* const* k_layers, const void* const* v_layers,
+                                const float* weights, int32_t f_begin, int32_t f_end,
+                                void* fused_k, void* fused_v, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(dt, "dt"));
+  if (n_layers < 1 || n_layers > WAM_MAX_FUSE_LAYERS)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n_layers must be in [1, %d]", WAM_MAX_FUSE_LAYERS);
+  if (!k_layers || !v_layers || !weights)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "k_layers, v_layers and weights must not be NULL");
+  if (f_begin < 0 || f_end > g.F || f_begin >= f_end)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "frame range [%d, %d) is not inside [0, %d)", f_begin,
+                f_end, g.F);
+  WAM_NONNULL_ALIGNED(fused_k);
+  WAM_NONNULL_ALIGNED(fused_v);
+  static thread_local wam::FuseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int l = 0; l < n_layers; ++l) {
+    if (!k_layers[l] || !v_layers[l] || !aligned16(k_layers[l]) || !aligned16(v_layers[l]))
+      return fail(WAM_ERR_INVALID_ARGUMENT, "layer %d pointer is NULL or not 16-byte aligned", l);
+    if (!std::isfinite(weights[l]))
+      return fail(WAM_ERR_INVALID_ARGUMENT, "weight %d is not finite", l);
+    a.k[l] = k_layers[l], a.v[l] = v_layers[l], a.w[l] = weights[l];
+  }
+  a.n_layers = n_layers, a.fk = fused_k, a.fv = fused_v, a.F = g.F;
+  a.frame_elems = int64_t(g.T) * g.H * g.D;
+  std::vector<uint32_t> items;
+  for (int b = 0; b < g.B; ++b)
+    for (int f = f_begin; f < f_end; ++f)
+      if (!g.pad[size_t(b) * g.F + f]) items.push_back(wam::pack_item(b, f, 0));
+  a.fl.n_items = int32_t(items.size());
+  std::copy(items.begin(), items.end(), a.fl.item);
+  return cuda_status(wam::launch_fuse(a, g.D, dt == WAM_BF16, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_fuse_interval_kv");
+}
+
+wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const void* fused_k,
+                           const void* fused_v, int32_t n_act, const void* qa, const void* ka,
+                           const void* va, void* o, wam_dtype o_dt, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(dt, "dt"));
+  WAM_CHECK(check_dtype(o_dt, "o_dt"));
+  if (o_dt != WAM_F32 && o_dt != dt)
+    return fail(WAM_ERR_UNSUPPORTED, "o_dt must be WAM_F32 or the input dtype");
+  if (n_act < 1 || n_act > 128)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n_act must be in [1, 128] (got %d)", n_act);
+  if ((fused_k == nullptr) != (fused_v == nullptr))
+    return fail(WAM_ERR_INVALID_ARGUMENT, "fused_k and fused_v must both be set or both NULL");
+  if (fused_k) {
+    WAM_NONNULL_ALIGNED(fused_k);
+    WAM_NONNULL_ALIGNED(fused_v);
+  }
+  WAM_NONNULL_ALIGNED(qa);
+  WAM_NONNULL_ALIGNED(ka);
+  WAM_NONNULL_ALIGNED(va);
+  WAM_NONNULL_ALIGNED(o);
+  static thread_local wam::ActionArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.fk = fused_k, a.fv = fused_v, a.qa = qa, a.ka = ka, a.va = va, a.o = o;
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.n_act = n_act;
+  a.o_f32 = o_dt == WAM_F32;
+  a.with_video = fused_k != nullptr;
+  a.scale_log2 = float(wam::kLog2e / std::sqrt(double(g.D)));
+  a.err = device_error_word();
+  fill_vlists(g, a.fl);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (tc_action_ok(g, dt, n_act)) {
+    cudaError_t e = wam::launch_action_tc(a, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e, "wam_action_attn (tensor cores)");
+  }
+  return cuda_status(wam::launch_action_simt(a, g.D, dt == WAM_BF16, s), "wam_action_attn");
+}
+
+wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
+                                uint8_t* mask, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_range(g, f_begin, f_end));
+  if (!mask) return fail(WAM_ERR_INVALID_ARGUMENT, "mask is NULL");
+  static thread_local wam::PrefillArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.f_begin = f_begin, a.f_end = f_end;
+  fill_vlists(g, a.fl);
+  fill_items(g, f_begin, f_end, a.fl);
+  return cuda_status(wam::launch_debug_mask(a, mask, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_debug_video_mask");
+}
+
+wam_status wam_device_error(int32_t clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "wam_device_error: synchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_wam_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e, "wam_device_error: read");
+  if (clear && v) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_wam_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_status(e, "wam_device_error: clear");
+  }
+  if (v) return fail(wam_status(v), "a kernel's bounded wait gave up (device error word = %d)", v);
+  return ok();
+}
+
+}  // extern "C"

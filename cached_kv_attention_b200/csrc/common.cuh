@@ -1,0 +1,189 @@
+// Shared definitions of the WAM attention kernels (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/wam.h"
+
+namespace wam {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------------------
+// Per-launch work tables (kernel parameters, built on the host from the padding mask and
+// the attention blocks).  A frame of an episode is a contiguous run of T*H*D elements in
+// every token-major tensor, so all work is addressed by (episode, frame).
+// ---------------------------------------------------------------------------------------
+
+// item = b | f << 10 | nk << 21: query frame f of episode b reads the first nk entries of
+// that episode's valid-frame list (keys of blocks <= its own, padding frames left out).
+__host__ __device__ inline uint32_t pack_item(int b, int f, int nk) {
+  return uint32_t(b) | (uint32_t(f) << 10) | (uint32_t(nk) << 21);
+}
+__host__ __device__ inline int item_b(uint32_t it) { return int(it & 1023u); }
+__host__ __device__ inline int item_f(uint32_t it) { return int((it >> 10) & 2047u); }
+__host__ __device__ inline int item_nk(uint32_t it) { return int(it >> 21); }
+
+struct FrameLists {
+  int32_t n_items;                               // prefill / store: valid query frames
+  uint32_t item[WAM_MAX_EPISODE_FRAMES];         // longest-first (descending nk)
+  uint16_t vlist[WAM_MAX_EPISODE_FRAMES];        // valid frames of episode b at [b*F, ...)
+  uint16_t nvalid[WAM_MAX_EPISODE_FRAMES];       // number of valid frames of episode b
+};
+
+struct PrefillArgs {
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  const void* k_cache;  // keys of frames < f_begin
+  const void* v_cache;
+  void* k_store;        // non-null: store new K/V of the call's valid frames
+  void* v_store;
+  void* o;
+  float* acc_k;
+  float* acc_v;
+  void* fused_k;
+  void* fused_v;
+  float fuse_w;
+  int32_t fuse_on, fuse_first, fuse_last;
+  int32_t B, H, T, F, f_begin, f_end;
+  int32_t o_f32;
+  float scale_log2;  // softmax scale * log2(e)
+  int* err;          // device error word (a bounded wait that gave up writes WAM_ERR_TIMEOUT)
+  FrameLists fl;
+};
+
+struct ActionArgs {
+  const void* fk;  // fused video K/V or null
+  const void* fv;
+  const void* qa;
+  const void* ka;
+  const void* va;
+  void* o;
+  int32_t B, H, T, F, n_act;
+  int32_t o_f32;
+  int32_t with_video;
+  int32_t splits;  // split-KV factor = cluster size
+  float scale_log2;
+  int* err;
+  FrameLists fl;
+};
+
+struct FuseArgs {
+  const void* k[WAM_MAX_FUSE_LAYERS];
+  const void* v[WAM_MAX_FUSE_LAYERS];
+  float w[WAM_MAX_FUSE_LAYERS];
+  int32_t n_layers;
+  void* fk;
+  void* fv;
+  int64_t frame_elems;  // T*H*D
+  int32_t F;
+  FrameLists fl;        // items: (b, f) frames to fuse
+};
+
+// ---------------------------------------------------------------------------------------
+// Element access
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+constexpr uint32_t kWaitSpinLimit = 1u << 24;  // try_wait rounds before a wait gives up
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers: shared-memory addresses, mbarriers, TMA, ldmatrix, mma.sync
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false if the phase never flips; the caller then records
+// WAM_ERR_TIMEOUT in the device error word (args.err) and leaves without waiting further.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 4-D tiled TMA load global -> shared, completion counted on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Byte offset of element (row, col) in a [rows x 128] bf16 tile stored as two 128B-swizzled
+// halves of [rows x 64] (the layout a TMA box of 64 x rows with SWIZZLE_128B writes).
+template <int ROWS>
+__device__ __forceinline__ uint32_t swz128(int row, int col) {
+  const int half = col >> 6, cc = col & 63;
+  return uint32_t(half * ROWS * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + ((cc & 7) << 1));
+}
+
+}  // namespace wam

@@ -1,0 +1,27 @@
+// Internal launchers shared by the C-ABI layer (host code only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace wam {
+
+cudaError_t launch_euler(int64_t n, float* x, const float* v, float dsigma, cudaStream_t s);
+cudaError_t launch_store_fuse(const PrefillArgs& a, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_fuse(const FuseArgs& a, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_debug_mask(const PrefillArgs& a, uint8_t* mask, cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_action_simt(const ActionArgs& a, int D, bool bf16, cudaStream_t s);
+
+// Tensor-core paths (bf16, D = 128).  Return cudaErrorNotSupported when the shape has no
+// tensor-core kernel; the caller then takes the CUDA-core path.
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s);
+
+// Tensor map of a token-major bf16 tensor [B, ntok, H, 128] with a box of 64 x rows
+// (128B swizzle), rows along the token dimension.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int B, int ntok, int H, int box_rows);
+
+}  // namespace wam

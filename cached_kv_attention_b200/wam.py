@@ -1,0 +1,202 @@
+"""Thin Python binding of libwam.so: the same entry points as include/wam.h, with torch
+tensors for device memory and streams.  Every wrapper only marshals arguments; all work runs
+in the library's CUDA kernels.  Importing this module fails loudly if the library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+__all__ = [
+    "WamError", "F32", "BF16", "VideoLayout", "FuseEpilogue", "lib",
+    "video_prefill_kv", "fuse_interval_kv", "action_attn", "flow_euler_step",
+    "flow_schedule", "fuse_weights", "debug_video_mask", "device_error", "exported_names",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "WAM_OK", 1: "WAM_ERR_INVALID_ARGUMENT", 2: "WAM_ERR_UNSUPPORTED",
+           3: "WAM_ERR_CUDA", 4: "WAM_ERR_WORKSPACE", 5: "WAM_ERR_TIMEOUT"}
+
+
+class WamError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("T", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("frame_pad", ctypes.c_void_p), ("frame_block", ctypes.c_void_p)]
+
+
+class _Fuse(ctypes.Structure):
+    _fields_ = [("weight", ctypes.c_float), ("first_in_interval", ctypes.c_int32),
+                ("last_in_interval", ctypes.c_int32), ("acc_k", ctypes.c_void_p),
+                ("acc_v", ctypes.c_void_p), ("fused_k", ctypes.c_void_p),
+                ("fused_v", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m cached_kv_attention_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, f64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, \
+        ctypes.c_double
+    lay = ctypes.POINTER(_Layout)
+    sigs = {
+        "wam_video_prefill_kv": [lay, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, i32,
+                                 ctypes.POINTER(_Fuse), vp],
+        "wam_fuse_interval_kv": [lay, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                 ctypes.POINTER(f32), i32, i32, vp, vp, vp],
+        "wam_action_attn": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp],
+        "wam_flow_euler_step": [i64, vp, vp, f32, vp],
+        "wam_flow_schedule": [i32, f64, f64, ctypes.POINTER(f64)],
+        "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
+        "wam_debug_video_mask": [lay, i32, i32, vp, vp],
+        "wam_device_error": [i32],
+    }
+    for name, args in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.wam_last_error.argtypes = []
+    L.wam_last_error.restype = ctypes.c_char_p
+    L.wam_version.argtypes = []
+    L.wam_version.restype = ctypes.c_int32
+    return L
+
+
+lib = _load()
+
+
+def exported_names() -> list:
+    """Names of the C entry points this binding declares (all must be exported)."""
+    return ["wam_video_prefill_kv", "wam_fuse_interval_kv", "wam_action_attn",
+            "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
+            "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version"]
+
+
+def check(status: int) -> None:
+    if status != 0:
+        raise WamError(status, lib.wam_last_error().decode())
+
+
+class VideoLayout:
+    """Geometry of one call: B episodes, H heads, D head dim, T tokens per frame, F frames,
+    an optional host padding mask [B, F] and optional attention-block ids [F]."""
+
+    def __init__(self, B: int, H: int, D: int, T: int, F: int,
+                 frame_pad=None, frame_block: Optional[Sequence[int]] = None):
+        self.B, self.H, self.D, self.T, self.F = B, H, D, T, F
+        self.pad = None if frame_pad is None else \
+            np.ascontiguousarray(np.asarray(frame_pad, dtype=np.uint8).reshape(B, F))
+        self.block = None if frame_block is None else \
+            np.ascontiguousarray(np.asarray(frame_block, dtype=np.int32))
+        self.c = _Layout(B, H, D, T, F,
+                         None if self.pad is None else self.pad.ctypes.data,
+                         None if self.block is None else self.block.ctypes.data)
+        self.ref = ctypes.byref(self.c)
+
+    @property
+    def N(self) -> int:
+        return self.F * self.T
+
+
+class FuseEpilogue:
+    """Interval KV-Fusion folded into one layer's cache store."""
+
+    def __init__(self, weight: float, first: bool, last: bool, acc_k=None, acc_v=None,
+                 fused_k=None, fused_v=None):
+        self.c = _Fuse(float(weight), int(first), int(last), _ptr(acc_k), _ptr(acc_v),
+                       _ptr(fused_k), _ptr(fused_v))
+        self.ref = ctypes.byref(self.c)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def video_prefill_kv(layout: VideoLayout, f_begin: int, f_end: int, q, k_new, v_new,
+                     k_cache, v_cache, o, store_kv: bool = True,
+                     fuse: Optional[FuseEpilogue] = None, stream=None) -> None:
+    check(lib.wam_video_prefill_kv(layout.ref, _dtype(q), f_begin, f_end, _ptr(q), _ptr(k_new),
+                                   _ptr(v_new), _ptr(k_cache), _ptr(v_cache), int(store_kv),
+                                   _ptr(o), _dtype(o), None if fuse is None else fuse.ref,
+                                   _stream(stream)))
+
+
+def fuse_interval_kv(layout: VideoLayout, k_layers, v_layers, weights, f_begin: int,
+                     f_end: int, fused_k, fused_v, stream=None) -> None:
+    n = len(k_layers)
+    kp = (ctypes.c_void_p * n)(*[_ptr(t) for t in k_layers])
+    vp = (ctypes.c_void_p * n)(*[_ptr(t) for t in v_layers])
+    w = (ctypes.c_float * n)(*[float(x) for x in weights])
+    check(lib.wam_fuse_interval_kv(layout.ref, _dtype(fused_k), n, kp, vp, w, f_begin, f_end,
+                                   _ptr(fused_k), _ptr(fused_v), _stream(stream)))
+
+
+def action_attn(layout: VideoLayout, fused_k, fused_v, qa, ka, va, o, stream=None) -> None:
+    check(lib.wam_action_attn(layout.ref, _dtype(qa), _ptr(fused_k), _ptr(fused_v), qa.shape[1],
+                              _ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _stream(stream)))
+
+
+def flow_euler_step(x, v, dsigma: float, stream=None) -> None:
+    if x.dtype != torch.float32 or v.dtype != torch.float32 or x.numel() != v.numel():
+        raise ValueError("x and v must be fp32 tensors of the same size")
+    check(lib.wam_flow_euler_step(x.numel(), _ptr(x), _ptr(v), float(dsigma), _stream(stream)))
+
+
+def flow_schedule(n_steps: int, sigma_end: float = 0.0, shift: float = 1.0) -> np.ndarray:
+    out = np.zeros(n_steps + 1, dtype=np.float64) if n_steps >= 0 else np.zeros(1)
+    check(lib.wam_flow_schedule(n_steps, sigma_end, shift,
+                                out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return out
+
+
+def fuse_weights(logits) -> np.ndarray:
+    x = np.ascontiguousarray(np.asarray(logits, dtype=np.float32))
+    out = np.zeros_like(x)
+    check(lib.wam_fuse_weights(x.size, x.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                               out.ctypes.data_as(ctypes.POINTER(ctypes.c_float))))
+    return out
+
+
+def debug_video_mask(layout: VideoLayout, f_begin: int, f_end: int, stream=None) -> torch.Tensor:
+    T = layout.T
+    mask = torch.empty((layout.B, (f_end - f_begin) * T, f_end * T), dtype=torch.uint8,
+                       device="cuda")
+    check(lib.wam_debug_video_mask(layout.ref, f_begin, f_end, _ptr(mask), _stream(stream)))
+    return mask
+
+
+def device_error(clear: bool = True) -> None:
+    """Synchronise and raise WamError if a kernel's bounded wait gave up."""
+    check(lib.wam_device_error(int(clear)))

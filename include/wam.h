@@ -1,0 +1,206 @@
+/*
+ * wam.h - C ABI of the B200 (sm_100a) attention stack of one world-action-model action chunk.
+ *
+ * The stack has three parts, each defined on the pages named below:
+ *   (a) block-causal video prefill of a per-layer K/V cache over history frames and imagined
+ *       future frames denoised to sigma* ("Long-WAM 源码精读" §03-§04: the video expert rolls the
+ *       future latents from pure noise to sigma* = 0.9 in 4 steps, then prefill_video_cache
+ *       builds a per-layer {"k","v"} list; "Long-WAM: Scaling the Context of World-Action
+ *       Models | Summary" §3.1-3.2: video queries read their own and earlier visual blocks);
+ *   (b) Interval KV-Fusion ("世界模型之Faster-WAM详解" §3.3: the K/V of one depth interval are
+ *       folded into one K/V pair of one layer's length with softmax-normalised weights);
+ *   (c) asymmetric action attention inside the flow-matching Euler loop ("Fast-WAM 精读"
+ *       SECTION 07: K = [K_video; K_action], V = [V_video; V_action], Q/K/V of the actions
+ *       recomputed every step; Long-WAM Summary §4.2: one online softmax over the two buffers).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are token-major [B, tokens, H, D], contiguous, as on "Fast-WAM 精读" SECTION 04
+ *     ([N, 24, 128] per episode).  A per-layer cache or fused cache holds all N = F*T tokens.
+ *   - Device pointers are caller-owned.  The library never allocates, frees or synchronises
+ *     device memory, and never keeps a pointer after a call returns.
+ *   - Every call that touches the GPU is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns once its kernels are enqueued.
+ *   - Every call returns a wam_status; nothing throws or aborts across the ABI.  On an error
+ *     the arguments are rejected before anything is launched, and wam_last_error() returns a
+ *     message for the calling thread.
+ *   - Frame padding and attention blocks are HOST arrays: the host knows which history frames
+ *     exist, and the library turns them into per-launch work lists (no device mask is read).
+ *   - Supported: dtype WAM_F32 or WAM_BF16; D in {64, 128}; 1 <= T; 1 <= F <= WAM_MAX_FRAMES;
+ *     B * F <= WAM_MAX_EPISODE_FRAMES.  bf16 with D = 128 and T % 128 == 0 runs on the tensor
+ *     cores; every other supported shape runs the fp32-accumulating CUDA-core path (also on
+ *     the GPU).  Anything else returns WAM_ERR_UNSUPPORTED.
+ *   - Pointers to bf16 or fp32 tensors must be 16-byte aligned.
+ */
+#ifndef WAM_H_
+#define WAM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* wam_stream_t; /* the same handle as cudaStream_t */
+
+#define WAM_MAX_FRAMES 256
+#define WAM_MAX_EPISODE_FRAMES 1024
+#define WAM_MAX_FUSE_LAYERS 16
+
+typedef enum {
+  WAM_OK = 0,
+  WAM_ERR_INVALID_ARGUMENT = 1, /* a null pointer, bad size, misaligned pointer, bad range */
+  WAM_ERR_UNSUPPORTED = 2,      /* a valid request this build has no kernel for */
+  WAM_ERR_CUDA = 3,             /* a CUDA runtime error while configuring or launching */
+  WAM_ERR_WORKSPACE = 4,        /* reserved */
+  WAM_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up (wam_device_error) */
+} wam_status;
+
+typedef enum { WAM_F32 = 0, WAM_BF16 = 1 } wam_dtype;
+
+/*
+ * Geometry shared by the video and action calls.
+ *   B episodes, H heads, D head dim, T tokens per latent frame, F = history + imagined frames;
+ *   token t belongs to frame t / T, and a cache holds N = F * T tokens.
+ *   frame_pad   host uint8 [B, F], 1 = padding frame (unavailable early history, Long-WAM
+ *               Summary §3.3), NULL = no padding.  Keys of padding frames are never read;
+ *               queries of padding frames are not computed and their output rows are not
+ *               written; their K/V are neither stored nor fused (those rows keep their
+ *               previous contents).
+ *   frame_block host int32 [F], nondecreasing attention-block id of each frame, NULL = one
+ *               block per frame.  A video query reads keys whose block id is <= its own
+ *               (Long-WAM Summary §3.1-3.2); grouping imagined frames into one block lets
+ *               future slots read each other (Faster-WAM详解 §3.1).
+ */
+typedef struct {
+  int32_t B, H, D, T, F;
+  const uint8_t* frame_pad;
+  const int32_t* frame_block;
+} wam_video_layout;
+
+/*
+ * Interval KV-Fusion folded into the cache write of one layer (Faster-WAM详解 §3.3):
+ * for the stored (non-padding) frames of the call,
+ *   first_in_interval:  acc  = w * K_j               (acc is not read)
+ *   middle layers:      acc += w * K_j
+ *   last_in_interval:   fused = round(acc + w * K_j) (acc is read, not written)
+ * and the same for V.  A one-layer interval sets both flags.  acc_k/acc_v are caller-owned
+ * fp32 device scratch [B, N, H, D]; fused_k/fused_v are device [B, N, H, D] of the call's dtype.
+ * The per-layer K/V is folded while it is in on-chip memory and never re-read for fusion.
+ */
+typedef struct {
+  float weight;
+  int32_t first_in_interval;
+  int32_t last_in_interval;
+  float* acc_k;
+  float* acc_v;
+  void* fused_k;
+  void* fused_v;
+} wam_fuse_epilogue;
+
+/*
+ * Block-causal video attention of one layer for the query frames [f_begin, f_end), with the
+ * store of their K/V into that layer's cache ("Long-WAM 源码精读" §04 prefill_video_cache;
+ * Long-WAM Summary §3.2, §4.2 observed-video KV computed once and reused).
+ *
+ *   q, k_new, v_new  device [B, (f_end - f_begin) * T, H, D], dtype dt
+ *   k_cache, v_cache device [B, N, H, D], dtype dt.  Keys of frames [0, f_begin) are read
+ *                    from here (frames stored by earlier calls); if store_kv != 0 the
+ *                    non-padding frames of [f_begin, f_end) are written here from k_new/v_new.
+ *                    May be NULL when f_begin == 0 and store_kv == 0.
+ *   o                device [B, (f_end - f_begin) * T, H, D], dtype o_dt (WAM_F32 or dt);
+ *                    O_q = sum_k softmax_k(q.k / sqrt(D)) v_k over the allowed keys; rows of
+ *                    padding frames are left unwritten.
+ *   fuse             NULL, or the fusion epilogue above (needs store semantics: the frames
+ *                    folded are the non-padding frames of [f_begin, f_end)).
+ * A call must not split an attention block: frame f_begin starts a block and f_end is F or
+ * starts a block.  Accumulation is fp32; P is rounded to bf16 for the PV product on the
+ * tensor-core path.
+ */
+wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt,
+                                int32_t f_begin, int32_t f_end,
+                                const void* q, const void* k_new, const void* v_new,
+                                void* k_cache, void* v_cache, int32_t store_kv,
+                                void* o, wam_dtype o_dt,
+                                const wam_fuse_epilogue* fuse, wam_stream_t stream);
+
+/*
+ * Standalone Interval KV-Fusion (Faster-WAM详解 §3.3): for the non-padding frames of
+ * [f_begin, f_end), fused = round(sum_j weights[j] * layer_j) computed in fp32, for K and V.
+ *   k_layers, v_layers host arrays of n_layers device pointers [B, N, H, D] (dtype dt)
+ *   weights            host float [n_layers] (softmax-normalised, see wam_fuse_weights)
+ *   fused_k, fused_v   device [B, N, H, D] (dtype dt); padding frames are not written.
+ * 1 <= n_layers <= WAM_MAX_FUSE_LAYERS.
+ */
+wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, int32_t n_layers,
+                                const void* const* k_layers, const void* const* v_layers,
+                                const float* weights, int32_t f_begin, int32_t f_end,
+                                void* fused_k, void* fused_v, wam_stream_t stream);
+
+/*
+ * Asymmetric action attention of one action-expert layer at one Euler step ("Fast-WAM 精读"
+ * SECTION 07; Long-WAM Summary §3.2, §4.2; Faster-WAM详解 §3.2 SparseMoT):
+ *   O = softmax(Q_a [K_video(non-padding frames); K_a]^T / sqrt(D)) [V_video; V_a]
+ * computed as split-KV partials over the video keys merged with the action buffer by one
+ * shared online-softmax normalisation (no concatenated buffer is formed).
+ *   fused_k, fused_v device [B, N, H, D] (dtype dt), or both NULL for a layer outside the
+ *                    interaction set (action self-attention only)
+ *   qa, ka, va       device [B, n_act, H, D] (dtype dt), 1 <= n_act <= 128
+ *   o                device [B, n_act, H, D], dtype o_dt (WAM_F32 or dt)
+ * Action tokens attend to each other bidirectionally.  No workspace: the split partials are
+ * merged on chip through the distributed shared memory of a thread-block cluster.
+ */
+wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt,
+                           const void* fused_k, const void* fused_v,
+                           int32_t n_act, const void* qa, const void* ka, const void* va,
+                           void* o, wam_dtype o_dt, wam_stream_t stream);
+
+/*
+ * One Euler step of the flow-matching sampler, x <- x + dsigma * v, elementwise over n fp32
+ * values ("Long-WAM 源码精读" §03: path x_s = (1-s) x + s eps, target u = eps - x;
+ * "Fast-WAM 精读" SECTION 07: the scheduler updates the action latent each step).
+ *   x device fp32 [n], updated in place; v device fp32 [n]; dsigma = sigma_{i+1} - sigma_i.
+ */
+wam_status wam_flow_euler_step(int64_t n, float* x, const float* v, float dsigma,
+                               wam_stream_t stream);
+
+/* ---- host helpers (no GPU work) ---------------------------------------------------------- */
+
+/*
+ * Noise levels of an n-step sampler into host double sigmas[n_steps + 1]:
+ *   u_i = (n - i) / n,  sigma_i = sigma_end + (1 - sigma_end) * phi(u_i)
+ * phi(u) = shift * u / (1 + (shift - 1) u) (identity at shift = 1).  sigma_0 = 1 and
+ * sigma_n = sigma_end exactly ("Long-WAM 源码精读" §04: linspace(1, 0, steps + 1), warped,
+ * then rescaled so the end lands exactly on sigma* and the start stays pure noise).
+ */
+wam_status wam_flow_schedule(int32_t n_steps, double sigma_end, double shift, double* sigmas);
+
+/* Softmax of n host logits into host weights (Faster-WAM详解 §3.3, W_fuse normalisation). */
+wam_status wam_fuse_weights(int32_t n, const float* logits, float* weights);
+
+/*
+ * The video predicate the prefill kernels apply, written out per element for inspection:
+ * mask[b, i, k] = 1 if query token f_begin*T + i may read key token k (k < f_end * T), else 0.
+ *   mask device uint8 [B, (f_end - f_begin) * T, f_end * T].
+ */
+wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
+                                uint8_t* mask, wam_stream_t stream);
+
+/*
+ * Synchronise the current device and report its error word: WAM_OK, or WAM_ERR_TIMEOUT when
+ * a kernel's bounded wait on an mbarrier gave up (the kernel then skipped its remaining work
+ * and returned without faulting).  clear != 0 resets the word.  Host-blocking.
+ */
+wam_status wam_device_error(int32_t clear);
+
+/* Thread-local message of the last failing call on this thread ("" if none). */
+const char* wam_last_error(void);
+
+/* ABI version of this build: major * 10000 + minor * 100 + patch. */
+int32_t wam_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAM_H_ */

@@ -112,18 +112,20 @@ def block_ids(frame_block: Optional[Sequence[int]], n_frames: int) -> np.ndarray
     return blk
 
 
-def video_allowed(pad, frame_block, T: int, f_begin: int, f_end: int) -> np.ndarray:
+def video_allowed(pad, frame_block, T: int, f_begin: int, f_end: int,
+                  rows: Optional[Sequence[int]] = None) -> np.ndarray:
     """Boolean [B, (f_end - f_begin) * T, f_end * T]: may video query q read video key k?
 
     A video query reads its own and earlier visual blocks and never an action token
     ([LW-sum] §3.2); keys of padded (unavailable) frames are never read and queries of padded
     frames produce nothing (reading R3).  Query tokens are the frames [f_begin, f_end) of the
-    call; key tokens are all frames [0, f_end).
+    call; key tokens are all frames [0, f_end).  ``rows`` keeps only those query rows.
     """
     pad = np.asarray(pad).astype(bool)
     B, F = pad.shape
     blk = block_ids(frame_block, F)
-    q_frame = np.arange(f_begin * T, f_end * T) // T
+    q_tok = np.arange(f_begin * T, f_end * T) if rows is None else f_begin * T + np.asarray(rows)
+    q_frame = q_tok // T
     k_frame = np.arange(0, f_end * T) // T
     causal = blk[k_frame][None, :] <= blk[q_frame][:, None]            # [Q, K]
     key_ok = ~pad[:, k_frame]                                            # [B, K]
@@ -205,14 +207,17 @@ def video_prefill(q, k_new, v_new, k_cache, v_cache, pad, frame_block, T: int,
         vals = np.concatenate([_f64(v_cache)[:, :n_old], _f64(v_new)], axis=1)
     else:
         keys, vals = _f64(k_new), _f64(v_new)
-    allowed = video_allowed(pad, frame_block, T, f_begin, f_end)
-    heads = range(H) if heads is None else heads
     rows = np.arange(Q) if rows is None else np.asarray(rows)
+    padb = np.asarray(pad).astype(bool)
+    heads = range(H) if heads is None else heads
     o = np.zeros((B, Q, H, v_new.shape[-1]), dtype=np.float64)
     for b in range(B):
+        # rows of padded query frames read nothing and stay 0 (reading R3): not computed
+        rows_b = rows[~padb[b, f_begin + rows // T]]
+        allowed = video_allowed(padb[b:b + 1], frame_block, T, f_begin, f_end, rows=rows_b)[0]
         for h in heads:
-            o[b, rows, h] = masked_attention(q[b, rows, h], keys[b, :, h], vals[b, :, h],
-                                             allowed[b][rows], scale)
+            o[b, rows_b, h] = masked_attention(q[b, rows_b, h], keys[b, :, h], vals[b, :, h],
+                                               allowed, scale)
     return o
 
 

@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--profile-call", default=None, choices=["history", "future", "action"],
+                    help="launch one stage call of the workload --repeat times and exit "
+                         "(a small case for ncu captures; prints nothing)")
+    ap.add_argument("--repeat", type=int, default=3)
     return ap.parse_args()
 
 
@@ -306,7 +310,10 @@ def run_mine(args, world, rank, local):
     work = algorithmic_work(w, pad)
 
     inp = C.make_inputs(w, device="cuda")
-    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    # one dedicated stream: the chunk is prepared, warmed up, captured and replayed on it
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
     runner = C.ChunkRunner(w, inp, pad=pad, distinct_out=False, fusion=args.fusion).prepare(stream)
     launches = runner.launches_per_chunk()
 
@@ -318,11 +325,11 @@ def run_mine(args, world, rank, local):
     graph = None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            runner.run(events=ev)
+        with torch.cuda.graph(graph, stream=stream):
+            runner.run(events=ev, stream=stream)
         step = graph.replay
     else:
-        step = lambda: runner.run(events=ev)
+        step = lambda: runner.run(events=ev, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -496,8 +503,45 @@ def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
                     "copied host->device each step, x_act read back"}
 
 
+def profile_call(args):
+    """One stage call of one layer at the workload's full size, repeated: the history prefill
+    (with the cache store and a fusion epilogue), a future-frame prefill reading the cache,
+    or a fused action read."""
+    from cached_kv_attention_b200 import wam
+    w = synth.WORKLOADS[args.workload]
+    pad = synth.pad_mask(w).numpy()
+    lay = wam.VideoLayout(w.B, w.H, w.D, w.T, w.F, pad)
+    bf = torch.bfloat16
+    g = lambda n, tok: synth.normal((w.B, tok, w.H, w.D), w.seed, "prof_" + n, std=w.qkv_std,
+                                    dtype=bf, device="cuda")
+    shape = (w.B, w.N, w.H, w.D)
+    kc, vc = g("kc", w.N), g("vc", w.N)
+    if args.profile_call == "history":
+        q, k, v = g("q", w.F_h * w.T), g("k", w.F_h * w.T), g("v", w.F_h * w.T)
+        o = torch.empty((w.B, w.F_h * w.T, w.H, w.D), device="cuda")
+        acc_k = torch.zeros(shape, device="cuda")
+        acc_v = torch.zeros(shape, device="cuda")
+        epi = wam.FuseEpilogue(0.25, False, False, acc_k, acc_v, None, None)
+        call = lambda: wam.video_prefill_kv(lay, 0, w.F_h, q, k, v, kc, vc, o, True, epi)
+    elif args.profile_call == "future":
+        q, k, v = g("q", w.F_f * w.T), g("k", w.F_f * w.T), g("v", w.F_f * w.T)
+        o = torch.empty((w.B, w.F_f * w.T, w.H, w.D), device="cuda")
+        call = lambda: wam.video_prefill_kv(lay, w.F_h, w.F, q, k, v, kc, vc, o, False)
+    else:
+        qa, ka, va = g("qa", w.n_act), g("ka", w.n_act), g("va", w.n_act)
+        o = torch.empty((w.B, w.n_act, w.H, w.D), device="cuda")
+        call = lambda: wam.action_attn(lay, kc, vc, qa, ka, va, o)
+    for _ in range(args.repeat):
+        call()
+    torch.cuda.synchronize()
+    wam.device_error()
+
+
 def main():
     args = parse()
+    if args.profile_call:
+        profile_call(args)
+        return
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

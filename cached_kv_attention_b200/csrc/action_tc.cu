@@ -3,8 +3,10 @@
 // 32 action queries read the fused video cache of one interaction layer plus their own K/V
 // ("Fast-WAM 精读" SECTION 07; Long-WAM Summary §4.2).  The read is HBM-bound: per key it
 // moves 512 B (K and V, bf16) and does 32 x 4 x 128 FLOP, 32 FLOP/B, above what the fp32
-// pipes can issue at full HBM bandwidth, so the dot products run on mma.sync bf16 tiles
-// (M = 32 queries) while the loads stream through TMA.
+// pipes can issue at full HBM bandwidth, so the contractions run on mma.sync tensor-core
+// tiles (M = 32 queries) while the loads stream through TMA: Q K^T on bf16 tiles, P V on tf32
+// tiles (the fused cache is already rounded to bf16 once, so P is kept at 10 mantissa bits
+// to leave the error budget to the storage rounding).
 //
 // Grid = (C splits, H, B), launched as clusters of C CTAs.  Split c of (b, h) reads a
 // contiguous run of 64-key tiles of the episode's valid frames; split 0 also reads the
@@ -208,22 +210,32 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
       for (int j = 0; j < 16; ++j) {
         oacc[j][0] *= al0, oacc[j][1] *= al0, oacc[j][2] *= al1, oacc[j][3] *= al1;
       }
-      // O += P V over this warp's 32 keys
+      // O += P V over this warp's 32 keys on tf32 tiles (m16n8k8): P keeps 10 mantissa bits
+      // instead of bf16's 7, and V widens from bf16 to tf32 exactly.  Within each 8-key group
+      // j the contraction index is permuted (logical k = t <-> key 8j + 2t, k = t + 4 <->
+      // key 8j + 2t + 1), which makes the S accumulators the A fragment and the two keys an
+      // ldmatrix.trans register holds the B fragment, with no data movement.
+      uint32_t pt[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        pt[j][0] = to_tf32(s[j][0]);  // row g,     key 8j + 2t
+        pt[j][1] = to_tf32(s[j][2]);  // row g + 8, key 8j + 2t
+        pt[j][2] = to_tf32(s[j][1]);  // row g,     key 8j + 2t + 1
+        pt[j][3] = to_tf32(s[j][3]);  // row g + 8, key 8j + 2t + 1
+      }
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
-        uint32_t pa[4];
-        pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-        pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-        pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+        const int j0 = 2 * kk, j1 = 2 * kk + 1;  // 8-key groups of this 16-key step
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          uint32_t b0, b1, b2, b3;
+          uint32_t r0, r1, r2, r3;
           ldsm_x4_t(vb + swz128<kBN>(32 * kh + 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8,
                                      16 * p + (lane >> 4) * 8),
-                    b0, b1, b2, b3);
-          mma_bf16(oacc[2 * p], pa, b0, b1);
-          mma_bf16(oacc[2 * p + 1], pa, b2, b3);
+                    r0, r1, r2, r3);
+          mma_tf32(oacc[2 * p], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r0), bf16_hi_bits(r0));
+          mma_tf32(oacc[2 * p], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r1), bf16_hi_bits(r1));
+          mma_tf32(oacc[2 * p + 1], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r2), bf16_hi_bits(r2));
+          mma_tf32(oacc[2 * p + 1], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r3), bf16_hi_bits(r3));
         }
       }
       __syncwarp();

@@ -1,6 +1,9 @@
 """Helpers shared by the GPU parity tests: seeded inputs on the CPU copied to the device, and
 the tolerances the checks apply."""
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -30,6 +33,12 @@ def assert_parity(got, ref, dtype, what=""):
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     err = np.abs(got - ref)
     scale = np.abs(ref).max()
+    log = os.environ.get("WAM_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"what": what, "dtype": str(dtype), "n": int(err.size),
+                                "max_rel": float(err.max() / max(scale, 1e-300)),
+                                "mean_rel": float(err.sum() / max(np.abs(ref).sum(), 1e-300))}) + "\n")
     if dtype in ("f32", torch.float32):
         assert err.max() <= F32_MAX_REL * scale, f"{what}: max err {err.max():.3e} vs {scale:.3e}"
     else:

@@ -171,6 +171,9 @@ bool tc_action_ok(const Geo& g, wam_dtype dt, int n_act) {
 // tensor maps (driver entry point fetched through the runtime; no -lcuda)
 // ---------------------------------------------------------------------------------------
 namespace wam {
+// Records a failure for wam_last_error() from entry points defined in other files.
+wam_status record_error(wam_status st, const char* msg) { return fail(st, "%s", msg); }
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int B, int ntok, int H, int box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;

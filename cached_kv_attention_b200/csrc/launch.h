@@ -24,4 +24,7 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s);
 // (128B swizzle), rows along the token dimension.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int B, int ntok, int H, int box_rows);
 
+// Sets the calling thread's wam_last_error() message and returns st.
+wam_status record_error(wam_status st, const char* msg);
+
 }  // namespace wam

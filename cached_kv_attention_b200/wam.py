@@ -16,6 +16,7 @@ __all__ = [
     "WamError", "F32", "BF16", "VideoLayout", "FuseEpilogue", "lib",
     "video_prefill_kv", "fuse_interval_kv", "action_attn", "flow_euler_step",
     "flow_schedule", "fuse_weights", "debug_video_mask", "device_error", "exported_names",
+    "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
@@ -62,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
         "wam_debug_video_mask": [lay, i32, i32, vp, vp],
         "wam_device_error": [i32],
+        "wam_video_prefill_kv_fuse_noalloc": [lay, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp,
+                                              i32, f32, i32, i32, vp, vp, vp],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -81,7 +84,8 @@ def exported_names() -> list:
     """Names of the C entry points this binding declares (all must be exported)."""
     return ["wam_video_prefill_kv", "wam_fuse_interval_kv", "wam_action_attn",
             "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
-            "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version"]
+            "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
+            "wam_video_prefill_kv_fuse_noalloc"]
 
 
 def check(status: int) -> None:
@@ -151,6 +155,21 @@ def video_prefill_kv(layout: VideoLayout, f_begin: int, f_end: int, q, k_new, v_
                                    _ptr(v_new), _ptr(k_cache), _ptr(v_cache), int(store_kv),
                                    _ptr(o), _dtype(o), None if fuse is None else fuse.ref,
                                    _stream(stream)))
+
+
+NOALLOC_FUSE_ACC_ELEMS = 4 * 1024 * 1024
+
+
+def video_prefill_kv_fuse_noalloc(layout: VideoLayout, f_begin: int, f_end: int, q, k_new, v_new,
+                                  k_cache, v_cache, o, weight: float, first: bool, last: bool,
+                                  fused_k=None, fused_v=None, store_kv: bool = True,
+                                  stream=None) -> None:
+    """The prefill with the fusion epilogue whose fp32 accumulator lives inside the library
+    (for callers that cannot allocate device memory); B*F*T*H*D <= NOALLOC_FUSE_ACC_ELEMS."""
+    check(lib.wam_video_prefill_kv_fuse_noalloc(
+        layout.ref, _dtype(q), f_begin, f_end, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+        _ptr(v_cache), int(store_kv), _ptr(o), _dtype(o), float(weight), int(first), int(last),
+        _ptr(fused_k), _ptr(fused_v), _stream(stream)))
 
 
 def fuse_interval_kv(layout: VideoLayout, k_layers, v_layers, weights, f_begin: int,

@@ -164,6 +164,37 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt,
 wam_status wam_flow_euler_step(int64_t n, float* x, const float* v, float dsigma,
                                wam_stream_t stream);
 
+/*
+ * wam_video_prefill_kv with the fusion epilogue, for callers that cannot allocate device memory
+ * (no counterpart on the pages: it is a deployment convenience of this library).
+ *
+ * The epilogue's fp32 accumulator normally comes from the caller (wam_fuse_epilogue.acc_k /
+ * acc_v).  Code that runs while a CUDA graph is being captured, plug-ins that get a fixed
+ * memory pool from their host, or runtimes that allocate everything up front cannot call
+ * cudaMalloc for it.  This entry point keeps the accumulator in a device array inside the
+ * library instead; the caller passes only inputs and outputs.  Arguments are those of
+ * wam_video_prefill_kv, with the epilogue given as weight / first / last / fused_k / fused_v.
+ *   - Limit: B * F * T * H * D <= WAM_NOALLOC_FUSE_ACC_ELEMS (about 4.2 million elements, for
+ *     K and for V); larger layouts return WAM_ERR_UNSUPPORTED and launch nothing.  The array
+ *     (2 x 16 MiB) is held on every GPU that loads the library until the process exits.
+ *   - The first call on a device looks the array's address up (cudaGetSymbolAddress): make
+ *     that first call before any stream capture.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - Every call shares the one array, which keeps what the last call left in it: a middle or
+ *     last call of an interval reads what the previous call of that interval accumulated, and
+ *     a first call overwrites it (nothing has to start at zero).  Calls that overlap on the
+ *     GPU (other streams, other threads) race on it; keep them ordered.
+ */
+#define WAM_NOALLOC_FUSE_ACC_ELEMS (4 * 1024 * 1024)
+wam_status wam_video_prefill_kv_fuse_noalloc(const wam_video_layout* layout, wam_dtype dt,
+                                             int32_t f_begin, int32_t f_end,
+                                             const void* q, const void* k_new, const void* v_new,
+                                             void* k_cache, void* v_cache, int32_t store_kv,
+                                             void* o, wam_dtype o_dt,
+                                             float weight, int32_t first_in_interval,
+                                             int32_t last_in_interval,
+                                             void* fused_k, void* fused_v, wam_stream_t stream);
+
 /* ---- host helpers (no GPU work) ---------------------------------------------------------- */
 
 /*

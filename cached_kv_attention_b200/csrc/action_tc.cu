@@ -142,7 +142,7 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
     for (int j = 0; j < 16; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     uint32_t qf[8][4];
-    if (!mbar_wait(sm.qbar, 0)) bad = true;
+    bad = !__all_sync(0xffffffffu, mbar_wait(sm.qbar, 0));  // warp-uniform before collectives
     if (!bad) {
       const uint32_t qbase = smem_u32(sm.q);
 #pragma unroll
@@ -153,7 +153,7 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
     const float c = a.scale_log2;
     for (int i = 0; i < n_tiles && !bad; ++i) {
       const int st = i % kStages;
-      if (!mbar_wait(&sm.full[st], (i / kStages) & 1)) { bad = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[st], (i / kStages) & 1))) { bad = true; break; }
       const uint32_t kb = smem_u32(sm.k[st]), vb = smem_u32(sm.v[st]);
       // S = Q K^T for this warp's 16 rows x 32 keys
       float s[4][4];
@@ -261,10 +261,14 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
       sm.lbuf[kh * 32 + r0] = l0, sm.lbuf[kh * 32 + r1] = l1;
     }
   }
-  if (warp == kConsumers) asm volatile("bar.sync 1, %0;" ::"n"(kThreads));
+  if (warp == kConsumers) {
+    __syncwarp();  // lane 0 ran the producer loop alone
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads));
+  }
   if (bad && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
 
   // ------------------------------------------------------------------ cluster merge
+  __syncwarp();
   cluster.sync();
   const int P = 2 * C;  // partials per (b, h)
   if (threadIdx.x < 32) {

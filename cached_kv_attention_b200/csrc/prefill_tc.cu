@@ -1,30 +1,34 @@
 // Block-causal video prefill on the sm_100a tensor cores (tcgen05.mma, TMEM accumulators,
 // TMA-fed shared memory); bf16 inputs, D = 128, T % 128 == 0.
 //
-// One CTA computes 128 query tokens of one (episode, frame, head) against every key tile the
-// block-causal predicate allows ("Long-WAM: Scaling the Context of World-Action Models |
-// Summary" §3.1-3.2).  T is a multiple of 128, so every 128 x 128 tile is wholly visible or
-// wholly masked: the host work list holds only the visible key frames and no element mask is
-// applied.  Keys of frames below f_begin come from the layer's cache, the others from the
-// call's new K/V.
+// One CTA computes up to 256 query tokens (two 128-row tiles Q0, Q1) of one (episode, frame,
+// head) against every key tile the block-causal predicate allows ("Long-WAM: Scaling the
+// Context of World-Action Models | Summary" §3.1-3.2).  T is a multiple of 128, so every
+// 128 x 128 tile is wholly visible or wholly masked: the host work list holds only visible key
+// frames and no element mask is applied.  Keys of frames below f_begin come from the layer's
+// cache, the others from the call's new K/V.  Each K/V tile loaded feeds both query tiles.
 //
-// Per key tile j (128 keys):   S_j = Q K_j^T          tcgen05.mma -> TMEM (two S buffers)
-//                              P_j = exp2(S_j c - m)   softmax warps, bf16 -> shared memory
-//                              O  += P_j V_j           tcgen05.mma -> TMEM (one O buffer)
-// The MMA thread issues S_{j+1} before P_j V_j, so the tensor core computes the next scores
-// while the softmax warps work on the current ones.  The reference max m of a row only moves
-// when a tile raises the row max by more than 8 (a factor 2^8); O and l are then rescaled in
-// TMEM, which needs P_{j-1} V_{j-1} to have landed.  Otherwise p stays below 2^8 and nothing
-// is rescaled (exact arithmetic either way: numerator and denominator share the reference).
+// For query tile w and key tile j (128 keys):
+//   S_w = Q_w K_j^T           tcgen05.mma, A and B from shared memory -> TMEM
+//   P_w = exp2(S_w c - m_w)   softmax warpgroup w; bf16 P written back over S_w in TMEM
+//   O_w += P_w V_j            tcgen05.mma, A from TMEM, B (V, MN-major) from shared memory
+// The MMA thread alternates the two tiles (P_0 V, next S_0, P_1 V, next S_1, ...), so the
+// tensor core works on one tile while the other tile's warpgroup runs its softmax.  A row's
+// reference max m_w only moves when a key tile raises the row max by more than 8 (a factor
+// 2^8); O_w is then rescaled in TMEM.  S_w of key tile j is issued after P_w V_{j-1}, so its
+// completion implies O_w is complete up to j-1 and the rescale needs no extra wait.  The
+// numerator and denominator share the reference, so the result is exact either way.
 //
-// While the CTA's own 128 tokens of K/V are resident, two helper warps store them into the
-// layer's cache and fold them into the Interval KV-Fusion accumulator ("世界模型之Faster-WAM
-// 详解" §3.3), so the per-layer K/V is never re-read for fusion.
+// While the CTA's own K/V tiles (the key tokens equal to its query tokens) are resident, two
+// helper warps store them into the layer's cache and fold them into the Interval KV-Fusion
+// accumulator ("世界模型之Faster-WAM详解" §3.3): the per-layer K/V is never re-read for fusion.
+// The own tiles come last in the key order, so the stages they hold are not needed afterwards.
 //
-// Warps: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-3 cache store and fusion |
-//        4-7 softmax (thread = query row; warp w reads TMEM lanes 32 (w % 4) ..).
-// Every mbarrier wait is bounded; a wait that gives up raises a CTA-wide abort flag, every
-// role drains what it started, TMEM is freed and the device error word is set.
+// Warps: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-3 cache store + fusion |
+//        4-7 softmax of Q0, 8-11 softmax of Q1 (thread = query row; warp w reads TMEM lanes
+//        32 (w % 4) ..).  Every mbarrier wait is bounded; a wait that gives up raises a
+//        CTA-wide abort flag, every role drains what it started, TMEM is freed and the
+//        device error word is set.
 #include "launch.h"
 #include "tcgen05.cuh"
 
@@ -32,10 +36,11 @@ namespace wam {
 namespace {
 
 constexpr int kBM = 128, kBN = 128;
-constexpr int kThreads = 256;
-constexpr int kTile = 128 * 128 * 2;  // one Q, K, V or P tile: two 64-column swizzled halves
+constexpr int kThreads = 384;
+constexpr int kTile = 128 * 128 * 2;  // one Q, K or V tile: two 64-column swizzled halves
 constexpr int kHalf = kTile / 2;
-constexpr uint32_t kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,384)
+constexpr int kKStages = 3, kVStages = 2;
+constexpr uint32_t kTmemCols = 512;   // query tile w: S/P at 256 w, O at 256 w + 128
 constexpr float kRescaleLog2 = 8.f;
 
 struct PrefillMaps {
@@ -44,14 +49,15 @@ struct PrefillMaps {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_free[2], p_full[2], p_empty[2];
-  uint64_t o_full, done;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t done;
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr int kSmemBytes = 1024 + 7 * kTile + int(sizeof(Bars)) + 64;
+constexpr int kSmemBytes = 1024 + (2 + kKStages + kVStages) * kTile + int(sizeof(Bars)) + 64;
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
   for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
@@ -111,50 +117,91 @@ __device__ __forceinline__ void store_fuse_tile128(const PrefillArgs& a, const u
   }
 }
 
-// Pulls the accumulator rows of the CTA's own 128 tokens into L2 ahead of the fold (64 threads).
-__device__ __forceinline__ void prefetch_acc_rows(const PrefillArgs& a, const float* acc, int64_t row0,
-                                                  int h, int t) {
-  for (int r = t; r < kBN; r += 64) {
+// Pulls accumulator rows into L2 ahead of the fold (64 threads, 512 B per row).
+__device__ __forceinline__ void prefetch_acc_rows(const PrefillArgs& a, const float* acc,
+                                                  int64_t row0, int rows, int h, int t) {
+  for (int r = t; r < rows; r += 64) {
     const float* p = acc + ((row0 + r) * a.H + h) * 128;
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], 512;" ::"l"(p) : "memory");
   }
+}
+
+// tcgen05.mma with A from tensor memory: D[tmem] (+)= A[tmem] * B[smem desc]^T.  A 16-bit A
+// operand keeps row m in TMEM lane m and elements 2i, 2i+1 of its K dimension in the low and
+// high half of column i.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = base;
-  uint8_t* sK[2] = {base + kTile, base + 2 * kTile};
-  uint8_t* sV[2] = {base + 3 * kTile, base + 4 * kTile};
-  uint8_t* sP[2] = {base + 5 * kTile, base + 6 * kTile};
-  Bars& bars = *reinterpret_cast<Bars*>(base + 7 * kTile);
+  uint8_t* sQ[2] = {base, base + kTile};
+  uint8_t* sK[kKStages];
+  uint8_t* sV[kVStages];
+  for (int i = 0; i < kKStages; ++i) sK[i] = base + (2 + i) * kTile;
+  for (int i = 0; i < kVStages; ++i) sV[i] = base + (2 + kKStages + i) * kTile;
+  Bars& bars = *reinterpret_cast<Bars*>(base + (2 + kKStages + kVStages) * kTile);
   volatile int* abort = &bars.abort;
 
-  const int QT = a.T / kBM;
+  // ---- work item: query tiles 2 qp and 2 qp + 1 of frame f (the second may not exist)
+  const int QT = a.T / kBM, QP = (QT + 1) / 2;
   const int h = int(blockIdx.x % a.H);
   const int rest = int(blockIdx.x / a.H);
-  const int qt = rest % QT;
-  const uint32_t it = a.fl.item[rest / QT];
+  const int qp = rest % QP;
+  const uint32_t it = a.fl.item[rest / QP];
   const int b = item_b(it), f = item_f(it), nk = item_nk(it);
+  const int nq = (2 * qp + 1 < QT) ? 2 : 1;            // query tiles in this CTA
   const int tpf = a.T / kBN;
-  const int n = nk * tpf;                              // key tiles
-  const int qtok0 = (f - a.f_begin) * a.T + qt * kBM;  // first query row of the call
+  const int n = nk * tpf;                               // key tiles
+  const int qtok0 = (f - a.f_begin) * a.T + qp * 2 * kBM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Key order: the visible tiles in list order with the CTA's own tiles (a contiguous block
+  // [own0, own0 + nq) of the list) moved to the end.
+  int own_u = nk - 1;
+  for (int u = 0; u < nk; ++u)
+    if (a.fl.vlist[b * a.F + u] == f) own_u = u;
+  const int own0 = own_u * tpf + 2 * qp;
+  auto key_tile = [&](int j, bool& old, int& tok, int& fk, int& jj) {
+    const int jm = j < n - nq ? (j < own0 ? j : j + nq) : own0 + (j - (n - nq));
+    fk = a.fl.vlist[b * a.F + jm / tpf];
+    jj = jm % tpf;
+    old = fk < a.f_begin;
+    tok = (old ? fk : fk - a.f_begin) * a.T + jj * kBN;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.v_full[s], 1);
       mbar_init(&bars.k_empty[s], 2);  // MMA completion + store warps
-      mbar_init(&bars.v_empty[s], 2);
-      mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_free[s], 4);
-      mbar_init(&bars.p_full[s], 4);
-      mbar_init(&bars.p_empty[s], 1);
     }
-    mbar_init(&bars.o_full, 1);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.v_empty[s], 2);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars.s_full[w], 1);
+      mbar_init(&bars.p_full[w], 4);
+      mbar_init(&bars.o_full[w], 1);
+    }
     mbar_init(&bars.done, 1);
     bars.abort = 0;
     fence_barrier_init();
@@ -167,57 +214,39 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = bars.tmem_base;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
-
-  // Key tiles in list order, except that the CTA's own tile (its own 128 tokens) is swapped to
-  // the end: the store warps then hold its K/V stage while no later tile needs that stage.
-  int own_u = nk - 1;  // position of the query frame among the visible frames
-  for (int u = 0; u < nk; ++u)
-    if (a.fl.vlist[b * a.F + u] == f) own_u = u;
-  const int own_j = own_u * tpf + qt;
-  auto key_tile = [&](int j, bool& old, int& tok, int& fk, int& jj) {
-    const int jm = j == n - 1 ? own_j : (j == own_j ? n - 1 : j);
-    fk = a.fl.vlist[b * a.F + jm / tpf];
-    jj = jm % tpf;
-    old = fk < a.f_begin;
-    tok = (old ? fk : fk - a.f_begin) * a.T + jj * kBN;
-  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(&bars.q_full, kTile);
-      tma_load_4d(sQ, &maps.q, &bars.q_full, 0, h, qtok0, b);
-      tma_load_4d(sQ + kHalf, &maps.q, &bars.q_full, 64, h, qtok0, b);
+      int k_issued = 0, v_issued = 0;
+      mbar_arrive_expect_tx(&bars.q_full, nq * kTile);
+      for (int w = 0; w < nq; ++w) {
+        tma_load_4d(sQ[w], &maps.q, &bars.q_full, 0, h, qtok0 + w * kBM, b);
+        tma_load_4d(sQ[w] + kHalf, &maps.q, &bars.q_full, 64, h, qtok0 + w * kBM, b);
+      }
       for (int j = 0; j < n; ++j) {
-        const int s = j & 1;
         bool old;
         int tok, fk, jj;
         key_tile(j, old, tok, fk, jj);
+        const int ks = j % kKStages, vs = j % kVStages;
+        if (j >= kKStages && !wait_bar(&bars.k_empty[ks], ((j / kKStages) - 1) & 1, abort)) break;
         const CUtensorMap* mk = old ? &maps.kc : &maps.kn;
+        mbar_arrive_expect_tx(&bars.k_full[ks], kTile);
+        tma_load_4d(sK[ks], mk, &bars.k_full[ks], 0, h, tok, b);
+        tma_load_4d(sK[ks] + kHalf, mk, &bars.k_full[ks], 64, h, tok, b);
+        k_issued = j + 1;
+        if (j >= kVStages && !wait_bar(&bars.v_empty[vs], ((j / kVStages) - 1) & 1, abort)) break;
         const CUtensorMap* mv = old ? &maps.vc : &maps.vn;
-        if (j >= 2 && !wait_bar(&bars.k_empty[s], ((j >> 1) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bars.k_full[s], kTile);
-        tma_load_4d(sK[s], mk, &bars.k_full[s], 0, h, tok, b);
-        tma_load_4d(sK[s] + kHalf, mk, &bars.k_full[s], 64, h, tok, b);
-        if (j >= 2 && !wait_bar(&bars.v_empty[s], ((j >> 1) - 1) & 1, abort)) {
-          issued = -(j + 1);  // K_j issued, V_j not
-          break;
-        }
-        mbar_arrive_expect_tx(&bars.v_full[s], kTile);
-        tma_load_4d(sV[s], mv, &bars.v_full[s], 0, h, tok, b);
-        tma_load_4d(sV[s] + kHalf, mv, &bars.v_full[s], 64, h, tok, b);
-        issued = j + 1;
+        mbar_arrive_expect_tx(&bars.v_full[vs], kTile);
+        tma_load_4d(sV[vs], mv, &bars.v_full[vs], 0, h, tok, b);
+        tma_load_4d(sV[vs] + kHalf, mv, &bars.v_full[vs], 64, h, tok, b);
+        v_issued = j + 1;
       }
       // Drain: loads issued must land before the CTA leaves (matters only after an abort).
-      const int nk_issued = issued < 0 ? -issued : issued;
-      const int nv_issued = issued < 0 ? -issued - 1 : issued;
-      for (int j = (nk_issued > 2 ? nk_issued - 2 : 0); j < nk_issued; ++j)
-        mbar_wait(&bars.k_full[j & 1], (j >> 1) & 1);
-      for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
-        mbar_wait(&bars.v_full[j & 1], (j >> 1) & 1);
+      for (int j = (k_issued > kKStages ? k_issued - kKStages : 0); j < k_issued; ++j)
+        mbar_wait(&bars.k_full[j % kKStages], (j / kKStages) & 1);
+      for (int j = (v_issued > kVStages ? v_issued - kVStages : 0); j < v_issued; ++j)
+        mbar_wait(&bars.v_full[j % kVStages], (j / kVStages) & 1);
       mbar_wait(&bars.q_full, 0);
     }
   } else if (warp == 1) {
@@ -225,41 +254,50 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     if (lane == 0) {
       const uint32_t idS = tc05::idesc_bf16_f32(128, 128, false);
       const uint32_t idO = tc05::idesc_bf16_f32(128, 128, true);
-      const uint32_t q_s = smem_u32(sQ);
-      bool ok = wait_bar(&bars.q_full, 0, abort);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int s = j & 1;
-          if (!wait_bar(&bars.k_full[s], (j >> 1) & 1, abort)) break;
-          if (j >= 2 && !wait_bar(&bars.s_free[s], ((j >> 1) - 1) & 1, abort)) break;
-          tc05::fence_after_sync();
-          const uint32_t k_s = smem_u32(sK[s]);
+      const uint32_t tS[2] = {tmem, tmem + 256}, tO[2] = {tmem + 128, tmem + 384};
+      auto issue_S = [&](int w, int j) {
+        const uint32_t q_s = smem_u32(sQ[w]), k_s = smem_u32(sK[j % kKStages]);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            tc05::mma_ss(tS[s], tc05::smem_desc_sw128(q_s + off, 16, 1024),
-                         tc05::smem_desc_sw128(k_s + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-          }
-          tc05::mma_commit(&bars.k_empty[s]);
-          tc05::mma_commit(&bars.s_full[s]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          tc05::mma_ss(tS[w], tc05::smem_desc_sw128(q_s + off, 16, 1024),
+                       tc05::smem_desc_sw128(k_s + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jp = j - 1, sp = jp & 1;
-          if (!wait_bar(&bars.v_full[sp], (jp >> 1) & 1, abort)) break;
-          if (!wait_bar(&bars.p_full[sp], (jp >> 1) & 1, abort)) break;
-          tc05::fence_after_sync();
-          const uint32_t p_s = smem_u32(sP[sp]), v_s = smem_u32(sV[sp]);
+      };
+      auto issue_PV = [&](int w, int j) {
+        const uint32_t v_s = smem_u32(sV[j % kVStages]);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t poff = (kk >> 2) * kHalf + (kk & 3) * 32;
-            tc05::mma_ss(tO, tc05::smem_desc_sw128(p_s + poff, 16, 1024),
-                         tc05::smem_desc_sw128(v_s + kk * 2048, kHalf, 1024), idO,
-                         (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc05::mma_commit(&bars.v_empty[sp]);
-          tc05::mma_commit(&bars.p_empty[sp]);
-          if (jp == n - 1) tc05::mma_commit(&bars.o_full);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tO[w], tS[w] + 8 * kk, tc05::smem_desc_sw128(v_s + kk * 2048, kHalf, 1024), idO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bar(&bars.q_full, 0, abort) && wait_bar(&bars.k_full[0], 0, abort);
+      if (ok) {
+        tc05::fence_after_sync();
+        for (int w = 0; w < nq; ++w) {
+          issue_S(w, 0);
+          tc05::mma_commit(&bars.s_full[w]);
         }
+        tc05::mma_commit(&bars.k_empty[0]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const bool more = j + 1 < n;
+        if (!wait_bar(&bars.v_full[j % kVStages], (j / kVStages) & 1, abort)) break;
+        if (more && !wait_bar(&bars.k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, abort)) break;
+        bool fail = false;
+        for (int w = 0; w < nq; ++w) {
+          if (!wait_bar(&bars.p_full[w], j & 1, abort)) { fail = true; break; }
+          tc05::fence_after_sync();
+          issue_PV(w, j);
+          if (j == n - 1) tc05::mma_commit(&bars.o_full[w]);
+          if (more) {
+            issue_S(w, j + 1);
+            tc05::mma_commit(&bars.s_full[w]);
+          }
+        }
+        if (fail) break;
+        tc05::mma_commit(&bars.v_empty[j % kVStages]);
+        if (more) tc05::mma_commit(&bars.k_empty[(j + 1) % kKStages]);
       }
       tc05::mma_commit(&bars.done);  // arrives once every MMA issued above has completed
     }
@@ -269,149 +307,137 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     const int t = threadIdx.x - 64;
     const bool do_store = a.k_store != nullptr || a.fuse_on;
     const int64_t N = int64_t(a.F) * a.T;
+    const int64_t own_row0 = int64_t(b) * N + int64_t(f) * a.T + qp * 2 * kBN;
     if (a.fuse_on && !a.fuse_first) {
-      const int64_t own_row0 = int64_t(b) * N + int64_t(f) * a.T + qt * kBN;
-      prefetch_acc_rows(a, a.acc_k, own_row0, h, t);
-      prefetch_acc_rows(a, a.acc_v, own_row0, h, t);
+      prefetch_acc_rows(a, a.acc_k, own_row0, nq * kBN, h, t);
+      prefetch_acc_rows(a, a.acc_v, own_row0, nq * kBN, h, t);
     }
     for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
+      const int ks = j % kKStages, vs = j % kVStages;
       bool old;
       int tok, fk, jj;
       key_tile(j, old, tok, fk, jj);
-      const bool own = do_store && fk == f && jj == qt;
+      const bool own = do_store && fk == f && (jj >> 1) == qp;
       const int64_t row0 = int64_t(b) * N + int64_t(f) * a.T + jj * kBN;
-      const bool okk = wait_bar(&bars.k_full[s], (j >> 1) & 1, abort);
-      if (okk && own) store_fuse_tile128(a, sK[s], a.k_store, a.acc_k, a.fused_k, row0, h, t);
+      const bool okk = wait_bar(&bars.k_full[ks], (j / kKStages) & 1, abort);
+      if (okk && own) store_fuse_tile128(a, sK[ks], a.k_store, a.acc_k, a.fused_k, row0, h, t);
       asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (t == 0 && okk) mbar_arrive(&bars.k_empty[s]);
-      const bool okv = wait_bar(&bars.v_full[s], (j >> 1) & 1, abort);
-      if (okv && own) store_fuse_tile128(a, sV[s], a.v_store, a.acc_v, a.fused_v, row0, h, t);
+      if (t == 0 && okk) mbar_arrive(&bars.k_empty[ks]);
+      const bool okv = wait_bar(&bars.v_full[vs], (j / kVStages) & 1, abort);
+      if (okv && own) store_fuse_tile128(a, sV[vs], a.v_store, a.acc_v, a.fused_v, row0, h, t);
       asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (t == 0 && okv) mbar_arrive(&bars.v_empty[s]);
+      if (t == 0 && okv) mbar_arrive(&bars.v_empty[vs]);
     }
   } else {
     // ------------------------------------------------------------ softmax, one row per thread
     // tcgen05.ld / tcgen05.st are warp-collective: every decision in front of one is voted
     // across the warp, so all 32 lanes always execute them together.
     const unsigned FULL = 0xffffffffu;
-    const int r = 32 * (warp & 3) + lane;
-    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    const float c = a.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
-      ok = __all_sync(FULL, ok && wait_bar(&bars.s_full[s], (j >> 1) & 1, abort));
-      if (!ok) continue;
-      tc05::fence_after_sync();
-      uint32_t x[4][32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tc05::tmem_ld32(tS[s] + lane_off + 32 * q, x[q]);
-      tc05::tmem_wait_ld();
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[s]);
-      // row max and row sum over 8 independent accumulators (short dependency chains)
-      float mx8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(x[q][i]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_cand = mx * c;
-      bool rescale = false;
-      float alpha = 1.f;
-      if (j == 0) {
-        m_ref = m_cand;
-      } else if (m_cand > m_ref + kRescaleLog2) {
-        alpha = exp2f(m_ref - m_cand);
-        l *= alpha;
-        m_ref = m_cand;
-        rescale = true;
-      }
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p = tc05::fast_exp2(fmaf(__uint_as_float(x[q][i]), c, -m_ref));
-          sum8[i & 7] += p;
-          x[q][i] = __float_as_uint(p);
-        }
-      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      // P buffer s is free once P_{j-2} V_{j-2} has completed
-      if (j >= 2) {
-        ok = __all_sync(FULL, wait_bar(&bars.p_empty[s], ((j >> 1) - 1) & 1, abort));
-        if (!ok) continue;
-      }
-      uint8_t* prow = sP[s] + r * 128;
-#pragma unroll
-      for (int cch = 0; cch < 16; ++cch) {
-        const int q = cch >> 2, i0 = (cch & 3) * 8;
-        uint4 u;
-        u.x = pack_bf16(__uint_as_float(x[q][i0 + 0]), __uint_as_float(x[q][i0 + 1]));
-        u.y = pack_bf16(__uint_as_float(x[q][i0 + 2]), __uint_as_float(x[q][i0 + 3]));
-        u.z = pack_bf16(__uint_as_float(x[q][i0 + 4]), __uint_as_float(x[q][i0 + 5]));
-        u.w = pack_bf16(__uint_as_float(x[q][i0 + 6]), __uint_as_float(x[q][i0 + 7]));
-        const int half = cch >> 3, chunk = cch & 7;
-        *reinterpret_cast<uint4*>(prow + half * kHalf + ((chunk ^ (r & 7)) << 4)) = u;
-      }
-      if (__any_sync(FULL, rescale)) {
-        // O holds P_{<j} V_{<j} once P_{j-1} V_{j-1} has landed; rows that keep their
-        // reference scale by 1 (exact), so the whole warp runs the TMEM round trip.
-        const int jp = j - 1;
-        ok = __all_sync(FULL, wait_bar(&bars.p_empty[jp & 1], (jp >> 1) & 1, abort));
+    const int w = (warp - 4) >> 2;  // query tile of this warpgroup
+    if (w < nq) {
+      const int r = 32 * (warp & 3) + lane;
+      const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
+      const uint32_t tS = tmem + 256 * w + lane_off, tO = tmem + 256 * w + 128 + lane_off;
+      const float c = a.scale_log2;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(FULL, ok && wait_bar(&bars.s_full[w], j & 1, abort));
         if (!ok) continue;
         tc05::fence_after_sync();
+        // pass 1: row max of S over the 128 keys
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t x[32];
+          tc05::tmem_ld32(tS + 32 * q, x);
+          tc05::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(x[i]));
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_cand = mx * c;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_ref = m_cand;
+        } else if (m_cand > m_ref + kRescaleLog2) {
+          alpha = tc05::fast_exp2(m_ref - m_cand);
+          l *= alpha;
+          m_ref = m_cand;
+          rescale = true;
+        }
+        // O_w holds P V of key tiles < j (S_w of tile j was issued after P_w V_{j-1}); rows
+        // that keep their reference scale by 1 (exact), so the whole warp runs the round trip.
+        if (__any_sync(FULL, rescale)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tc05::tmem_ld32(tO + 32 * q, o);
+            tc05::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tc05::tmem_st32(tO + 32 * q, o);
+          }
+        }
+        // pass 2: P = exp2(S c - m_ref) as bf16 pairs over the first 64 columns of S (chunk q
+        // writes columns [16 q, 16 q + 16), all of which it or an earlier chunk already read)
+        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t x[32];
+          tc05::tmem_ld32(tS + 32 * q, x);
+          tc05::tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = tc05::fast_exp2(fmaf(__uint_as_float(x[2 * i]), c, -m_ref));
+            const float p1 = tc05::fast_exp2(fmaf(__uint_as_float(x[2 * i + 1]), c, -m_ref));
+            sum8[(2 * i) & 7] += p0;
+            sum8[(2 * i + 1) & 7] += p1;
+            pk[i] = pack_bf16(p0, p1);  // key 2i in the low half
+          }
+          tmem_st16(tS + 16 * q, pk);
+        }
+        l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        tc05::tmem_wait_st();
+        tc05::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[w]);
+      }
+      // epilogue: O / l to global memory
+      ok = __all_sync(FULL, ok && wait_bar(&bars.o_full[w], 0, abort));
+      if (ok) {
+        tc05::fence_after_sync();
+        const float inv = 1.f / l;
+        const int64_t qtok = int64_t(a.f_end - a.f_begin) * a.T;
+        const int64_t row = int64_t(b) * qtok + qtok0 + w * kBM + r;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
-          tc05::tmem_ld32(tO + lane_off + 32 * q, o);
+          tc05::tmem_ld32(tO + 32 * q, o);
           tc05::tmem_wait_ld();
+          const int64_t off = (row * a.H + h) * 128 + 32 * q;
+          if (a.o_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tc05::tmem_st32(tO + lane_off + 32 * q, o);
-        }
-        tc05::tmem_wait_st();
-      }
-      tc05::fence_proxy_async_smem();
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full[s]);
-    }
-    // epilogue: O / l to global memory
-    ok = __all_sync(FULL, ok && wait_bar(&bars.o_full, 0, abort));
-    if (ok) {
-      tc05::fence_after_sync();
-      const float inv = 1.f / l;
-      const int64_t qtok = int64_t(a.f_end - a.f_begin) * a.T;
-      const int64_t row = int64_t(b) * qtok + qtok0 + r;
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tc05::tmem_ld32(tO + lane_off + 32 * q, o);
-        tc05::tmem_wait_ld();
-        const int64_t off = (row * a.H + h) * 128 + 32 * q;
-        if (a.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                 __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-            u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-            u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-            u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-            dst[i] = u;
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+              u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+              u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+              u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+              dst[i] = u;
+            }
           }
         }
       }
@@ -455,7 +481,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured |= 1u << dev;
   }
-  const int64_t grid = int64_t(a.fl.n_items) * (a.T / kBM) * a.H;
+  const int QP = (a.T / kBM + 1) / 2;
+  const int64_t grid = int64_t(a.fl.n_items) * QP * a.H;
   prefill_tc_kernel<<<unsigned(grid), kThreads, kSmemBytes, s>>>(a, maps);
   return cudaGetLastError();
 }

@@ -120,6 +120,8 @@ class ChunkRunner:
         self.sig_a = wam.flow_schedule(w.n_euler_steps, 0.0)
         self.parts = interval_partition(w.L, w.S)
         self.fw = [wam.fuse_weights(lg.cpu().numpy()) for lg in inputs["fuse_logits"]]
+        ws_bytes = wam.action_attn_workspace_size(self.layout, dt, w.n_act, True)
+        self.workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         self.calls: List = []
         self._keep: List = []
 
@@ -192,7 +194,8 @@ class ChunkRunner:
                 calls.append((L.wam_action_attn,
                               (lay, dt, fk, fv, w.n_act, _vp(inp["act_q"][i][l]),
                                _vp(inp["act_k"][i][l]), _vp(inp["act_v"][i][l]),
-                               o_of(self.act_o, i * w.L + l), o_dt, s)))
+                               o_of(self.act_o, i * w.L + l), o_dt, _vp(self.workspace),
+                               self.workspace.numel(), s)))
             ds = float(self.sig_a[i + 1] - self.sig_a[i])
             calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
         self.calls = calls

@@ -5,97 +5,151 @@
 // moves 512 B (K and V, bf16) and does 32 x 4 x 128 FLOP, 32 FLOP/B, above what the fp32
 // pipes can issue at full HBM bandwidth, so the contractions run on mma.sync tensor-core
 // tiles (M = 32 queries) while the loads stream through TMA: Q K^T on bf16 tiles, P V on tf32
-// tiles (the fused cache is already rounded to bf16 once, so P is kept at 10 mantissa bits
-// to leave the error budget to the storage rounding).
+// tiles (the fused cache is already rounded to bf16 once, so P keeps 10 mantissa bits to
+// leave the error budget to the storage rounding).
 //
-// Grid = (C splits, H, B), launched as clusters of C CTAs.  Split c of (b, h) reads a
-// contiguous run of 64-key tiles of the episode's valid frames; split 0 also reads the
-// action tile.  Each CTA keeps an fp32 online-softmax partial per key half; the 2C partials
-// of a (b, h) are merged through distributed shared memory, so no workspace is needed.
+// Work split (persistent, balanced): the call's tiles are laid out as, for every (episode b,
+// head h), one action tile (the n_act action keys, zero-padded to 64 and masked) followed by
+// the 64-key tiles of b's valid frames.  The G tiles are cut into P equal runs, one per CTA
+// (P = SM count), so every CTA streams the same amount whatever the padding.  A CTA keeps one
+// online-softmax state per (b, h) run it touches; a (b, h) contained in one CTA writes O
+// directly, otherwise each CTA writes its partial (O, m, l) into the workspace and the last
+// to arrive (atomic ticket) merges all partials by their log-sum-exp and resets the ticket.
 //
-// Warp roles: warps 0-3 consume (warp w: query rows 16*(w&1).., keys 32*(w>>1).. of each
-// tile), warp 4 lane 0 issues the TMA loads.  3-stage K/V ring with full/empty mbarriers.
-#include <cooperative_groups.h>
-
+// Tiles hold 128 keys when T % 128 == 0 (2-stage K/V ring), else 64 (4 stages).  Warps 0-7
+// consume (warp w: query rows 16 (w & 1) .., keys (w >> 1) * tile / 4 .. of each tile), warp
+// 8 lane 0 issues TMA loads into the ring and a 2-slot Q buffer.
 #include "launch.h"
-
-namespace cg = cooperative_groups;
 
 namespace wam {
 namespace {
 
-constexpr int kBN = 64;          // keys per tile
-constexpr int kStages = 3;
-constexpr int kConsumers = 4;    // consumer warps
+constexpr int kRingBytes = 128 * 1024;    // K/V ring: 2 stages of 128 keys or 4 of 64
+constexpr int kConsumers = 8;
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kQBytes = 32 * 128 * 2;
-constexpr int kTileBytes = kBN * 128 * 2;   // one of K or V
 constexpr int kOStride = 132;               // fp32 row stride of the merge buffers
-constexpr int kSmemBytes = 1024 + kQBytes + kStages * 2 * kTileBytes + 256;
+constexpr int kSlotFloats = 32 * 128 + 64;  // one workspace partial: O [32][128], m [32], l [32]
+constexpr int kMergeBytes = 4 * 32 * kOStride * 4 + 2 * 4 * 32 * 4;
+constexpr int kSmemBytes = 1024 + 2 * kQBytes + kRingBytes + kMergeBytes + 256;
+constexpr int kMaxStages = 4;
+constexpr float kLazyLog2 = 8.f;  // headroom of a row's softmax reference (log2 units)
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 struct ActionMaps {
   CUtensorMap q, ka, va, fk, fv;
 };
 
-struct SmemLayout {
-  uint8_t* q;
-  uint8_t* k[kStages];
-  uint8_t* v[kStages];
-  uint64_t* full;
-  uint64_t* empty;
-  uint64_t* qbar;
-  // merge area (aliases the K/V ring once every load has landed)
-  float* obuf;    // [2][32][kOStride]
-  float* mbuf;    // [2][32]
-  float* lbuf;    // [2][32]
-  float* fbuf;    // [32][2 * 16]
+struct Bars {
+  uint64_t full[kMaxStages], empty[kMaxStages];
+  uint64_t qfull[2], qempty[2];
+  int last;  // merge flag of the current run
 };
 
-__device__ __forceinline__ SmemLayout carve(uint8_t* raw) {
-  SmemLayout s;
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-  s.q = base;
-  uint8_t* p = base + kQBytes;
-  for (int i = 0; i < kStages; ++i) {
-    s.k[i] = p;
-    s.v[i] = p + kTileBytes;
-    p += 2 * kTileBytes;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(p);
-  s.full = bars;
-  s.empty = bars + kStages;
-  s.qbar = bars + 2 * kStages;
-  float* m = reinterpret_cast<float*>(base + kQBytes);
-  s.obuf = m;
-  s.mbuf = m + 2 * 32 * kOStride;
-  s.lbuf = s.mbuf + 64;
-  s.fbuf = s.lbuf + 64;
-  return s;
+template <int kBN>
+__device__ __forceinline__ int tiles_of(const ActionArgs& a, int b) {
+  return 1 + (a.with_video ? int(a.fl.nvalid[b]) * (a.T / kBN) : 0);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
-  extern __shared__ uint8_t smem_raw[];
-  SmemLayout sm = carve(smem_raw);
-  cg::cluster_group cluster = cg::this_cluster();
-  const int split = int(cluster.block_rank());
-  const int C = a.splits, h = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Walks the call's tile sequence: (b, h, t) of global tile g, nb tiles per (b, h).
+template <int kBN>
+struct TileWalk {
+  int b, h, t, nb;
+  __device__ __forceinline__ void init(const ActionArgs& a, int g) {
+    b = 0;
+    for (;;) {
+      nb = tiles_of<kBN>(a, b);
+      if (g < a.H * nb || b == a.B - 1) break;
+      g -= a.H * nb;
+      ++b;
+    }
+    h = g / nb;
+    t = g % nb;
+  }
+  __device__ __forceinline__ void next(const ActionArgs& a) {
+    if (++t < nb) return;
+    t = 0;
+    if (++h < a.H) return;
+    h = 0;
+    if (++b < a.B) nb = tiles_of<kBN>(a, b);
+  }
+};
 
-  // tiles of this split: [t0, t1) of the episode's valid video tiles, plus the action tile
-  const int tiles_per_frame = a.T / kBN;
-  const int nvt = a.with_video ? int(a.fl.nvalid[b]) * tiles_per_frame : 0;
-  const int per = (nvt + C - 1) / C;
-  const int t0 = min(nvt, split * per), t1 = min(nvt, t0 + per);
-  const int has_act = split == 0 ? 1 : 0;
-  const int n_tiles = (t1 - t0) + has_act;
+template <int kBN>
+__device__ __forceinline__ int first_tile_of(const ActionArgs& a, int b, int h) {
+  int g = 0;
+  for (int e = 0; e < b; ++e) g += a.H * tiles_of<kBN>(a, e);
+  return g + h * tiles_of<kBN>(a, b);
+}
+
+// First and last CTA whose run touches tiles [s, e) when CTA i runs [iG/P, (i+1)G/P).
+__device__ __forceinline__ int cta_of_start(int s, int G, int P) {
+  return int((int64_t(s + 1) * P + G - 1) / G) - 1;
+}
+__device__ __forceinline__ int cta_of_end(int e, int G, int P) {
+  return int((int64_t(e) * P + G - 1) / G) - 1;
+}
+
+__device__ __forceinline__ void store_out(const ActionArgs& a, int b, int h, int row, int col,
+                                          const float* v /*16*/) {
+  const int64_t off = ((int64_t(b) * a.n_act + row) * a.H + h) * 128 + col;
+  if (a.o_f32) {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint4 u;
+      u.x = pack_bf16(v[8 * i], v[8 * i + 1]), u.y = pack_bf16(v[8 * i + 2], v[8 * i + 3]);
+      u.z = pack_bf16(v[8 * i + 4], v[8 * i + 5]), u.w = pack_bf16(v[8 * i + 6], v[8 * i + 7]);
+      d[i] = u;
+    }
+  }
+}
+
+// kBN keys per tile (64 or 128); each consumer warp handles kBN / 4 keys of a tile.
+template <int kBN>
+__global__ void __launch_bounds__(kThreads, 1)
+action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
+  constexpr int kTileBytes = kBN * 128 * 2;  // one of K or V
+  constexpr int kStages = kRingBytes / (2 * kTileBytes);
+  constexpr int kWK = kBN / 4;               // keys per warp per tile
+  constexpr int kNT = kWK / 8;               // 8-key groups per warp per tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq[2] = {base, base + kQBytes};
+  uint8_t* sk[kStages];
+  uint8_t* sv[kStages];
+  for (int i = 0; i < kStages; ++i) {
+    sk[i] = base + 2 * kQBytes + i * 2 * kTileBytes;
+    sv[i] = sk[i] + kTileBytes;
+  }
+  float* obuf = reinterpret_cast<float*>(base + 2 * kQBytes + kStages * 2 * kTileBytes);  // [4][32][132]
+  float* mbuf = obuf + 4 * 32 * kOStride;  // [4][32]
+  float* lbuf = mbuf + 4 * 32;             // [4][32]
+  Bars& bars = *reinterpret_cast<Bars*>(lbuf + 4 * 32);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g0 = int(int64_t(blockIdx.x) * a.G / a.P), g1 = int(int64_t(blockIdx.x + 1) * a.G / a.P);
+  const int tpf = a.T / kBN;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], kConsumers);
+      mbar_init(&bars.full[i], 1);
+      mbar_init(&bars.empty[i], kConsumers);
     }
-    mbar_init(sm.qbar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.qfull[i], 1);
+      mbar_init(&bars.qempty[i], kConsumers);
+    }
     fence_barrier_init();
   }
   __syncthreads();
@@ -104,272 +158,473 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
   if (warp == kConsumers) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      prefetch_tmap(&maps.q);
-      mbar_arrive_expect_tx(sm.qbar, kQBytes);
-      tma_load_4d(sm.q, &maps.q, sm.qbar, 0, h, 0, b);
-      tma_load_4d(sm.q + kQBytes / 2, &maps.q, sm.qbar, 64, h, 0, b);
-      int issued = 0;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int st = i % kStages;
-        if (i >= kStages && !mbar_wait(&sm.empty[st], ((i / kStages) - 1) & 1)) { bad = true; break; }
-        mbar_arrive_expect_tx(&sm.full[st], 2 * kTileBytes);
+      TileWalk<kBN> tw;
+      tw.init(a, g0);
+      int seg = 0, issued = 0;
+      for (int g = g0; g < g1; ++g, tw.next(a)) {
+        const int i = g - g0, st = i % kStages;
+        if (g == g0 || tw.t == 0) {  // a new (b, h) run: its Q first
+          const int qs = seg & 1;
+          if (seg >= 2 && !mbar_wait(&bars.qempty[qs], ((seg >> 1) - 1) & 1)) { bad = true; break; }
+          mbar_arrive_expect_tx(&bars.qfull[qs], kQBytes);
+          tma_load_4d(sq[qs], &maps.q, &bars.qfull[qs], 0, tw.h, 0, tw.b);
+          tma_load_4d(sq[qs] + kQBytes / 2, &maps.q, &bars.qfull[qs], 64, tw.h, 0, tw.b);
+          ++seg;
+        }
+        if (i >= kStages && !mbar_wait(&bars.empty[st], ((i / kStages) - 1) & 1)) { bad = true; break; }
+        mbar_arrive_expect_tx(&bars.full[st], 2 * kTileBytes);
         const CUtensorMap *mk, *mv;
         int tok;
-        if (has_act && i == 0) {
+        if (tw.t == 0) {
           mk = &maps.ka, mv = &maps.va, tok = 0;
         } else {
-          const int t = t0 + i - has_act;
+          const int vt = tw.t - 1;
           mk = &maps.fk, mv = &maps.fv;
-          tok = int(a.fl.vlist[b * a.F + t / tiles_per_frame]) * a.T + (t % tiles_per_frame) * kBN;
+          tok = int(a.fl.vlist[tw.b * a.F + vt / tpf]) * a.T + (vt % tpf) * kBN;
         }
-        tma_load_4d(sm.k[st], mk, &sm.full[st], 0, h, tok, b);
-        tma_load_4d(sm.k[st] + kTileBytes / 2, mk, &sm.full[st], 64, h, tok, b);
-        tma_load_4d(sm.v[st], mv, &sm.full[st], 0, h, tok, b);
-        tma_load_4d(sm.v[st] + kTileBytes / 2, mv, &sm.full[st], 64, h, tok, b);
+        tma_load_4d(sk[st], mk, &bars.full[st], 0, tw.h, tok, tw.b);
+        tma_load_4d(sk[st] + kTileBytes / 2, mk, &bars.full[st], 64, tw.h, tok, tw.b);
+        tma_load_4d(sv[st], mv, &bars.full[st], 0, tw.h, tok, tw.b);
+        tma_load_4d(sv[st] + kTileBytes / 2, mv, &bars.full[st], 64, tw.h, tok, tw.b);
         issued = i + 1;
       }
-      // Drain: every issued load must land before the ring is reused as merge space.
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        if (!mbar_wait(&sm.full[i % kStages], (i / kStages) & 1)) break;
-      if (!mbar_wait(sm.qbar, 0)) bad = true;
+      // Drain the loads still in flight (only after a failed wait can any be outstanding).
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait(&bars.full[i % kStages], (i / kStages) & 1);
     }
+    __syncwarp();
   } else {
     // ---------------------------------------------------------------- consumers
-    const int qh = warp & 1, kh = warp >> 1;
-    const int g = lane >> 2, t = lane & 3;
-    float oacc[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    uint32_t qf[8][4];
-    bad = !__all_sync(0xffffffffu, mbar_wait(sm.qbar, 0));  // warp-uniform before collectives
-    if (!bad) {
-      const uint32_t qbase = smem_u32(sm.q);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        ldsm_x4(qbase + swz128<32>(16 * qh + (lane & 15), 16 * kk + (lane >> 4) * 8), qf[kk][0],
-                qf[kk][1], qf[kk][2], qf[kk][3]);
-    }
+    // Every wait in front of a warp-collective (ldmatrix, mma.sync) is voted across the warp;
+    // after a failed wait a warp keeps walking its tiles and runs without doing work, and it
+    // still arrives on every barrier and ticket, so peers and later calls are not stranded.
+    const unsigned FULL = 0xffffffffu;
+    const int qh = warp & 1, kq = warp >> 1;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int tid = threadIdx.x;  // 0..255
     const float c = a.scale_log2;
-    for (int i = 0; i < n_tiles && !bad; ++i) {
-      const int st = i % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[st], (i / kStages) & 1))) { bad = true; break; }
-      const uint32_t kb = smem_u32(sm.k[st]), vb = smem_u32(sm.v[st]);
-      // S = Q K^T for this warp's 16 rows x 32 keys
-      float s[4][4];
+    TileWalk<kBN> tw;
+    tw.init(a, g0);
+    int seg = 0;
+    int gi = g0;
+    while (gi < g1) {
+      // ---- one (b, h) run [gi, ge) of this CTA
+      const int b = tw.b, h = tw.h;
+      const int ge = min(g1, gi + (tw.nb - tw.t));
+      const int s_bh = first_tile_of<kBN>(a, b, h), e_bh = s_bh + tw.nb;
+      const int qs = seg & 1;
+      uint32_t qf[8][4];
+      bad = bad || !__all_sync(FULL, mbar_wait(&bars.qfull[qs], (seg >> 1) & 1));
+      if (!bad) {
+        const uint32_t qbase = smem_u32(sq[qs]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + swz128<kBN>(32 * kh + 16 * p + (lane & 7) + (lane >> 4) * 8,
-                                   16 * kk + ((lane >> 3) & 1) * 8),
-                  b0, b1, b2, b3);
-          mma_bf16(s[2 * p], qf[kk], b0, b1);
-          mma_bf16(s[2 * p + 1], qf[kk], b2, b3);
-        }
-      }
-      if (has_act && i == 0) {  // action tile: keys >= n_act are the zero-filled tail
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int key = 32 * kh + 8 * j + 2 * t;
-          if (key >= a.n_act) s[j][0] = s[j][2] = -INFINITY;
-          if (key + 1 >= a.n_act) s[j][1] = s[j][3] = -INFINITY;
-        }
-      }
-      // online softmax (rows g and g + 8), quad shuffles for the row reductions
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
-        mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
-      }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0 * c), mn1 = fmaxf(m1, mx1 * c);
-      const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        s[j][0] = exp2f(fmaf(s[j][0], c, -mu0));
-        s[j][1] = exp2f(fmaf(s[j][1], c, -mu0));
-        s[j][2] = exp2f(fmaf(s[j][2], c, -mu1));
-        s[j][3] = exp2f(fmaf(s[j][3], c, -mu1));
-        rs0 += s[j][0] + s[j][1];
-        rs1 += s[j][2] + s[j][3];
-      }
-      l0 = fmaf(l0, al0, rs0);
-      l1 = fmaf(l1, al1, rs1);
-      m0 = mn0, m1 = mn1;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        oacc[j][0] *= al0, oacc[j][1] *= al0, oacc[j][2] *= al1, oacc[j][3] *= al1;
-      }
-      // O += P V over this warp's 32 keys on tf32 tiles (m16n8k8): P keeps 10 mantissa bits
-      // instead of bf16's 7, and V widens from bf16 to tf32 exactly.  Within each 8-key group
-      // j the contraction index is permuted (logical k = t <-> key 8j + 2t, k = t + 4 <->
-      // key 8j + 2t + 1), which makes the S accumulators the A fragment and the two keys an
-      // ldmatrix.trans register holds the B fragment, with no data movement.
-      uint32_t pt[4][4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        pt[j][0] = to_tf32(s[j][0]);  // row g,     key 8j + 2t
-        pt[j][1] = to_tf32(s[j][2]);  // row g + 8, key 8j + 2t
-        pt[j][2] = to_tf32(s[j][1]);  // row g,     key 8j + 2t + 1
-        pt[j][3] = to_tf32(s[j][3]);  // row g + 8, key 8j + 2t + 1
-      }
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const int j0 = 2 * kk, j1 = 2 * kk + 1;  // 8-key groups of this 16-key step
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_t(vb + swz128<kBN>(32 * kh + 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8,
-                                     16 * p + (lane >> 4) * 8),
-                    r0, r1, r2, r3);
-          mma_tf32(oacc[2 * p], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r0), bf16_hi_bits(r0));
-          mma_tf32(oacc[2 * p], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r1), bf16_hi_bits(r1));
-          mma_tf32(oacc[2 * p + 1], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r2), bf16_hi_bits(r2));
-          mma_tf32(oacc[2 * p + 1], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r3), bf16_hi_bits(r3));
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          ldsm_x4(qbase + swz128<32>(16 * qh + (lane & 15), 16 * kk + (lane >> 4) * 8), qf[kk][0],
+                  qf[kk][1], qf[kk][2], qf[kk][3]);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[st]);
-    }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    // The ring becomes merge space once every consumer left the loop and the producer
-    // drained its loads: named barrier 1 over all threads of the CTA.
-    asm volatile("bar.sync 1, %0;" ::"n"(kThreads));
-    // partial of this warp -> obuf[kh]
-    float* ob = sm.obuf + kh * 32 * kOStride;
-    const int r0 = 16 * qh + g, r1 = r0 + 8;
+      if (lane == 0) mbar_arrive(&bars.qempty[qs]);
+      float oacc[16][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      *reinterpret_cast<float2*>(ob + r0 * kOStride + 8 * j + 2 * t) = make_float2(oacc[j][0], oacc[j][1]);
-      *reinterpret_cast<float2*>(ob + r1 * kOStride + 8 * j + 2 * t) = make_float2(oacc[j][2], oacc[j][3]);
+      for (int j = 0; j < 16; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+      for (; gi < ge; ++gi, tw.next(a)) {
+        const int i = gi - g0, st = i % kStages;
+        if (!bad && !__all_sync(FULL, mbar_wait(&bars.full[st], (i / kStages) & 1))) bad = true;
+        if (!bad) {
+          const uint32_t kb = smem_u32(sk[st]), vb = smem_u32(sv[st]);
+          // S = Q K^T: this warp's 16 rows x kWK keys (kNT independent 8-key accumulators)
+          const int kbase = kWK * kq;
+          float s[kNT][4];
+#pragma unroll
+          for (int j = 0; j < kNT; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int p = 0; p < kNT / 2; ++p) {
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(kb + swz128<kBN>(kbase + 16 * p + (lane & 7) + (lane >> 4) * 8,
+                                       16 * kk + ((lane >> 3) & 1) * 8),
+                      b0, b1, b2, b3);
+              mma_bf16(s[2 * p], qf[kk], b0, b1);
+              mma_bf16(s[2 * p + 1], qf[kk], b2, b3);
+            }
+          }
+          if (tw.t == 0) {  // action tile: keys >= n_act are the zero-filled tail
+#pragma unroll
+            for (int j = 0; j < kNT; ++j) {
+              const int key = kbase + 8 * j + 2 * t4;
+              if (key >= a.n_act) s[j][0] = s[j][2] = -INFINITY;
+              if (key + 1 >= a.n_act) s[j][1] = s[j][3] = -INFINITY;
+            }
+          }
+          // online softmax (rows g and g + 8), quad shuffles for the row reductions
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < kNT; ++j) {
+            mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+            mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+          }
+          mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
+          // The reference max of a row only moves when the tile's max exceeds it by more than
+          // 2^8 (p = 2^(s c - m) then stays below 2^8), so the accumulators are rarely rescaled;
+          // the rescale runs only when some row of the warp needs it.
+          const float c0 = mx0 * c, c1 = mx1 * c;
+          const float mn0 = c0 > m0 + kLazyLog2 ? c0 : m0, mn1 = c1 > m1 + kLazyLog2 ? c1 : m1;
+          const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+          float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < kNT; ++j) {
+            s[j][0] = ex2(fmaf(s[j][0], c, -mu0));
+            s[j][1] = ex2(fmaf(s[j][1], c, -mu0));
+            s[j][2] = ex2(fmaf(s[j][2], c, -mu1));
+            s[j][3] = ex2(fmaf(s[j][3], c, -mu1));
+            rs0 += s[j][0] + s[j][1];
+            rs1 += s[j][2] + s[j][3];
+          }
+          if (__any_sync(FULL, mn0 != m0 || mn1 != m1)) {
+            const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
+            l0 *= al0, l1 *= al1;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              oacc[j][0] *= al0, oacc[j][1] *= al0, oacc[j][2] *= al1, oacc[j][3] *= al1;
+            }
+          }
+          l0 += rs0, l1 += rs1;
+          m0 = mn0, m1 = mn1;
+          // O += P V over this warp's keys on tf32 tiles (m16n8k8).  Within each 8-key group
+          // j the contraction index is permuted (k = t <-> key 8j + 2t, k = t + 4 <-> 8j + 2t + 1)
+          // so the S accumulators are the A fragment and the two keys of an ldmatrix.trans
+          // register are the B fragment, with no data movement.
+          uint32_t pt[kNT][4];
+#pragma unroll
+          for (int j = 0; j < kNT; ++j) {
+            pt[j][0] = to_tf32(s[j][0]);
+            pt[j][1] = to_tf32(s[j][2]);
+            pt[j][2] = to_tf32(s[j][1]);
+            pt[j][3] = to_tf32(s[j][3]);
+          }
+#pragma unroll
+          for (int kb16 = 0; kb16 < kNT / 2; ++kb16) {
+            const int j0 = 2 * kb16, j1 = 2 * kb16 + 1;
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4_t(vb + swz128<kBN>(kbase + 16 * kb16 + (lane & 7) + ((lane >> 3) & 1) * 8,
+                                         16 * p + (lane >> 4) * 8),
+                        r0, r1, r2, r3);
+              mma_tf32(oacc[2 * p], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r0), bf16_hi_bits(r0));
+              mma_tf32(oacc[2 * p], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r1), bf16_hi_bits(r1));
+              mma_tf32(oacc[2 * p + 1], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r2), bf16_hi_bits(r2));
+              mma_tf32(oacc[2 * p + 1], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r3), bf16_hi_bits(r3));
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.empty[st]);
+      }
+      ++seg;
+      // ---- run done: the four key quarters of each query half -> one partial for 32 rows
+      l0 += __shfl_xor_sync(FULL, l0, 1);
+      l0 += __shfl_xor_sync(FULL, l0, 2);
+      l1 += __shfl_xor_sync(FULL, l1, 1);
+      l1 += __shfl_xor_sync(FULL, l1, 2);
+      {
+        float* ob = obuf + kq * 32 * kOStride;
+        const int r0 = 16 * qh + g, r1 = r0 + 8;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          *reinterpret_cast<float2*>(ob + r0 * kOStride + 8 * j + 2 * t4) = make_float2(oacc[j][0], oacc[j][1]);
+          *reinterpret_cast<float2*>(ob + r1 * kOStride + 8 * j + 2 * t4) = make_float2(oacc[j][2], oacc[j][3]);
+        }
+        if (t4 == 0) {
+          mbuf[kq * 32 + r0] = m0, mbuf[kq * 32 + r1] = m1;
+          lbuf[kq * 32 + r0] = l0, lbuf[kq * 32 + r1] = l1;
+        }
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      // thread -> (row, 16 columns) of the 32 x 128 partial
+      const int row = tid >> 3, col = (tid & 7) * 16;
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) M = fmaxf(M, mbuf[k * 32 + row]);
+      const float Mu = M == -INFINITY ? 0.f : M;
+      float fk[4], L = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        fk[k] = exp2f(mbuf[k * 32 + row] - Mu);
+        L = fmaf(lbuf[k * 32 + row], fk[k], L);
+      }
+      float ov[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ov[i] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(obuf + (k * 32 + row) * kOStride + col + i);
+          ov[i] = fmaf(fk[k], x.x, ov[i]), ov[i + 1] = fmaf(fk[k], x.y, ov[i + 1]);
+          ov[i + 2] = fmaf(fk[k], x.z, ov[i + 2]), ov[i + 3] = fmaf(fk[k], x.w, ov[i + 3]);
+        }
+      const int bh = b * a.H + h;
+      if (s_bh >= g0 && e_bh <= g1) {
+        // this CTA holds the whole (b, h): write O directly
+        if (row < a.n_act) {
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ov[i] *= inv;
+          store_out(a, b, h, row, col, ov);
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // merge buffers reused by the next run
+      } else {
+        // partial -> workspace slot (b, h, this CTA's rank among the CTAs touching (b, h))
+        const int i_lo = cta_of_start(s_bh, a.G, a.P), n_parts = cta_of_end(e_bh, a.G, a.P) - i_lo + 1;
+        float* slot = a.ws_part + (int64_t(bh) * a.max_parts + (int(blockIdx.x) - i_lo)) * kSlotFloats;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          __stcg(reinterpret_cast<float4*>(slot + row * 128 + col + i), make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]));
+        if ((tid & 7) == 0) {
+          __stcg(slot + 32 * 128 + row, M);
+          __stcg(slot + 32 * 128 + 32 + row, L);
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (tid == 0) bars.last = atomicAdd(a.ws_count + bh, 1) == n_parts - 1;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (bars.last) {
+          // every partial of (b, h) is in the workspace: merge them by log-sum-exp
+          __threadfence();
+          const float* slots = a.ws_part + int64_t(bh) * a.max_parts * kSlotFloats;
+          float Mt = -INFINITY;
+          for (int k = 0; k < n_parts; ++k) Mt = fmaxf(Mt, __ldcg(slots + k * kSlotFloats + 32 * 128 + row));
+          const float Mtu = Mt == -INFINITY ? 0.f : Mt;
+          float Lt = 0.f, acc[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+          // two partials per round, all their loads issued before any is used
+          for (int k = 0; k < n_parts; k += 2) {
+            const bool two = k + 1 < n_parts;
+            const float* sa = slots + k * kSlotFloats;
+            const float* sb = slots + (two ? k + 1 : k) * kSlotFloats;
+            float4 xa[4], xb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              xa[i] = __ldcg(reinterpret_cast<const float4*>(sa + row * 128 + col + 4 * i));
+              xb[i] = __ldcg(reinterpret_cast<const float4*>(sb + row * 128 + col + 4 * i));
+            }
+            const float ma = __ldcg(sa + 32 * 128 + row), la = __ldcg(sa + 32 * 128 + 32 + row);
+            const float mb = __ldcg(sb + 32 * 128 + row), lb = __ldcg(sb + 32 * 128 + 32 + row);
+            const float fa = exp2f(ma - Mtu), fb = two ? exp2f(mb - Mtu) : 0.f;
+            Lt = fmaf(la, fa, fmaf(lb, fb, Lt));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[4 * i] = fmaf(fa, xa[i].x, fmaf(fb, xb[i].x, acc[4 * i]));
+              acc[4 * i + 1] = fmaf(fa, xa[i].y, fmaf(fb, xb[i].y, acc[4 * i + 1]));
+              acc[4 * i + 2] = fmaf(fa, xa[i].z, fmaf(fb, xb[i].z, acc[4 * i + 2]));
+              acc[4 * i + 3] = fmaf(fa, xa[i].w, fmaf(fb, xb[i].w, acc[4 * i + 3]));
+            }
+          }
+          if (row < a.n_act) {
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] *= inv;
+            store_out(a, b, h, row, col, acc);
+          }
+          if (tid == 0) a.ws_count[bh] = 0;  // ready for the next call
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+      }
     }
-    if (t == 0) {
-      sm.mbuf[kh * 32 + r0] = m0, sm.mbuf[kh * 32 + r1] = m1;
-      sm.lbuf[kh * 32 + r0] = l0, sm.lbuf[kh * 32 + r1] = l1;
-    }
-  }
-  if (warp == kConsumers) {
-    __syncwarp();  // lane 0 ran the producer loop alone
-    asm volatile("bar.sync 1, %0;" ::"n"(kThreads));
   }
   if (bad && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
-
-  // ------------------------------------------------------------------ cluster merge
-  __syncwarp();
-  cluster.sync();
-  const int P = 2 * C;  // partials per (b, h)
-  if (threadIdx.x < 32) {
-    const int row = threadIdx.x;
-    float mv[32], M = -INFINITY;
-    for (int p = 0; p < P; ++p) {
-      const float* rm = cluster.map_shared_rank(sm.mbuf, p >> 1);
-      mv[p] = rm[(p & 1) * 32 + row];
-      M = fmaxf(M, mv[p]);
-    }
-    if (M == -INFINITY) M = 0.f;
-    float L = 0.f;
-    for (int p = 0; p < P; ++p) {
-      const float* rl = cluster.map_shared_rank(sm.lbuf, p >> 1);
-      mv[p] = exp2f(mv[p] - M);
-      L = fmaf(rl[(p & 1) * 32 + row], mv[p], L);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int p = 0; p < P; ++p) sm.fbuf[row * 32 + p] = mv[p] * inv;
-  }
-  __syncthreads();
-  const int rows_per = 32 / C;
-  const int rb = split * rows_per;
-  if (threadIdx.x < 128) {
-    const int col = (threadIdx.x & 31) * 4;
-    for (int row = rb + (threadIdx.x >> 5); row < rb + rows_per; row += 4) {
-      if (row >= a.n_act) break;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int p = 0; p < P; ++p) {
-        const float* ro = cluster.map_shared_rank(sm.obuf, p >> 1);
-        const float4 x = *reinterpret_cast<const float4*>(ro + (p & 1) * 32 * kOStride + row * kOStride + col);
-        const float f = sm.fbuf[row * 32 + p];
-        acc.x = fmaf(f, x.x, acc.x), acc.y = fmaf(f, x.y, acc.y);
-        acc.z = fmaf(f, x.z, acc.z), acc.w = fmaf(f, x.w, acc.w);
-      }
-      const int64_t off = ((int64_t(b) * a.n_act + row) * a.H + h) * 128 + col;
-      if (a.o_f32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(a.o) + off) = acc;
-      } else {
-        uint2 u;
-        u.x = pack_bf16(acc.x, acc.y);
-        u.y = pack_bf16(acc.z, acc.w);
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + off) = u;
-      }
-    }
-  }
-  cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
-int pick_splits(const ActionArgs& a) {
-  if (!a.with_video) return 1;
-  int maxv = 0;
-  for (int b = 0; b < a.B; ++b) maxv = maxv > a.fl.nvalid[b] ? maxv : a.fl.nvalid[b];
-  const int tiles = maxv * (a.T / kBN);
-  const int target = 2 * 148;  // two resident CTAs per SM
-  int C = 1;
-  while (C < 16 && a.B * a.H * C < target && tiles / (2 * C) >= 4) C *= 2;
-  return C;
+// Action self-attention of a layer outside the interaction set (no video buffer): one CTA of
+// two warps per (episode, head), the n_act <= 32 action keys staged with cp.async into padded
+// shared memory rows (272 B pitch: conflict-free ldmatrix), one softmax per row in registers.
+constexpr int kSelfPitch = 128 * 2 + 16;
+
+__global__ void __launch_bounds__(64)
+action_self_kernel(const __grid_constant__ ActionArgs a) {
+  __shared__ __align__(16) uint8_t sm[3][32 * kSelfPitch];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned FULL = 0xffffffffu;
+  const __nv_bfloat16* src[3] = {static_cast<const __nv_bfloat16*>(a.qa),
+                                 static_cast<const __nv_bfloat16*>(a.ka),
+                                 static_cast<const __nv_bfloat16*>(a.va)};
+  for (int cidx = tid; cidx < 3 * 32 * 16; cidx += 64) {
+    const int ts = cidx >> 9, r = (cidx >> 4) & 31, ch = cidx & 15;
+    const int rr = r < a.n_act ? r : 0;  // rows past n_act read nothing and are zero-filled
+    const __nv_bfloat16* g = src[ts] + ((int64_t(b) * a.n_act + rr) * a.H + h) * 128 + ch * 8;
+    const uint32_t d = smem_u32(&sm[ts][r * kSelfPitch + ch * 16]);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(g),
+                 "r"(r < a.n_act ? 16 : 0)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  const int g = lane >> 2, t4 = lane & 3;
+  const uint32_t sq = smem_u32(sm[0]), sk = smem_u32(sm[1]), sv = smem_u32(sm[2]);
+  // S = Q K^T for this warp's 16 rows x 32 keys
+  float s[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    uint32_t qf[4];
+    ldsm_x4(sq + (16 * warp + (lane & 15)) * kSelfPitch + (16 * kk + (lane >> 4) * 8) * 2, qf[0],
+            qf[1], qf[2], qf[3]);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(sk + (16 * p + (lane & 7) + (lane >> 4) * 8) * kSelfPitch + (16 * kk + ((lane >> 3) & 1) * 8) * 2,
+              b0, b1, b2, b3);
+      mma_bf16(s[2 * p], qf, b0, b1);
+      mma_bf16(s[2 * p + 1], qf, b2, b3);
+    }
+  }
+  const float c = a.scale_log2;
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int key = 8 * j + 2 * t4;
+    if (key >= a.n_act) s[j][0] = s[j][2] = -INFINITY;
+    if (key + 1 >= a.n_act) s[j][1] = s[j][3] = -INFINITY;
+    mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+    mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+  }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    s[j][0] = ex2(fmaf(s[j][0], c, -mx0 * c));
+    s[j][1] = ex2(fmaf(s[j][1], c, -mx0 * c));
+    s[j][2] = ex2(fmaf(s[j][2], c, -mx1 * c));
+    s[j][3] = ex2(fmaf(s[j][3], c, -mx1 * c));
+    l0 += s[j][0] + s[j][1];
+    l1 += s[j][2] + s[j][3];
+  }
+  l0 += __shfl_xor_sync(FULL, l0, 1);
+  l0 += __shfl_xor_sync(FULL, l0, 2);
+  l1 += __shfl_xor_sync(FULL, l1, 1);
+  l1 += __shfl_xor_sync(FULL, l1, 2);
+  // O = P V on tf32 tiles, with the same key permutation inside each 8-key group as the
+  // fused read (S accumulators are the A fragment, ldmatrix.trans registers the B fragment)
+  uint32_t pt[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    pt[j][0] = to_tf32(s[j][0]);
+    pt[j][1] = to_tf32(s[j][2]);
+    pt[j][2] = to_tf32(s[j][1]);
+    pt[j][3] = to_tf32(s[j][3]);
+  }
+  float o[16][4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+#pragma unroll
+  for (int kb16 = 0; kb16 < 2; ++kb16) {
+    const int j0 = 2 * kb16, j1 = j0 + 1;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(sv + (16 * kb16 + (lane & 7) + ((lane >> 3) & 1) * 8) * kSelfPitch + (16 * p + (lane >> 4) * 8) * 2,
+                r0, r1, r2, r3);
+      mma_tf32(o[2 * p], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r0), bf16_hi_bits(r0));
+      mma_tf32(o[2 * p], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r1), bf16_hi_bits(r1));
+      mma_tf32(o[2 * p + 1], pt[j0][0], pt[j0][1], pt[j0][2], pt[j0][3], bf16_lo_bits(r2), bf16_hi_bits(r2));
+      mma_tf32(o[2 * p + 1], pt[j1][0], pt[j1][1], pt[j1][2], pt[j1][3], bf16_lo_bits(r3), bf16_hi_bits(r3));
+    }
+  }
+  const float i0 = 1.f / l0, i1 = 1.f / l1;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int col = 8 * j + 2 * t4;
+    if (r0 < a.n_act) {
+      const int64_t off = ((int64_t(b) * a.n_act + r0) * a.H + h) * 128 + col;
+      if (a.o_f32) *reinterpret_cast<float2*>(static_cast<float*>(a.o) + off) = make_float2(o[j][0] * i0, o[j][1] * i0);
+      else *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(a.o) + off) = pack_bf16(o[j][0] * i0, o[j][1] * i0);
+    }
+    if (r1 < a.n_act) {
+      const int64_t off = ((int64_t(b) * a.n_act + r1) * a.H + h) * 128 + col;
+      if (a.o_f32) *reinterpret_cast<float2*>(static_cast<float*>(a.o) + off) = make_float2(o[j][2] * i1, o[j][3] * i1);
+      else *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(a.o) + off) = pack_bf16(o[j][2] * i1, o[j][3] * i1);
+    }
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_action_tc(const ActionArgs& args, cudaStream_t s) {
-  ActionArgs a = args;
-  a.splits = pick_splits(a);
+static int action_bn(const ActionArgs& a) { return a.T % 128 == 0 ? 128 : 64; }
+
+int action_tc_total_tiles(const ActionArgs& a) {
+  const int bn = action_bn(a);
+  int G = 0;
+  for (int b = 0; b < a.B; ++b)
+    G += a.H * (1 + (a.with_video ? int(a.fl.nvalid[b]) * (a.T / bn) : 0));
+  return G;
+}
+
+int action_tc_max_parts(const ActionArgs& a, int P, int G) {
+  const int bn = action_bn(a);
+  int g = 0, mx = 1;
+  for (int b = 0; b < a.B; ++b) {
+    const int nb = 1 + (a.with_video ? int(a.fl.nvalid[b]) * (a.T / bn) : 0);
+    for (int h = 0; h < a.H; ++h, g += nb) {
+      const int lo = int((int64_t(g + 1) * P + G - 1) / G) - 1;
+      const int hi = int((int64_t(g + nb) * P + G - 1) / G) - 1;
+      if (hi - lo + 1 > mx) mx = hi - lo + 1;
+    }
+  }
+  return mx;
+}
+
+size_t action_tc_workspace_bytes(int BH, int max_parts) {
+  if (max_parts <= 1) return 0;
+  return kTicketBytes + size_t(BH) * max_parts * kSlotFloats * sizeof(float);
+}
+
+cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
+  if (!a.with_video) {
+    action_self_kernel<<<dim3(a.H, a.B), 64, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  const int bn = action_bn(a);
   ActionMaps maps;
   const int N = a.F * a.T;
   if (!make_tmap_bf16(&maps.q, a.qa, a.B, a.n_act, a.H, 32) ||
-      !make_tmap_bf16(&maps.ka, a.ka, a.B, a.n_act, a.H, kBN) ||
-      !make_tmap_bf16(&maps.va, a.va, a.B, a.n_act, a.H, kBN))
+      !make_tmap_bf16(&maps.ka, a.ka, a.B, a.n_act, a.H, bn) ||
+      !make_tmap_bf16(&maps.va, a.va, a.B, a.n_act, a.H, bn))
     return cudaErrorInvalidValue;
   if (a.with_video) {
-    if (!make_tmap_bf16(&maps.fk, a.fk, a.B, N, a.H, kBN) ||
-        !make_tmap_bf16(&maps.fv, a.fv, a.B, N, a.H, kBN))
+    if (!make_tmap_bf16(&maps.fk, a.fk, a.B, N, a.H, bn) ||
+        !make_tmap_bf16(&maps.fv, a.fv, a.B, N, a.H, bn))
       return cudaErrorInvalidValue;
   } else {
     maps.fk = maps.ka, maps.fv = maps.va;
   }
-  static unsigned configured = 0;  // one bit per device
+  static unsigned configured = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 32) return cudaErrorInvalidDevice;
   if (!(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(action_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(action_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured |= 1u << dev;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.splits, a.H, a.B);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, action_tc_kernel, a, maps);
+  if (bn == 128)
+    action_tc_kernel<128><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
+  else
+    action_tc_kernel<64><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
+  return cudaGetLastError();
 }
 
 }  // namespace wam

@@ -136,6 +136,19 @@ void fill_items(const Geo& g, int f_begin, int f_end, wam::FrameLists& fl) {
   std::copy(items.begin(), items.end(), fl.item);
 }
 
+// SM count of the current device (looked up once per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 wam_status check_range(const Geo& g, int f_begin, int f_end) {
   if (f_begin < 0 || f_end > g.F || f_begin >= f_end)
     return fail(WAM_ERR_INVALID_ARGUMENT, "frame range [%d, %d) is not inside [0, %d)", f_begin,
@@ -346,9 +359,41 @@ wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, in
                      "wam_fuse_interval_kv");
 }
 
+// Geometry of the persistent tensor-core action read: tiles G, CTAs P, partial slots.
+static wam_status action_plan(wam::ActionArgs& a, size_t* bytes) {
+  const int sms = sm_count();
+  if (sms <= 0) return fail(WAM_ERR_CUDA, "wam_action_attn: no CUDA device");
+  if (int64_t(a.B) * a.H * int64_t(sizeof(int)) > int64_t(wam::kTicketBytes))
+    return fail(WAM_ERR_UNSUPPORTED, "wam_action_attn: B * H exceeds %d", int(wam::kTicketBytes / sizeof(int)));
+  a.G = wam::action_tc_total_tiles(a);
+  a.P = a.G < sms ? a.G : sms;
+  a.max_parts = wam::action_tc_max_parts(a, a.P, a.G);
+  *bytes = wam::action_tc_workspace_bytes(a.B * a.H, a.max_parts);
+  return WAM_OK;
+}
+
+wam_status wam_action_attn_workspace_size(const wam_video_layout* layout, wam_dtype dt,
+                                          int32_t n_act, int32_t with_video, size_t* bytes) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(dt, "dt"));
+  if (!bytes) return fail(WAM_ERR_INVALID_ARGUMENT, "bytes is NULL");
+  if (n_act < 1 || n_act > 128)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n_act must be in [1, 128] (got %d)", n_act);
+  *bytes = 0;
+  if (!tc_action_ok(g, dt, n_act)) return ok();
+  static thread_local wam::ActionArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.n_act = n_act, a.with_video = with_video ? 1 : 0;
+  fill_vlists(g, a.fl);
+  WAM_CHECK(action_plan(a, bytes));
+  return ok();
+}
+
 wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const void* fused_k,
                            const void* fused_v, int32_t n_act, const void* qa, const void* ka,
-                           const void* va, void* o, wam_dtype o_dt, wam_stream_t stream) {
+                           const void* va, void* o, wam_dtype o_dt, void* workspace,
+                           size_t ws_bytes, wam_stream_t stream) {
   Geo g;
   WAM_CHECK(check_layout(layout, g));
   WAM_CHECK(check_dtype(dt, "dt"));
@@ -378,6 +423,17 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const v
   fill_vlists(g, a.fl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (tc_action_ok(g, dt, n_act)) {
+    size_t need = 0;
+    WAM_CHECK(action_plan(a, &need));
+    if (need) {
+      if (!workspace || ws_bytes < need)
+        return fail(WAM_ERR_WORKSPACE, "wam_action_attn: workspace of %zu bytes needed (got %zu)",
+                    need, workspace ? ws_bytes : size_t(0));
+      if (!aligned16(workspace))
+        return fail(WAM_ERR_INVALID_ARGUMENT, "workspace is not 16-byte aligned");
+      a.ws_count = static_cast<int*>(workspace);
+      a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + wam::kTicketBytes);
+    }
     cudaError_t e = wam::launch_action_tc(a, s);
     if (e != cudaErrorNotSupported) return cuda_status(e, "wam_action_attn (tensor cores)");
   }

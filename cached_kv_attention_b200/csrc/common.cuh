@@ -66,7 +66,11 @@ struct ActionArgs {
   int32_t B, H, T, F, n_act;
   int32_t o_f32;
   int32_t with_video;
-  int32_t splits;  // split-KV factor = cluster size
+  int32_t P;          // CTAs of the persistent grid
+  int32_t G;          // tiles of the whole call (all episodes and heads)
+  int32_t max_parts;  // workspace slots per (episode, head)
+  float* ws_part;     // partial (O, m, l) slots [B*H][max_parts][32*128 + 64]
+  int* ws_count;      // arrival tickets [B*H]; zero between calls
   float scale_log2;
   int* err;
   FrameLists fl;

@@ -20,6 +20,12 @@ cudaError_t launch_action_simt(const ActionArgs& a, int D, bool bf16, cudaStream
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);   // tcgen05 + TMEM
 cudaError_t launch_prefill_mma(const PrefillArgs& a, cudaStream_t s);  // mma.sync tiles
 cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s);
+int action_tc_total_tiles(const ActionArgs& a);
+int action_tc_max_parts(const ActionArgs& a, int P, int G);
+size_t action_tc_workspace_bytes(int BH, int max_parts);
+// The action-read workspace starts with a fixed ticket region, so tickets never land on
+// partial data of an earlier call with another layout; partial slots follow it.
+constexpr size_t kTicketBytes = 65536;  // one int per (episode, head): B * H <= 16384
 
 // Tensor map of a token-major bf16 tensor [B, ntok, H, 128] with a box of 64 x rows
 // (128B swizzle), rows along the token dimension.

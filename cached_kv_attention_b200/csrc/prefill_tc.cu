@@ -13,16 +13,17 @@
 //   P_w = exp2(S_w c - m_w)   softmax warpgroup w; bf16 P written back over S_w in TMEM
 //   O_w += P_w V_j            tcgen05.mma, A from TMEM, B (V, MN-major) from shared memory
 // The MMA thread alternates the two tiles (P_0 V, next S_0, P_1 V, next S_1, ...), so the
-// tensor core works on one tile while the other tile's warpgroup runs its softmax.  A row's
-// reference max m_w only moves when a key tile raises the row max by more than 8 (a factor
-// 2^8); O_w is then rescaled in TMEM.  S_w of key tile j is issued after P_w V_{j-1}, so its
-// completion implies O_w is complete up to j-1 and the rescale needs no extra wait.  The
+// tensor core works on one tile while the other tile's warpgroup runs its softmax, a single
+// pass over S per tile.  A row's reference max m_w is set by its first 32 scores and only
+// moves when a later chunk's max exceeds it by more than 2^64; l, O_w and the P already
+// written are then rescaled in TMEM.  S_w of key tile j is issued after P_w V_{j-1}, so its
+// completion implies O_w is complete up to j-1 and a rescale needs no extra wait.  The
 // numerator and denominator share the reference, so the result is exact either way.
 //
-// While the CTA's own K/V tiles (the key tokens equal to its query tokens) are resident, two
-// helper warps store them into the layer's cache and fold them into the Interval KV-Fusion
-// accumulator ("世界模型之Faster-WAM详解" §3.3): the per-layer K/V is never re-read for fusion.
-// The own tiles come last in the key order, so the stages they hold are not needed afterwards.
+// Two helper warps store the CTA's own new K/V tokens (those equal to its query tokens) into
+// the layer's cache and fold them into the Interval KV-Fusion accumulator ("世界模型之Faster-WAM
+// 详解" §3.3) from the call's input while the attention loop runs, so the store and the fold
+// never wait on the pipeline and the per-layer cache is never re-read for fusion.
 //
 // Warps: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-3 cache store + fusion |
 //        4-7 softmax of Q0, 8-11 softmax of Q1 (thread = query row; warp w reads TMEM lanes
@@ -41,7 +42,10 @@ constexpr int kTile = 128 * 128 * 2;  // one Q, K or V tile: two 64-column swizz
 constexpr int kHalf = kTile / 2;
 constexpr int kKStages = 3, kVStages = 2;
 constexpr uint32_t kTmemCols = 512;   // query tile w: S/P at 256 w, O at 256 w + 128
-constexpr float kRescaleLog2 = 8.f;
+// A row's reference max only moves when a key tile's row max exceeds it by more than this
+// (log2 units): below it p = 2^(s c - m) stays under 2^64, far from fp32 overflow even summed
+// over every key, and bf16/fp32 keep their relative precision at any scale.
+constexpr float kHeadroomLog2 = 64.f;
 
 struct PrefillMaps {
   CUtensorMap q, kn, vn, kc, vc;
@@ -68,22 +72,28 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
-// Store (and fold into the fusion accumulator) one resident 128-token K or V tile; 64 threads.
-// Each thread handles 4 chunks of 8 elements per round and issues all their accumulator loads
-// before using any of them, so the read-modify-write keeps several loads in flight.
-__device__ __forceinline__ void store_fuse_tile128(const PrefillArgs& a, const uint8_t* tile,
-                                                   void* store_base, float* acc_base,
-                                                   void* fused_base, int64_t row0, int h, int t) {
+// Store the CTA's own new K or V rows into the layer's cache and fold them into the fusion
+// accumulator, straight from the call's input (64 threads, `rows` tokens from row0_in of the
+// input to row0_out of the cache).  Each thread keeps 4 chunks of 8 elements in flight.
+__device__ __forceinline__ void store_fuse_rows(const PrefillArgs& a, const void* in_base,
+                                                void* store_base, float* acc_base,
+                                                void* fused_base, int64_t row0_in,
+                                                int64_t row0_out, int rows, int h, int t) {
   constexpr int kU = 4;
-  for (int c0 = t; c0 < kBN * 16; c0 += 64 * kU) {
+  const int chunks = rows * 16;
+  for (int c0 = t; c0 < chunks; c0 += 64 * kU) {
     uint4 raw[kU];
     float4 p0[kU], p1[kU];
     int64_t off[kU];
+    bool live[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int c = c0 + 64 * u, r = c >> 4, cc = (c & 15) * 8;
-      raw[u] = *reinterpret_cast<const uint4*>(tile + swz128<kBN>(r, cc));
-      off[u] = ((row0 + r) * a.H + h) * 128 + cc;
+      live[u] = c < chunks;
+      if (!live[u]) continue;
+      raw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(in_base) +
+                                               ((row0_in + r) * a.H + h) * 128 + cc);
+      off[u] = ((row0_out + r) * a.H + h) * 128 + cc;
       if (a.fuse_on && !a.fuse_first) {
         p0[u] = *reinterpret_cast<const float4*>(acc_base + off[u]);
         p1[u] = *reinterpret_cast<const float4*>(acc_base + off[u] + 4);
@@ -91,6 +101,7 @@ __device__ __forceinline__ void store_fuse_tile128(const PrefillArgs& a, const u
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
+      if (!live[u]) continue;
       if (store_base)
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(store_base) + off[u]) = raw[u];
       if (!a.fuse_on) continue;
@@ -117,15 +128,6 @@ __device__ __forceinline__ void store_fuse_tile128(const PrefillArgs& a, const u
   }
 }
 
-// Pulls accumulator rows into L2 ahead of the fold (64 threads, 512 B per row).
-__device__ __forceinline__ void prefetch_acc_rows(const PrefillArgs& a, const float* acc,
-                                                  int64_t row0, int rows, int h, int t) {
-  for (int r = t; r < rows; r += 64) {
-    const float* p = acc + ((row0 + r) * a.H + h) * 128;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], 512;" ::"l"(p) : "memory");
-  }
-}
-
 // tcgen05.mma with A from tensor memory: D[tmem] (+)= A[tmem] * B[smem desc]^T.  A 16-bit A
 // operand keeps row m in TMEM lane m and elements 2i, 2i+1 of its K dimension in the low and
 // high half of column i.
@@ -136,6 +138,16 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -152,11 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ[2] = {base, base + kTile};
-  uint8_t* sK[kKStages];
-  uint8_t* sV[kVStages];
-  for (int i = 0; i < kKStages; ++i) sK[i] = base + (2 + i) * kTile;
-  for (int i = 0; i < kVStages; ++i) sV[i] = base + (2 + kKStages + i) * kTile;
+  // Tiles by arithmetic, not through pointer arrays (a runtime index would put those in local memory).
+  auto sQ = [&](int w) { return base + w * kTile; };
+  auto sK = [&](int i) { return base + (2 + i) * kTile; };
+  auto sV = [&](int i) { return base + (2 + kKStages + i) * kTile; };
   Bars& bars = *reinterpret_cast<Bars*>(base + (2 + kKStages + kVStages) * kTile);
   volatile int* abort = &bars.abort;
 
@@ -173,16 +184,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const int qtok0 = (f - a.f_begin) * a.T + qp * 2 * kBM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Key order: the visible tiles in list order with the CTA's own tiles (a contiguous block
-  // [own0, own0 + nq) of the list) moved to the end.
-  int own_u = nk - 1;
-  for (int u = 0; u < nk; ++u)
-    if (a.fl.vlist[b * a.F + u] == f) own_u = u;
-  const int own0 = own_u * tpf + 2 * qp;
-  auto key_tile = [&](int j, bool& old, int& tok, int& fk, int& jj) {
-    const int jm = j < n - nq ? (j < own0 ? j : j + nq) : own0 + (j - (n - nq));
-    fk = a.fl.vlist[b * a.F + jm / tpf];
-    jj = jm % tpf;
+  auto key_tile = [&](int j, bool& old, int& tok) {
+    const int fk = a.fl.vlist[b * a.F + j / tpf], jj = j % tpf;
     old = fk < a.f_begin;
     tok = (old ? fk : fk - a.f_begin) * a.T + jj * kBN;
   };
@@ -191,11 +194,11 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.k_empty[s], 2);  // MMA completion + store warps
+      mbar_init(&bars.k_empty[s], 1);  // MMA completion
     }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.v_empty[s], 2);
+      mbar_init(&bars.v_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars.s_full[w], 1);
@@ -221,25 +224,25 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       int k_issued = 0, v_issued = 0;
       mbar_arrive_expect_tx(&bars.q_full, nq * kTile);
       for (int w = 0; w < nq; ++w) {
-        tma_load_4d(sQ[w], &maps.q, &bars.q_full, 0, h, qtok0 + w * kBM, b);
-        tma_load_4d(sQ[w] + kHalf, &maps.q, &bars.q_full, 64, h, qtok0 + w * kBM, b);
+        tma_load_4d(sQ(w), &maps.q, &bars.q_full, 0, h, qtok0 + w * kBM, b);
+        tma_load_4d(sQ(w) + kHalf, &maps.q, &bars.q_full, 64, h, qtok0 + w * kBM, b);
       }
       for (int j = 0; j < n; ++j) {
         bool old;
-        int tok, fk, jj;
-        key_tile(j, old, tok, fk, jj);
+        int tok;
+        key_tile(j, old, tok);
         const int ks = j % kKStages, vs = j % kVStages;
         if (j >= kKStages && !wait_bar(&bars.k_empty[ks], ((j / kKStages) - 1) & 1, abort)) break;
         const CUtensorMap* mk = old ? &maps.kc : &maps.kn;
         mbar_arrive_expect_tx(&bars.k_full[ks], kTile);
-        tma_load_4d(sK[ks], mk, &bars.k_full[ks], 0, h, tok, b);
-        tma_load_4d(sK[ks] + kHalf, mk, &bars.k_full[ks], 64, h, tok, b);
+        tma_load_4d(sK(ks), mk, &bars.k_full[ks], 0, h, tok, b);
+        tma_load_4d(sK(ks) + kHalf, mk, &bars.k_full[ks], 64, h, tok, b);
         k_issued = j + 1;
         if (j >= kVStages && !wait_bar(&bars.v_empty[vs], ((j / kVStages) - 1) & 1, abort)) break;
         const CUtensorMap* mv = old ? &maps.vc : &maps.vn;
         mbar_arrive_expect_tx(&bars.v_full[vs], kTile);
-        tma_load_4d(sV[vs], mv, &bars.v_full[vs], 0, h, tok, b);
-        tma_load_4d(sV[vs] + kHalf, mv, &bars.v_full[vs], 64, h, tok, b);
+        tma_load_4d(sV(vs), mv, &bars.v_full[vs], 0, h, tok, b);
+        tma_load_4d(sV(vs) + kHalf, mv, &bars.v_full[vs], 64, h, tok, b);
         v_issued = j + 1;
       }
       // Drain: loads issued must land before the CTA leaves (matters only after an abort).
@@ -256,7 +259,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       const uint32_t idO = tc05::idesc_bf16_f32(128, 128, true);
       const uint32_t tS[2] = {tmem, tmem + 256}, tO[2] = {tmem + 128, tmem + 384};
       auto issue_S = [&](int w, int j) {
-        const uint32_t q_s = smem_u32(sQ[w]), k_s = smem_u32(sK[j % kKStages]);
+        const uint32_t q_s = smem_u32(sQ(w)), k_s = smem_u32(sK(j % kKStages));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
@@ -265,7 +268,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         }
       };
       auto issue_PV = [&](int w, int j) {
-        const uint32_t v_s = smem_u32(sV[j % kVStages]);
+        const uint32_t v_s = smem_u32(sV(j % kVStages));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tO[w], tS[w] + 8 * kk, tc05::smem_desc_sw128(v_s + kk * 2048, kHalf, 1024), idO,
@@ -303,30 +306,14 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ cache store + fusion
-    // The 64 threads run every iteration (a failed wait skips work, never the named barrier).
+    // The CTA's own tokens, read from the call's new K/V while the attention loop runs.
     const int t = threadIdx.x - 64;
-    const bool do_store = a.k_store != nullptr || a.fuse_on;
-    const int64_t N = int64_t(a.F) * a.T;
-    const int64_t own_row0 = int64_t(b) * N + int64_t(f) * a.T + qp * 2 * kBN;
-    if (a.fuse_on && !a.fuse_first) {
-      prefetch_acc_rows(a, a.acc_k, own_row0, nq * kBN, h, t);
-      prefetch_acc_rows(a, a.acc_v, own_row0, nq * kBN, h, t);
-    }
-    for (int j = 0; j < n; ++j) {
-      const int ks = j % kKStages, vs = j % kVStages;
-      bool old;
-      int tok, fk, jj;
-      key_tile(j, old, tok, fk, jj);
-      const bool own = do_store && fk == f && (jj >> 1) == qp;
-      const int64_t row0 = int64_t(b) * N + int64_t(f) * a.T + jj * kBN;
-      const bool okk = wait_bar(&bars.k_full[ks], (j / kKStages) & 1, abort);
-      if (okk && own) store_fuse_tile128(a, sK[ks], a.k_store, a.acc_k, a.fused_k, row0, h, t);
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (t == 0 && okk) mbar_arrive(&bars.k_empty[ks]);
-      const bool okv = wait_bar(&bars.v_full[vs], (j / kVStages) & 1, abort);
-      if (okv && own) store_fuse_tile128(a, sV[vs], a.v_store, a.acc_v, a.fused_v, row0, h, t);
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (t == 0 && okv) mbar_arrive(&bars.v_empty[vs]);
+    if (a.k_store != nullptr || a.fuse_on) {
+      const int64_t N = int64_t(a.F) * a.T, qtok = int64_t(a.f_end - a.f_begin) * a.T;
+      const int64_t row_in = int64_t(b) * qtok + qtok0;
+      const int64_t row_out = int64_t(b) * N + int64_t(f) * a.T + qp * 2 * kBM;
+      store_fuse_rows(a, a.k_new, a.k_store, a.acc_k, a.fused_k, row_in, row_out, nq * kBN, h, t);
+      store_fuse_rows(a, a.v_new, a.v_store, a.acc_v, a.fused_v, row_in, row_out, nq * kBN, h, t);
     }
   } else {
     // ------------------------------------------------------------ softmax, one row per thread
@@ -345,62 +332,69 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         ok = __all_sync(FULL, ok && wait_bar(&bars.s_full[w], j & 1, abort));
         if (!ok) continue;
         tc05::fence_after_sync();
-        // pass 1: row max of S over the 128 keys
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t x[32];
-          tc05::tmem_ld32(tS + 32 * q, x);
-          tc05::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(x[i]));
-        }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_cand = mx * c;
-        bool rescale = false;
-        float alpha = 1.f;
-        if (j == 0) {
-          m_ref = m_cand;
-        } else if (m_cand > m_ref + kRescaleLog2) {
-          alpha = tc05::fast_exp2(m_ref - m_cand);
-          l *= alpha;
-          m_ref = m_cand;
-          rescale = true;
-        }
-        // O_w holds P V of key tiles < j (S_w of tile j was issued after P_w V_{j-1}); rows
-        // that keep their reference scale by 1 (exact), so the whole warp runs the round trip.
-        if (__any_sync(FULL, rescale)) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t o[32];
-            tc05::tmem_ld32(tO + 32 * q, o);
-            tc05::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tc05::tmem_st32(tO + 32 * q, o);
-          }
-        }
-        // pass 2: P = exp2(S c - m_ref) as bf16 pairs over the first 64 columns of S (chunk q
-        // writes columns [16 q, 16 q + 16), all of which it or an earlier chunk already read)
+        // One pass over S in four 32-column chunks (two per TMEM wait).  P of chunk q goes to
+        // TMEM columns [16 q, 16 q + 16), all already read.  A chunk whose row max exceeds the
+        // reference by more than the headroom moves the reference up (the first chunk of a row
+        // always does: m_ref starts at -inf); l, the partial sums, O (key tiles < j) and the P
+        // chunks already written are then scaled by alpha = 2^(m_ref - m_new).  Lanes that keep
+        // their reference scale by 1 (exact), so every TMEM access is warp-collective.
         float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t x[32];
-          tc05::tmem_ld32(tS + 32 * q, x);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t x[2][32];
+          tc05::tmem_ld32(tS + 64 * q2, x[0]);
+          tc05::tmem_ld32(tS + 64 * q2 + 32, x[1]);
           tc05::tmem_wait_ld();
-          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = tc05::fast_exp2(fmaf(__uint_as_float(x[2 * i]), c, -m_ref));
-            const float p1 = tc05::fast_exp2(fmaf(__uint_as_float(x[2 * i + 1]), c, -m_ref));
-            sum8[(2 * i) & 7] += p0;
-            sum8[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16(p0, p1);  // key 2i in the low half
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int q = 2 * q2 + h2;
+            float cm8[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) cm8[i & 3] = fmaxf(cm8[i & 3], __uint_as_float(x[h2][i]));
+            const float m_c = fmaxf(fmaxf(cm8[0], cm8[1]), fmaxf(cm8[2], cm8[3])) * c;
+            const bool up = m_c > m_ref + kHeadroomLog2;
+            if (__any_sync(FULL, up)) {
+              const float m_new = up ? m_c : m_ref;
+              const float alpha = up ? tc05::fast_exp2(m_ref - m_new) : 1.f;
+              l *= alpha;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) sum8[u] *= alpha;
+              if (j > 0) {  // O holds P V of key tiles < j (S_w of tile j followed P_w V_{j-1})
+#pragma unroll
+                for (int qo = 0; qo < 4; ++qo) {
+                  uint32_t o[32];
+                  tc05::tmem_ld32(tO + 32 * qo, o);
+                  tc05::tmem_wait_ld();
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                  tc05::tmem_st32(tO + 32 * qo, o);
+                }
+              }
+              for (int qp2 = 0; qp2 < q; ++qp2) {  // P chunks of this tile already written
+                uint32_t pk[16];
+                tmem_ld16(tS + 16 * qp2, pk);
+                tc05::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
+                  pk[i] = pack_bf16(__low2float(v) * alpha, __high2float(v) * alpha);
+                }
+                tmem_st16(tS + 16 * qp2, pk);
+              }
+              tc05::tmem_wait_st();
+              m_ref = m_new;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i]), c, -m_ref));
+              const float p1 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i + 1]), c, -m_ref));
+              sum8[(2 * i) & 7] += p0;
+              sum8[(2 * i + 1) & 7] += p1;
+              pk[i] = pack_bf16(p0, p1);  // key 2i in the low half
+            }
+            tmem_st16(tS + 16 * q, pk);
           }
-          tmem_st16(tS + 16 * q, pk);
         }
         l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         tc05::tmem_wait_st();

@@ -16,7 +16,8 @@ __all__ = [
     "WamError", "F32", "BF16", "VideoLayout", "FuseEpilogue", "lib",
     "video_prefill_kv", "fuse_interval_kv", "action_attn", "flow_euler_step",
     "flow_schedule", "fuse_weights", "debug_video_mask", "device_error", "exported_names",
-    "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS",
+    "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS", "action_attn_workspace_size",
+    "action_workspace",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
@@ -57,7 +58,8 @@ def _load() -> ctypes.CDLL:
                                  ctypes.POINTER(_Fuse), vp],
         "wam_fuse_interval_kv": [lay, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                  ctypes.POINTER(f32), i32, i32, vp, vp, vp],
-        "wam_action_attn": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp],
+        "wam_action_attn": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp],
+        "wam_action_attn_workspace_size": [lay, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)],
         "wam_flow_euler_step": [i64, vp, vp, f32, vp],
         "wam_flow_schedule": [i32, f64, f64, ctypes.POINTER(f64)],
         "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
@@ -85,7 +87,7 @@ def exported_names() -> list:
     return ["wam_video_prefill_kv", "wam_fuse_interval_kv", "wam_action_attn",
             "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
             "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
-            "wam_video_prefill_kv_fuse_noalloc"]
+            "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size"]
 
 
 def check(status: int) -> None:
@@ -182,9 +184,42 @@ def fuse_interval_kv(layout: VideoLayout, k_layers, v_layers, weights, f_begin: 
                                    _ptr(fused_k), _ptr(fused_v), _stream(stream)))
 
 
-def action_attn(layout: VideoLayout, fused_k, fused_v, qa, ka, va, o, stream=None) -> None:
-    check(lib.wam_action_attn(layout.ref, _dtype(qa), _ptr(fused_k), _ptr(fused_v), qa.shape[1],
-                              _ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _stream(stream)))
+def action_attn_workspace_size(layout: VideoLayout, dtype: torch.dtype, n_act: int,
+                               with_video: bool = True) -> int:
+    """Bytes of workspace wam_action_attn needs for this layout on the current device."""
+    out = ctypes.c_size_t(0)
+    dt = BF16 if dtype == torch.bfloat16 else F32
+    check(lib.wam_action_attn_workspace_size(layout.ref, dt, n_act, int(with_video),
+                                             ctypes.byref(out)))
+    return out.value
+
+
+_workspaces = {}
+
+
+def action_workspace(nbytes: int, device=None) -> Optional[torch.Tensor]:
+    """A zero-filled device workspace of at least nbytes, cached per device.  The library
+    leaves it ready for the next call; calls sharing it must not overlap on the GPU."""
+    if nbytes == 0:
+        return None
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    ws = _workspaces.get(dev)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        _workspaces[dev] = ws
+    return ws
+
+
+def action_attn(layout: VideoLayout, fused_k, fused_v, qa, ka, va, o, workspace=None,
+                stream=None) -> None:
+    n_act = qa.shape[1]
+    if workspace is None:
+        need = action_attn_workspace_size(layout, qa.dtype, n_act, fused_k is not None)
+        workspace = action_workspace(need, qa.device.index)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.wam_action_attn(layout.ref, _dtype(qa), _ptr(fused_k), _ptr(fused_v), n_act,
+                              _ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _ptr(workspace),
+                              ws_bytes, _stream(stream)))
 
 
 def flow_euler_step(x, v, dsigma: float, stream=None) -> None:

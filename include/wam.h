@@ -52,7 +52,7 @@ typedef enum {
   WAM_ERR_INVALID_ARGUMENT = 1, /* a null pointer, bad size, misaligned pointer, bad range */
   WAM_ERR_UNSUPPORTED = 2,      /* a valid request this build has no kernel for */
   WAM_ERR_CUDA = 3,             /* a CUDA runtime error while configuring or launching */
-  WAM_ERR_WORKSPACE = 4,        /* reserved */
+  WAM_ERR_WORKSPACE = 4,        /* a workspace that is missing or too small */
   WAM_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up (wam_device_error) */
 } wam_status;
 
@@ -141,19 +141,33 @@ wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, in
  * Asymmetric action attention of one action-expert layer at one Euler step ("Fast-WAM 精读"
  * SECTION 07; Long-WAM Summary §3.2, §4.2; Faster-WAM详解 §3.2 SparseMoT):
  *   O = softmax(Q_a [K_video(non-padding frames); K_a]^T / sqrt(D)) [V_video; V_a]
- * computed as split-KV partials over the video keys merged with the action buffer by one
+ * computed as split-KV partials over the video keys and the action buffer, merged by one
  * shared online-softmax normalisation (no concatenated buffer is formed).
  *   fused_k, fused_v device [B, N, H, D] (dtype dt), or both NULL for a layer outside the
  *                    interaction set (action self-attention only)
  *   qa, ka, va       device [B, n_act, H, D] (dtype dt), 1 <= n_act <= 128
  *   o                device [B, n_act, H, D], dtype o_dt (WAM_F32 or dt)
- * Action tokens attend to each other bidirectionally.  No workspace: the split partials are
- * merged on chip through the distributed shared memory of a thread-block cluster.
+ *   workspace        device scratch of at least wam_action_attn_workspace_size() bytes, 16-byte
+ *                    aligned, zero-filled before its first use.  Its first 64 KiB hold one
+ *                    arrival ticket per (episode, head) (B * H <= 16384); every call that
+ *                    completes leaves them at zero, so one workspace serves calls of any layout
+ *                    in turn.  Calls that share a workspace must not overlap on the GPU.  May be
+ *                    NULL when the size is 0.
+ * Action tokens attend to each other bidirectionally.  Returns WAM_ERR_WORKSPACE if the
+ * workspace is missing or too small.
  */
 wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt,
                            const void* fused_k, const void* fused_v,
                            int32_t n_act, const void* qa, const void* ka, const void* va,
-                           void* o, wam_dtype o_dt, wam_stream_t stream);
+                           void* o, wam_dtype o_dt, void* workspace, size_t ws_bytes,
+                           wam_stream_t stream);
+
+/*
+ * Bytes of workspace wam_action_attn needs for this layout on the current device
+ * (with_video != 0: a layer that reads a fused pair).  Depends on the device's SM count.
+ */
+wam_status wam_action_attn_workspace_size(const wam_video_layout* layout, wam_dtype dt,
+                                          int32_t n_act, int32_t with_video, size_t* bytes);
 
 /*
  * One Euler step of the flow-matching sampler, x <- x + dsigma * v, elementwise over n fp32

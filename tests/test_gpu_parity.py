@@ -310,3 +310,45 @@ def test_action_padded_frames_are_never_read():
     wam.action_attn(lay, fk, fv, qa, ka, va, o2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
+
+
+def test_action_workspace_is_reused_and_checked():
+    # 24 heads x 85 tiles over 148 CTAs: every (b, h) is split over several CTAs and merged
+    # through the workspace; calling twice with one workspace must give identical outputs.
+    B, H, T, F, n = 2, 24, 768, 7, 32
+    pad = [[1, 0, 0, 0, 0, 0, 0], [0, 0, 1, 1, 0, 0, 0]]
+    lay = wam.VideoLayout(B, H, 128, T, F, pad)
+    fk, fv = (dev_normal((B, F * T, H, 128), 63, x, std=1 / np.sqrt(128), dtype=torch.bfloat16)
+              for x in ("fk", "fv"))
+    qa, ka, va = (dev_normal((B, n, H, 128), 63, x, std=1 / np.sqrt(128), dtype=torch.bfloat16)
+                  for x in ("qa", "ka", "va"))
+    need = wam.action_attn_workspace_size(lay, torch.bfloat16, n, True)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    o1 = torch.zeros((B, n, H, 128), device="cuda")
+    o2 = torch.zeros_like(o1)
+    wam.action_attn(lay, fk, fv, qa, ka, va, o1, workspace=ws)
+    wam.action_attn(lay, fk, fv, qa, ka, va, o2, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    assert int(ws[: B * H * 4].view(torch.int32).abs().sum()) == 0   # tickets back at zero
+    ref = O.action_attention(to64(qa), to64(ka), to64(va), to64(fk), to64(fv), np.array(pad), T)
+    assert_parity(to64(o1), ref, "bf16", "action split over CTAs")
+    with pytest.raises(wam.WamError) as e:
+        wam.action_attn(lay, fk, fv, qa, ka, va, o1, workspace=ws[: need // 2])
+    assert e.value.status == 4
+
+
+@pytest.mark.parametrize("big_frame", [0, 1, 2])
+def test_prefill_tensor_core_large_logit_jumps(big_frame):
+    # Keys of one frame scaled by 100: logits jump by ~100+ log2 units between key tiles, which
+    # moves the softmax reference mid-row (O, l and the P already written are rescaled in TMEM)
+    # when the big frame comes after others in the key order.
+    B, H, T, F = 1, 2, 128, 3
+    lay = wam.VideoLayout(B, H, 128, T, F)
+    q, k, v = (dev_normal((B, F * T, H, 128), 33, n, dtype=torch.bfloat16) for n in "qkv")
+    k[:, big_frame * T:(big_frame + 1) * T] *= 100.0
+    o = torch.zeros((B, F * T, H, 128), device="cuda")
+    wam.video_prefill_kv(lay, 0, F, q, k, v, torch.zeros_like(k), torch.zeros_like(v), o)
+    ref = O.video_prefill(to64(q), to64(k), to64(v), None, None, np.zeros((1, F)), None, T, 0, F)
+    assert_parity(to64(o), ref, "bf16", f"logit jumps, big frame {big_frame}")

@@ -107,7 +107,7 @@ def test_action_rejects_bad_arguments():
     lay = _lay()
     call = lambda **kw: L.wam_action_attn(lay.ref, kw.get("dt", wam.F32), kw.get("fk", FAKE),
                                           kw.get("fv", FAKE), kw.get("n", 8), kw.get("qa", FAKE),
-                                          FAKE, FAKE, FAKE, wam.F32, None)
+                                          FAKE, FAKE, FAKE, wam.F32, None, 0, None)
     assert call(n=0) == 1 and "n_act" in _msg()
     assert call(n=129) == 1 and "n_act" in _msg()
     assert call(fv=0) == 1 and "both" in _msg()

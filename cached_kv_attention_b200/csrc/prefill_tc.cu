@@ -42,10 +42,15 @@ constexpr int kTile = 128 * 128 * 2;  // one Q, K or V tile: two 64-column swizz
 constexpr int kHalf = kTile / 2;
 constexpr int kKStages = 3, kVStages = 2;
 constexpr uint32_t kTmemCols = 512;   // query tile w: S/P at 256 w, O at 256 w + 128
-// A row's reference max only moves when a key tile's row max exceeds it by more than this
-// (log2 units): below it p = 2^(s c - m) stays under 2^64, far from fp32 overflow even summed
-// over every key, and bf16/fp32 keep their relative precision at any scale.
-constexpr float kHeadroomLog2 = 64.f;
+// A row's reference max only moves when a 32-key chunk's sum of p = 2^(s c - m) exceeds this:
+// below it every p stays under 2^64, far from fp32 overflow even summed over every key, and
+// bf16/fp32 keep their relative precision at any scale.
+constexpr float kChunkSumLimit = 18446744073709551616.f;  // 2^64
+// Key pairs (of the 16 in a 32-key chunk) whose exponentials run on the FMA pipe
+// (exp2_poly2) instead of the special-function unit.
+constexpr uint32_t kPolyPairs = 0x0u;
+// P to bf16 by integer rounding and a byte permute instead of the conversion instruction.
+constexpr bool kPackPermute = false;
 
 struct PrefillMaps {
   CUtensorMap q, kn, vn, kc, vc;
@@ -126,6 +131,69 @@ __device__ __forceinline__ void store_fuse_rows(const PrefillArgs& a, const void
       }
     }
   }
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic)
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^y for a pair on the FMA pipe.  Cody-Waite style range reduction: y = n + f with
+// n = round(y) taken from the low mantissa bits of y + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f by
+// a cubic fitted for minimax relative error on that interval (coefficients computed for this
+// file with a Remez exchange; max relative error 7.5e-5, below bf16's 2^-9 rounding of P); the
+// integer n is then added into the exponent field.  y is clamped to [-126, 127] so the
+// exponent stays in range: below -126 the result is 2^-126 instead of ~0, negligible against
+// a row sum >= 1.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y2) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  float y0, y1;
+  f2unpack(y2, y0, y1);
+  y0 = fminf(fmaxf(y0, -126.f), 127.f);
+  y1 = fminf(fmaxf(y1, -126.f), 127.f);
+  const uint64_t yc = f2pack(y0, y1);
+  const uint64_t t = f2add(yc, f2pack(kRound, kRound));
+  const uint64_t f = f2sub(yc, f2sub(t, f2pack(kRound, kRound)));
+  uint64_t q = f2fma(f2pack(0.0551716685f, 0.0551716685f), f, f2pack(0.2426111251f, 0.2426111251f));
+  q = f2fma(q, f, f2pack(0.6932609677f, 0.6932609677f));
+  q = f2fma(q, f, f2pack(0.9999280572f, 0.9999280572f));
+  float t0, t1, q0, q1;
+  f2unpack(t, t0, t1);
+  f2unpack(q, q0, q1);
+  return f2pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
+// Two non-negative finite floats to a bf16 pair (first in the low half), rounded to nearest
+// (ties away from zero).
+__device__ __forceinline__ uint32_t pack_p(float p0, float p1) {
+  if (kPackPermute) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(p0) + 0x8000u),
+        "r"(__float_as_uint(p1) + 0x8000u));
+    return r;
+  }
+  return pack_bf16(p0, p1);
 }
 
 // tcgen05.mma with A from tensor memory: D[tmem] (+)= A[tmem] * B[smem desc]^T.  A 16-bit A
@@ -333,12 +401,14 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         if (!ok) continue;
         tc05::fence_after_sync();
         // One pass over S in four 32-column chunks (two per TMEM wait).  P of chunk q goes to
-        // TMEM columns [16 q, 16 q + 16), all already read.  A chunk whose row max exceeds the
-        // reference by more than the headroom moves the reference up (the first chunk of a row
-        // always does: m_ref starts at -inf); l, the partial sums, O (key tiles < j) and the P
-        // chunks already written are then scaled by alpha = 2^(m_ref - m_new).  Lanes that keep
-        // their reference scale by 1 (exact), so every TMEM access is warp-collective.
-        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // TMEM columns [16 q, 16 q + 16), all already read.  Each chunk is first exponentiated
+        // against the row's current reference m_ref.  A lane whose chunk sum exceeds 2^64 (or
+        // is inf: the first chunk of a row always is, m_ref starts at -inf) moves its reference
+        // to the chunk max; l, O (key tiles < j) and the P chunks already written are then
+        // scaled by alpha = 2^(m_ref - m_new) and the chunk is redone on the special-function
+        // unit.  Lanes that keep their reference scale by 1 (exact), so every TMEM access is
+        // warp-collective.
+        const uint64_t c2 = f2pack(c, c);
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t x[2][32];
@@ -348,17 +418,38 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int q = 2 * q2 + h2;
-            float cm8[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            uint32_t pk[16];
+            uint64_t acc[4] = {0, 0, 0, 0};
+            const uint64_t nm2 = f2pack(-m_ref, -m_ref);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) cm8[i & 3] = fmaxf(cm8[i & 3], __uint_as_float(x[h2][i]));
-            const float m_c = fmaxf(fmaxf(cm8[0], cm8[1]), fmaxf(cm8[2], cm8[3])) * c;
-            const bool up = m_c > m_ref + kHeadroomLog2;
+            for (int i = 0; i < 16; ++i) {
+              const uint64_t y = f2fma(f2pack(__uint_as_float(x[h2][2 * i]), __uint_as_float(x[h2][2 * i + 1])), c2, nm2);
+              uint64_t p;
+              if ((kPolyPairs >> i) & 1u) {
+                p = exp2_poly2(y);
+              } else {
+                float y0, y1;
+                f2unpack(y, y0, y1);
+                p = f2pack(tc05::fast_exp2(y0), tc05::fast_exp2(y1));
+              }
+              acc[i & 3] = f2add(acc[i & 3], p);
+              float p0, p1;
+              f2unpack(p, p0, p1);
+              pk[i] = pack_p(p0, p1);  // key 2i in the low half
+            }
+            float s0, s1;
+            f2unpack(f2add(f2add(acc[0], acc[1]), f2add(acc[2], acc[3])), s0, s1);
+            float csum = s0 + s1;
+            const bool up = !(csum <= kChunkSumLimit);
             if (__any_sync(FULL, up)) {
+              float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+              for (int i = 0; i < 32; i += 2)
+                cm[(i >> 1) & 3] = fmaxf(cm[(i >> 1) & 3], fmaxf(__uint_as_float(x[h2][i]), __uint_as_float(x[h2][i + 1])));
+              const float m_c = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * c;
               const float m_new = up ? m_c : m_ref;
               const float alpha = up ? tc05::fast_exp2(m_ref - m_new) : 1.f;
               l *= alpha;
-#pragma unroll
-              for (int u = 0; u < 8; ++u) sum8[u] *= alpha;
               if (j > 0) {  // O holds P V of key tiles < j (S_w of tile j followed P_w V_{j-1})
 #pragma unroll
                 for (int qo = 0; qo < 4; ++qo) {
@@ -371,32 +462,31 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
                 }
               }
               for (int qp2 = 0; qp2 < q; ++qp2) {  // P chunks of this tile already written
-                uint32_t pk[16];
-                tmem_ld16(tS + 16 * qp2, pk);
+                uint32_t pw[16];
+                tmem_ld16(tS + 16 * qp2, pw);
                 tc05::tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                  const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
-                  pk[i] = pack_bf16(__low2float(v) * alpha, __high2float(v) * alpha);
+                  const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pw[i]);
+                  pw[i] = pack_p(__low2float(v) * alpha, __high2float(v) * alpha);
                 }
-                tmem_st16(tS + 16 * qp2, pk);
+                tmem_st16(tS + 16 * qp2, pw);
               }
               tc05::tmem_wait_st();
               m_ref = m_new;
-            }
-            uint32_t pk[16];
+              csum = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i]), c, -m_ref));
-              const float p1 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i + 1]), c, -m_ref));
-              sum8[(2 * i) & 7] += p0;
-              sum8[(2 * i + 1) & 7] += p1;
-              pk[i] = pack_bf16(p0, p1);  // key 2i in the low half
+              for (int i = 0; i < 16; ++i) {
+                const float p0 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i]), c, -m_ref));
+                const float p1 = tc05::fast_exp2(fmaf(__uint_as_float(x[h2][2 * i + 1]), c, -m_ref));
+                csum += p0 + p1;
+                pk[i] = pack_p(p0, p1);
+              }
             }
+            l += csum;
             tmem_st16(tS + 16 * q, pk);
           }
         }
-        l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         tc05::tmem_wait_st();
         tc05::fence_before_sync();
         __syncwarp();

@@ -20,6 +20,7 @@
 // consume (warp w: query rows 16 (w & 1) .., keys (w >> 1) * tile / 4 .. of each tile), warp
 // 8 lane 0 issues TMA loads into the ring and a 2-slot Q buffer.
 #include "launch.h"
+#include "tcgen05.cuh"
 
 namespace wam {
 namespace {
@@ -442,6 +443,414 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
   if (bad && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
 }
 
+// ============================================================================================
+// The same read on the sm_100 tensor cores, for 128-key tiles (T % 128 == 0).  It is written
+// transposed so that the 128-row MMA is filled by keys rather than by the 32 queries:
+//   S^T = K Q^T    M = 128 keys, N = 32 queries, K = D; both operands K-major in shared memory;
+//   O^T += V^T P^T M = D = 128, N = 64 (32 query columns of P_hi, 32 of P_lo), K = 128 keys;
+//                  V^T is the MN-major view of the V tile as TMA wrote it, P^T a tile of
+//                  128-byte rows.
+// S^T (two buffers) and O^T live in tensor memory.  One softmax thread per key reads its 32
+// scores; each query keeps one reference max, shared by all threads, that moves (with O^T and
+// the row sums rescaled) only when a tile exceeds it by more than 2^16, which one OR-reduction
+// barrier per tile detects.
+//
+// Work split: one thread-block cluster of k <= 8 CTAs per (episode, head); CTA r of the
+// cluster streams the r-th of k contiguous slices of the (episode, head)'s tiles (the action
+// tile first, then the valid frames' tiles).  The k partials (O, m, l) meet in distributed
+// shared memory: after a cluster barrier CTA r merges query rows [r n_act / k, (r+1) n_act / k)
+// by reading its peers' partials, so no partial leaves the chip.
+// Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-5 softmax (TMEM lane quarters 2, 3, 0, 1).
+namespace um {
+constexpr int kKeys = 128;
+constexpr int kTile = kKeys * 128 * 2;   // one of K or V: 32 KB
+constexpr int kStages = 3;
+constexpr int kQ = 32 * 128 * 2;         // 8 KB
+constexpr int kP = kKeys * 128;          // P^T: 128 keys x (32 P_hi + 32 P_lo) bf16 = 16 KB
+constexpr int kThreads = 6 * 32;
+constexpr uint32_t kTmemCols = 128;      // S^T buffers at columns 0 and 32, O^T at 64
+constexpr float kLazy = 16.f;            // reference headroom (log2 units): P <= 2^16
+constexpr int kMaxSplit = 8;             // portable cluster size
+struct Bars {
+  uint64_t kvfull[kStages], kvempty[kStages];
+  uint64_t qfull, sfull[2], sfree[2], pfull, pfree, ofull, done;
+  uint32_t tmem_base;
+  int abort;
+  float red[4][32];
+  float part_m[32], part_l[32];  // this CTA's partial: reference max and row sum per query
+};
+constexpr int kSmemBytes = 1024 + kQ + kStages * 2 * kTile + kP + int(sizeof(Bars)) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(32 * 128 * 4 == kP, "the partial O [32][128] fp32 reuses the P^T buffer");
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 31u && *abort) return false;
+  }
+  *abort = 1;
+  return false;
+}
+// Named barrier 1 over the 128 softmax threads, and the same barrier with an OR-reduction.
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool softmax_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n barrier.red.or.pred p, 1, 128, q;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
+}
+// Every thread of every CTA of the cluster; shared-memory writes before it are visible after.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// A float in CTA `peer`'s shared memory at the offset of `local` in this CTA's.
+__device__ __forceinline__ float ld_peer(const float* local, uint32_t peer) {
+  uint32_t pa;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(pa) : "r"(smem_u32(local)), "r"(peer));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(pa) : "memory");
+  return v;
+}
+// After the call lane q holds the max (or sum) over the warp's lanes of v[q]; v is clobbered.
+template <bool kMax>
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool hi = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = hi ? v[i] : v[i + off];
+      const float keep = hi ? v[i + off] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+}  // namespace um
+
+__global__ void __launch_bounds__(um::kThreads, 1)
+action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
+  using namespace um;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  auto sK = [&](int st) { return base + kQ + st * 2 * kTile; };
+  auto sV = [&](int st) { return base + kQ + st * 2 * kTile + kTile; };
+  uint8_t* sP = base + kQ + kStages * 2 * kTile;
+  um::Bars& bars = *reinterpret_cast<um::Bars*>(sP + kP);
+  volatile int* abort = &bars.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned FULL = 0xffffffffu;
+  // this CTA's slice [t0, t1) of the tiles of (b, h): tile 0 the action keys, tile 1 + v the
+  // v-th 128-key tile of b's valid frames
+  const int k = a.ksplit;
+  const int bh = int(blockIdx.x) / k, rank = int(blockIdx.x) % k;
+  const int b = bh / a.H, h = bh % a.H;
+  const int tpf = a.T / kKeys;
+  const int nb = tiles_of<kKeys>(a, b);
+  const int t0 = rank * nb / k, t1 = (rank + 1) * nb / k, n = t1 - t0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&bars.kvfull[i], 1);
+      mbar_init(&bars.kvempty[i], 1);
+    }
+    mbar_init(&bars.qfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.sfull[i], 1);
+      mbar_init(&bars.sfree[i], 4);
+    }
+    mbar_init(&bars.pfull, 4);
+    mbar_init(&bars.pfree, 1);
+    mbar_init(&bars.ofull, 1);
+    mbar_init(&bars.done, 1);
+    bars.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc05::tmem_alloc(&bars.tmem_base, kTmemCols);
+    tc05::tmem_relinquish();
+  }
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0 && n > 0) {
+      mbar_arrive_expect_tx(&bars.qfull, kQ);
+      tma_load_4d(sQ, &maps.q, &bars.qfull, 0, h, 0, b);
+      tma_load_4d(sQ + kQ / 2, &maps.q, &bars.qfull, 64, h, 0, b);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % kStages, t = t0 + i;
+        if (i >= kStages && !wait_or_abort(&bars.kvempty[st], ((i / kStages) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars.kvfull[st], 2 * kTile);
+        const CUtensorMap *mk, *mv;
+        int tok;
+        if (t == 0) {
+          mk = &maps.ka, mv = &maps.va, tok = 0;
+        } else {
+          const int vt = t - 1;
+          mk = &maps.fk, mv = &maps.fv;
+          tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
+        }
+        tma_load_4d(sK(st), mk, &bars.kvfull[st], 0, h, tok, b);
+        tma_load_4d(sK(st) + kTile / 2, mk, &bars.kvfull[st], 64, h, tok, b);
+        tma_load_4d(sV(st), mv, &bars.kvfull[st], 0, h, tok, b);
+        tma_load_4d(sV(st) + kTile / 2, mv, &bars.kvfull[st], 64, h, tok, b);
+        issued = i + 1;
+      }
+      // Loads still in flight land before the CTA leaves (only after an abort can any be).
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait(&bars.kvfull[i % kStages], (i / kStages) & 1);
+      mbar_wait(&bars.qfull, 0);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = tc05::idesc_bf16_f32(128, 32, false, false);
+      const uint32_t idO = tc05::idesc_bf16_f32(128, 64, true, true);
+      auto issue_S = [&](int i) -> bool {
+        const int st = i % kStages;
+        if (!wait_or_abort(&bars.kvfull[st], (i / kStages) & 1, abort)) return false;
+        if (i == 0 && !wait_or_abort(&bars.qfull, 0, abort)) return false;
+        if (i >= 2 && !wait_or_abort(&bars.sfree[i & 1], ((i >> 1) - 1) & 1, abort)) return false;
+        tc05::fence_after_sync();
+        const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc05::mma_ss(tmem + 32 * (i & 1),
+                       tc05::smem_desc_sw128(k_s + (kk >> 2) * (kTile / 2) + (kk & 3) * 32, 16, 1024),
+                       tc05::smem_desc_sw128(q_s + (kk >> 2) * (kQ / 2) + (kk & 3) * 32, 16, 1024), idS,
+                       kk > 0 ? 1u : 0u);
+        tc05::mma_commit(&bars.sfull[i & 1]);
+        return true;
+      };
+      bool ok = n > 0 && issue_S(0);
+      for (int i = 0; ok && i < n; ++i) {
+        if (!wait_or_abort(&bars.pfull, i & 1, abort)) break;
+        tc05::fence_after_sync();
+        const int st = i % kStages;
+        const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc05::mma_ss(tmem + 64, tc05::smem_desc_sw128(v_s + kk * 2048, kTile / 2, 1024),
+                       tc05::smem_desc_sw128(p_s + kk * 2048, kTile / 2, 1024), idO,
+                       (i > 0 || kk > 0) ? 1u : 0u);
+        tc05::mma_commit(&bars.pfree);
+        tc05::mma_commit(&bars.kvempty[st]);
+        if (i == n - 1) tc05::mma_commit(&bars.ofull);
+        if (i + 1 < n) ok = issue_S(i + 1);
+      }
+      tc05::mma_commit(&bars.done);  // arrives once every MMA issued above has completed
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax, one key per thread
+    // Every wait in front of a warp-collective instruction is voted across the warp, and all
+    // four warps run the same sequence of named barriers whatever happens, so after a timeout
+    // they keep walking their tiles without doing work and no barrier waits on a warp that left.
+    const int quarter = warp & 3;
+    const int L = 32 * quarter + lane;  // key of the tile (S^T lane) and column d of O (O^T lane)
+    const uint32_t lane_off = uint32_t(32 * quarter) << 16;
+    const int wr = warp - 2;            // this warp's row of bars.red
+    const float c = a.scale_log2;
+    bool ok = true;
+    float m[32], l[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) m[q] = -INFINITY, l[q] = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const int t = t0 + i;
+      ok = __all_sync(FULL, ok && wait_or_abort(&bars.sfull[i & 1], (i >> 1) & 1, abort));
+      uint32_t sr[32];
+      if (ok) {
+        tc05::fence_after_sync();
+        tc05::tmem_ld32(tmem + 32 * (i & 1) + lane_off, sr);
+        tc05::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) sr[q] = 0u;
+      }
+      tc05::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.sfree[i & 1]);
+      const bool kv = t != 0 || L < a.n_act;  // keys past n_act in the action tile are padding
+      float ymax = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));
+      if (softmax_any(ok && kv && !(ymax <= kLazy))) {
+        // Some query's reference must move: the tile's max per query over its valid keys.
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = kv ? __uint_as_float(sr[q]) * c : -INFINITY;
+        bars.red[wr][lane] = reduce_scatter32<true>(v, lane);
+        softmax_sync();
+        float al[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const float tm = fmaxf(fmaxf(bars.red[0][q], bars.red[1][q]), fmaxf(bars.red[2][q], bars.red[3][q]));
+          const float mn = tm > m[q] + kLazy ? tm : m[q];
+          al[q] = tc05::fast_exp2(m[q] - mn);  // 0 when m was -inf, 1 when it stays
+          l[q] *= al[q];
+          m[q] = mn;
+        }
+        if (i > 0) {  // O^T holds the P V of the earlier tiles: rescale it
+          ok = __all_sync(FULL, ok && wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
+          if (ok) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // the P_hi and P_lo column blocks
+              uint32_t o[32];
+              tc05::tmem_ld32(tmem + 64 + 32 * half + lane_off, o);
+              tc05::tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
+              tc05::tmem_st32(tmem + 64 + 32 * half + lane_off, o);
+            }
+            tc05::tmem_wait_st();
+          }
+        }
+        softmax_sync();  // bars.red is rewritten by the next tile
+      }
+      // P = P_hi + P_lo, both bf16: query columns 0-31 of the P^T row hold P_hi and columns
+      // 32-63 P_lo, so the one N = 64 MMA accumulates both and O^T's two column halves add up
+      // to P V with P carried to ~16 significant bits (the cache itself is bf16 already).
+      uint32_t pk[16], pl[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j]), c, -m[2 * j])) : 0.f;
+        const float p1 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -m[2 * j + 1])) : 0.f;
+        l[2 * j] += p0, l[2 * j + 1] += p1;
+        pk[j] = pack_bf16(p0, p1);  // query 2j in the low half
+        pl[j] = pack_bf16(p0 - __uint_as_float(pk[j] << 16), p1 - __uint_as_float(pk[j] & 0xffff0000u));
+      }
+      // P^T row L (the 128-byte-swizzled layout the MMA descriptor names) once P V of the
+      // previous tile has read the buffer.
+      if (i > 0) ok = __all_sync(FULL, ok && wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
+      if (ok) {
+        uint8_t* row = sP + L * 128;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          *reinterpret_cast<uint4*>(row + ((ch ^ (L & 7)) << 4)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(row + (((ch + 4) ^ (L & 7)) << 4)) =
+              make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+        }
+      }
+      tc05::fence_proxy_async_smem();  // P^T (generic stores) and O^T (tcgen05.st) before the MMA
+      tc05::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.pfull);
+    }
+    // ---- slice done: O^T column d = L of this thread and the row sums over all 128 keys
+    float o[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) o[q] = 0.f;
+    if (n > 0) {
+      ok = __all_sync(FULL, ok && wait_or_abort(&bars.ofull, 0, abort));
+      if (ok) {
+        uint32_t ohi[32], olo[32];
+        tc05::fence_after_sync();
+        tc05::tmem_ld32(tmem + 64 + lane_off, ohi);
+        tc05::tmem_ld32(tmem + 96 + lane_off, olo);
+        tc05::tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
+      }
+    }
+    {
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = l[q];
+      bars.red[wr][lane] = reduce_scatter32<false>(v, lane);
+    }
+    softmax_sync();
+    float lt[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
+    if (k == 1) {
+      // the whole (b, h) in this CTA: O = O^T / l
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        if (q >= a.n_act) continue;
+        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
+        const float val = o[q] / lt[q];
+        if (a.o_f32) static_cast<float*>(a.o)[off] = val;
+        else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
+      }
+    } else {
+      // the partial into this CTA's shared memory (the P^T buffer is free: every P V is done)
+      float* part = reinterpret_cast<float*>(sP);  // [32 queries][128]
+#pragma unroll
+      for (int q = 0; q < 32; ++q) part[q * 128 + L] = o[q];
+      if (wr == 0) {
+        float mm = -INFINITY, ll = 0.f;
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (q == lane) mm = m[q], ll = lt[q];
+        bars.part_m[lane] = mm;
+        bars.part_l[lane] = ll;
+      }
+    }
+  }
+
+  if (k > 1) {
+    // ---------------------------------------------------------------- merge over the cluster
+    __syncwarp();
+    cluster_sync_all();  // every CTA's partial is in its shared memory
+    if (warp >= 2) {
+      const int L = 32 * (warp & 3) + lane;
+      const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k;
+      const float* part = reinterpret_cast<const float*>(sP);
+      for (int q = r0; q < r1; ++q) {
+        float pm[kMaxSplit], pl_[kMaxSplit], po[kMaxSplit];
+#pragma unroll
+        for (int p = 0; p < kMaxSplit; ++p) {
+          if (p >= k) continue;
+          pm[p] = ld_peer(&bars.part_m[q], uint32_t(p));
+          pl_[p] = ld_peer(&bars.part_l[q], uint32_t(p));
+          po[p] = ld_peer(part + q * 128 + L, uint32_t(p));
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int p = 0; p < kMaxSplit; ++p)
+          if (p < k) M = fmaxf(M, pm[p]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int p = 0; p < kMaxSplit; ++p) {
+          if (p >= k) continue;
+          const float wgt = exp2f(pm[p] - Mu);
+          num = fmaf(wgt, po[p], num);
+          den = fmaf(wgt, pl_[p], den);
+        }
+        const float val = den > 0.f ? num / den : 0.f;
+        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
+        if (a.o_f32) static_cast<float*>(a.o)[off] = val;
+        else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncwarp();
+  tc05::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    mbar_wait(&bars.done, 0);  // every MMA has completed (bounded)
+    tc05::fence_after_sync();
+    tc05::tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars.abort && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
+}
+
 // Action self-attention of a layer outside the interaction set (no video buffer): one CTA of
 // two warps per (episode, head), the n_act <= 32 action keys staged with cp.async into padded
 // shared memory rows (272 B pitch: conflict-free ldmatrix), one softmax per row in registers.
@@ -591,12 +1000,46 @@ size_t action_tc_workspace_bytes(int BH, int max_parts) {
   return kTicketBytes + size_t(BH) * max_parts * kSlotFloats * sizeof(float);
 }
 
+// CTAs per (episode, head) of the cluster read: as many as the SMs allow (at most 8, the
+// portable cluster size) while all B*H clusters still fit on the GPU at once.  The number of
+// co-resident clusters of each size is asked of the runtime once per device.
+static int umma_split(int BH, int dev) {
+  static int max_clusters[32][um::kMaxSplit + 1];
+  static bool known[32];
+  if (!known[dev]) {
+    for (int k = 1; k <= um::kMaxSplit; ++k) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(k));
+      cfg.blockDim = dim3(um::kThreads);
+      cfg.dynamicSmemBytes = um::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = unsigned(k);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, action_umma_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      max_clusters[dev][k] = n;
+    }
+    known[dev] = true;
+  }
+  for (int k = um::kMaxSplit; k > 1; --k)
+    if (max_clusters[dev][k] >= BH) return k;
+  return max_clusters[dev][1] > 0 ? 1 : 0;
+}
+
 cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
   if (!a.with_video) {
     action_self_kernel<<<dim3(a.H, a.B), 64, 0, s>>>(a);
     return cudaGetLastError();
   }
   const int bn = action_bn(a);
+  const bool umma = bn == 128;
   ActionMaps maps;
   const int N = a.F * a.T;
   if (!make_tmap_bf16(&maps.q, a.qa, a.B, a.n_act, a.H, 32) ||
@@ -617,10 +1060,29 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(action_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, um::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured |= 1u << dev;
   }
-  if (bn == 128)
+  if (umma) {
+    ActionArgs ac = a;
+    ac.ksplit = umma_split(a.B * a.H, dev);
+    if (ac.ksplit < 1) return cudaErrorUnknown;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(a.B * a.H * ac.ksplit));
+    cfg.blockDim = dim3(um::kThreads);
+    cfg.dynamicSmemBytes = um::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(ac.ksplit);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, action_umma_kernel, ac, maps);
+  } else if (bn == 128)
     action_tc_kernel<128><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
   else
     action_tc_kernel<64><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);

@@ -71,6 +71,7 @@ struct ActionArgs {
   int32_t max_parts;  // workspace slots per (episode, head)
   float* ws_part;     // partial (O, m, l) slots [B*H][max_parts][32*128 + 64]
   int* ws_count;      // arrival tickets [B*H]; zero between calls
+  int32_t ksplit;     // CTAs (one thread-block cluster) per (episode, head) of the cluster read
   float scale_log2;
   int* err;
   FrameLists fl;

@@ -242,6 +242,7 @@ ACTION_CASES = [
     (2, 3, 128, 64, 3, 32, [[0, 0, 0], [1, 1, 0]], "bf16", 1.0, False),   # self-only layer
     (1, 2, 128, 40, 3, 32, [[0, 1, 0]], "bf16", 1.0, True),               # T % 64 != 0
     (1, 2, 128, 64, 3, 48, [[0, 1, 0]], "bf16", 1.0, True),               # n_act > 32
+    (4, 64, 128, 128, 1, 32, [[0]] * 4, "bf16", 1.0, True),               # whole (b, h) per CTA
 ]
 
 
@@ -257,6 +258,23 @@ def test_action_attention(B, H, D, T, F, n_act, pad, dtype, std, video):
     ref = O.action_attention(to64(qa), to64(ka), to64(va), to64(fk) if video else None,
                              to64(fv) if video else None, np.array(pad), T)
     assert_parity(to64(o), ref, dtype, "action O")
+
+
+@pytest.mark.parametrize("n_act", [32, 5])
+def test_action_large_logit_jumps(n_act):
+    # Later key frames score far above earlier ones, so each query's running reference has to
+    # move in the middle of a CTA's run (and the accumulated output be rescaled) several times.
+    B, H, T, F = 1, 6, 128, 8
+    lay = wam.VideoLayout(B, H, 128, T, F)
+    scale = torch.tensor([1.0 + 2.5 * f for f in range(F)], device="cuda").repeat_interleave(T)
+    fk = dev_normal((B, F * T, H, 128), 64, "fk", dtype=torch.float32) * scale[None, :, None, None]
+    fk = fk.to(torch.bfloat16)
+    fv = dev_normal((B, F * T, H, 128), 64, "fv", dtype=torch.bfloat16)
+    qa, ka, va = (dev_normal((B, n_act, H, 128), 64, x, dtype=torch.bfloat16) for x in ("qa", "ka", "va"))
+    o = torch.full((B, n_act, H, 128), SENTINEL, device="cuda")
+    wam.action_attn(lay, fk, fv, qa, ka, va, o)
+    ref = O.action_attention(to64(qa), to64(ka), to64(va), to64(fk), to64(fv), np.zeros((1, F)), T)
+    assert_parity(to64(o), ref, "bf16", "action logit jumps")
 
 
 def test_action_output_in_bf16():

@@ -472,7 +472,7 @@ constexpr uint32_t kTmemCols = 128;      // S^T buffers at columns 0 and 32, O^T
 constexpr float kLazy = 16.f;            // reference headroom (log2 units): P <= 2^16
 constexpr int kMaxSplit = 8;             // portable cluster size
 struct Bars {
-  uint64_t kvfull[kStages], kvempty[kStages];
+  uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t qfull, sfull[2], sfree[2], pfull, pfree, ofull, done;
   uint32_t tmem_base;
   int abort;
@@ -557,8 +557,10 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.kvfull[i], 1);
-      mbar_init(&bars.kvempty[i], 1);
+      mbar_init(&bars.kfull[i], 1);
+      mbar_init(&bars.kempty[i], 1);
+      mbar_init(&bars.vfull[i], 1);
+      mbar_init(&bars.vempty[i], 1);
     }
     mbar_init(&bars.qfull, 1);
     for (int i = 0; i < 2; ++i) {
@@ -583,59 +585,93 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // K and V stream through separate 3-stage rings: a K stage is refilled as soon as its S^T
+    // MMA has completed, a V stage once its P V has.  The two sequences advance independently.
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(&bars.qfull, kQ);
       tma_load_4d(sQ, &maps.q, &bars.qfull, 0, h, 0, b);
       tma_load_4d(sQ + kQ / 2, &maps.q, &bars.qfull, 64, h, 0, b);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int st = i % kStages, t = t0 + i;
-        if (i >= kStages && !wait_or_abort(&bars.kvempty[st], ((i / kStages) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bars.kvfull[st], 2 * kTile);
-        const CUtensorMap *mk, *mv;
-        int tok;
+      auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
+        const int t = t0 + i;
         if (t == 0) {
-          mk = &maps.ka, mv = &maps.va, tok = 0;
+          mp = is_v ? &maps.va : &maps.ka, tok = 0;
         } else {
           const int vt = t - 1;
-          mk = &maps.fk, mv = &maps.fv;
+          mp = is_v ? &maps.fv : &maps.fk;
           tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
         }
-        tma_load_4d(sK(st), mk, &bars.kvfull[st], 0, h, tok, b);
-        tma_load_4d(sK(st) + kTile / 2, mk, &bars.kvfull[st], 64, h, tok, b);
-        tma_load_4d(sV(st), mv, &bars.kvfull[st], 0, h, tok, b);
-        tma_load_4d(sV(st) + kTile / 2, mv, &bars.kvfull[st], 64, h, tok, b);
-        issued = i + 1;
+      };
+      int nk = 0, nv = 0;
+      for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
+        if ((it & 31u) == 31u && *abort) break;
+        if (nk < n && (nk < kStages || mbar_try_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1))) {
+          const int st = nk % kStages;
+          const CUtensorMap* mp;
+          int tok;
+          tile_src(nk, false, mp, tok);
+          mbar_arrive_expect_tx(&bars.kfull[st], kTile);
+          tma_load_4d(sK(st), mp, &bars.kfull[st], 0, h, tok, b);
+          tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, h, tok, b);
+          ++nk;
+        }
+        if (nv < n && (nv < kStages || mbar_try_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))) {
+          const int st = nv % kStages;
+          const CUtensorMap* mp;
+          int tok;
+          tile_src(nv, true, mp, tok);
+          mbar_arrive_expect_tx(&bars.vfull[st], kTile);
+          tma_load_4d(sV(st), mp, &bars.vfull[st], 0, h, tok, b);
+          tma_load_4d(sV(st) + kTile / 2, mp, &bars.vfull[st], 64, h, tok, b);
+          ++nv;
+        }
       }
+      if (nk < n || nv < n) *abort = 1;
       // Loads still in flight land before the CTA leaves (only after an abort can any be).
-      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait(&bars.kvfull[i % kStages], (i / kStages) & 1);
+      for (int i = (nk > kStages ? nk - kStages : 0); i < nk; ++i) mbar_wait(&bars.kfull[i % kStages], (i / kStages) & 1);
+      for (int i = (nv > kStages ? nv - kStages : 0); i < nv; ++i) mbar_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
       mbar_wait(&bars.qfull, 0);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // S^T of up to two tiles ahead is issued as soon as its K tile has landed and its tensor-
+    // memory buffer has been read, while P V of the current tile waits for its P: the softmax
+    // of tile i + 1 never waits for P V of tile i.
     if (lane == 0) {
       const uint32_t idS = tc05::idesc_bf16_f32(128, 32, false, false);
       const uint32_t idO = tc05::idesc_bf16_f32(128, 64, true, true);
-      auto issue_S = [&](int i) -> bool {
-        const int st = i % kStages;
-        if (!wait_or_abort(&bars.kvfull[st], (i / kStages) & 1, abort)) return false;
-        if (i == 0 && !wait_or_abort(&bars.qfull, 0, abort)) return false;
-        if (i >= 2 && !wait_or_abort(&bars.sfree[i & 1], ((i >> 1) - 1) & 1, abort)) return false;
+      auto s_ready = [&](int j) {
+        return mbar_try_wait(&bars.kfull[j % kStages], (j / kStages) & 1) &&
+               (j > 0 || mbar_try_wait(&bars.qfull, 0)) &&
+               (j < 2 || mbar_try_wait(&bars.sfree[j & 1], ((j >> 1) - 1) & 1));
+      };
+      auto issue_S = [&](int j) {
+        const int st = j % kStages;
         tc05::fence_after_sync();
         const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc05::mma_ss(tmem + 32 * (i & 1),
+          tc05::mma_ss(tmem + 32 * (j & 1),
                        tc05::smem_desc_sw128(k_s + (kk >> 2) * (kTile / 2) + (kk & 3) * 32, 16, 1024),
                        tc05::smem_desc_sw128(q_s + (kk >> 2) * (kQ / 2) + (kk & 3) * 32, 16, 1024), idS,
                        kk > 0 ? 1u : 0u);
-        tc05::mma_commit(&bars.sfull[i & 1]);
-        return true;
+        tc05::mma_commit(&bars.sfull[j & 1]);
+        tc05::mma_commit(&bars.kempty[st]);
       };
-      bool ok = n > 0 && issue_S(0);
+      int ns = 0;  // S^T issued for tiles < ns
+      bool ok = true;
       for (int i = 0; ok && i < n; ++i) {
-        if (!wait_or_abort(&bars.pfull, i & 1, abort)) break;
+        bool p_ready = false, v_ready = false;
+        for (uint32_t it = 0;; ++it) {
+          if (ns < n && ns <= i + 2 && s_ready(ns)) issue_S(ns++);
+          if (ns > i) {
+            v_ready = v_ready || mbar_try_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
+            p_ready = v_ready && mbar_try_wait(&bars.pfull, i & 1);
+            if (p_ready) break;
+          }
+          if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
+          if ((it & 31u) == 31u && *abort) { ok = false; break; }
+        }
+        if (!ok) break;
         tc05::fence_after_sync();
         const int st = i % kStages;
         const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP);
@@ -645,9 +681,8 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
                        tc05::smem_desc_sw128(p_s + kk * 2048, kTile / 2, 1024), idO,
                        (i > 0 || kk > 0) ? 1u : 0u);
         tc05::mma_commit(&bars.pfree);
-        tc05::mma_commit(&bars.kvempty[st]);
+        tc05::mma_commit(&bars.vempty[st]);
         if (i == n - 1) tc05::mma_commit(&bars.ofull);
-        if (i + 1 < n) ok = issue_S(i + 1);
       }
       tc05::mma_commit(&bars.done);  // arrives once every MMA issued above has completed
     }

@@ -77,50 +77,62 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// acc[0..3] += v[0..3] at the L2, without a round trip (vector reduction, sm_90+).
+__device__ __forceinline__ void red_add_v4(float* acc, float a0, float a1, float a2, float a3) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a0), "f"(a1), "f"(a2),
+               "f"(a3)
+               : "memory");
+}
+
 // Store the CTA's own new K or V rows into the layer's cache and fold them into the fusion
 // accumulator, straight from the call's input (64 threads, `rows` tokens from row0_in of the
-// input to row0_out of the cache).  Each thread keeps 4 chunks of 8 elements in flight.
+// input to row0_out of the cache).  The first layer of an interval writes w x, a middle layer
+// adds w x by L2 reductions (nothing to wait for), the last reads the sum and writes the fused
+// bf16 pair.  Each thread keeps 4 chunks of 8 elements in flight (more measured slower).
 __device__ __forceinline__ void store_fuse_rows(const PrefillArgs& a, const void* in_base,
                                                 void* store_base, float* acc_base,
                                                 void* fused_base, int64_t row0_in,
                                                 int64_t row0_out, int rows, int h, int t) {
   constexpr int kU = 4;
   const int chunks = rows * 16;
+  const bool need_acc = a.fuse_on && !a.fuse_first && a.fuse_last;
+  const bool middle = a.fuse_on && !a.fuse_first && !a.fuse_last;
   for (int c0 = t; c0 < chunks; c0 += 64 * kU) {
     uint4 raw[kU];
     float4 p0[kU], p1[kU];
     int64_t off[kU];
-    bool live[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int c = c0 + 64 * u, r = c >> 4, cc = (c & 15) * 8;
-      live[u] = c < chunks;
-      if (!live[u]) continue;
+      if (c >= chunks) continue;
       raw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(in_base) +
                                                ((row0_in + r) * a.H + h) * 128 + cc);
       off[u] = ((row0_out + r) * a.H + h) * 128 + cc;
-      if (a.fuse_on && !a.fuse_first) {
+      if (need_acc) {
         p0[u] = *reinterpret_cast<const float4*>(acc_base + off[u]);
         p1[u] = *reinterpret_cast<const float4*>(acc_base + off[u] + 4);
       }
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      if (!live[u]) continue;
+      if (c0 + 64 * u >= chunks) continue;
       if (store_base)
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(store_base) + off[u]) = raw[u];
       if (!a.fuse_on) continue;
       const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
       float s[8];
-      if (a.fuse_first) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = a.fuse_w * __bfloat162float(x[j]);
-      } else {
+      if (need_acc) {
         const float p[8] = {p0[u].x, p0[u].y, p0[u].z, p0[u].w, p1[u].x, p1[u].y, p1[u].z, p1[u].w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) s[j] = fmaf(a.fuse_w, __bfloat162float(x[j]), p[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] = a.fuse_w * __bfloat162float(x[j]);
       }
-      if (a.fuse_last) {
+      if (middle) {
+        red_add_v4(acc_base + off[u], s[0], s[1], s[2], s[3]);
+        red_add_v4(acc_base + off[u] + 4, s[4], s[5], s[6], s[7]);
+      } else if (a.fuse_last) {
         uint4 v;
         v.x = pack_bf16(s[0], s[1]), v.y = pack_bf16(s[2], s[3]);
         v.z = pack_bf16(s[4], s[5]), v.w = pack_bf16(s[6], s[7]);

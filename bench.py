@@ -89,6 +89,7 @@ def algorithmic_work(w: synth.Workload, pad: np.ndarray) -> dict:
     action_bytes = valid_keys * H * D * 2 * 2 * reads + act_qkvo * calls
     fused_read_bytes = valid_keys * H * D * 2 * 2  # one fused pair read
     return {
+        "imag_flops_per_launch": pair * fut_pairs,
         "prefill_flops": flops_hist + flops_fut,
         "prefill_launches": w.L * (1 + n_pass_fut),
         "action_bytes": action_bytes,
@@ -306,6 +307,32 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------------------ this library
 
+# DRAM bytes (read + write) of one imagination-pass prefill launch, from one ncu capture of
+# the same kernel (profiles/prefill_tc_ctx19.2s_imagination.md); None for other workloads.
+IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 79.436e6}
+
+
+def time_fused_read(runner, stream, n=20) -> float:
+    """Mean device time (ms) of one fused-cache action read of the prepared chunk, each launch
+    after a 256 MB write that flushes the L2, timed by CUDA events around the call alone."""
+    fn, args = runner.calls[runner.fused_read_call]
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    ts = []
+    for i in range(n + 3):
+        flush.fill_(float(i))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st = fn(*args)
+        b.record(stream)
+        if st:
+            raise RuntimeError(f"fused read call failed: {st}")
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    return statistics.mean(ts)
+
+
 def run_mine(args, world, rank, local):
     from cached_kv_attention_b200 import chunk as C
     from cached_kv_attention_b200 import wam
@@ -326,7 +353,8 @@ def run_mine(args, world, rank, local):
     launches = runner.launches_per_chunk()
 
     ev = {name: (torch.cuda.Event(enable_timing=True, external=True),
-                 torch.cuda.Event(enable_timing=True, external=True)) for name in ("video", "action")}
+                 torch.cuda.Event(enable_timing=True, external=True))
+          for name in ("history", "imagination", "final", "action")}
     runner.run()  # first call: one-time per-device set-up outside any capture
     torch.cuda.synchronize()
     wam.device_error()
@@ -366,8 +394,10 @@ def run_mine(args, world, rank, local):
             stage_ms[k].append(a.elapsed_time(b))
     wam.device_error()
     ms, value = replica_throughput(total_ms / args.steps, world)
-    video_ms = statistics.mean(stage_ms["video"])
-    action_ms = statistics.mean(stage_ms["action"])
+    st_ms = {k: statistics.mean(v) for k, v in stage_ms.items()}
+    video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"]
+    action_ms = st_ms["action"]
+    fused_ms = time_fused_read(runner, stream)
 
     peaks = {}
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -381,19 +411,27 @@ def run_mine(args, world, rank, local):
     if hbm_peak is None:
         hbm_peak = 6650.0
 
-    prefill_tflops = work["prefill_flops"] / (video_ms * 1e-3) / 1e12
-    action_gbs = work["action_bytes"] / (action_ms * 1e-3) / 1e9
-    roofline = {"bound": "tensor", "achieved": prefill_tflops, "peak": tflops_peak,
-                "unit": "TFLOP/s", "frac": prefill_tflops / tflops_peak, "traffic": None,
-                "kernel": "wam_video_prefill_kv (tensor-core prefill)",
+    # Dominant kernel: the imagination-pass prefill (4 passes x L layers per chunk, the largest
+    # share of the step).  Its launch time is the imagination stage over its prefill launches
+    # (the stage's four Euler launches, ~3 us each, are included).
+    n_imag = w.n_video_steps * w.L
+    imag_ms = st_ms["imagination"] / n_imag
+    imag_tflops = work["imag_flops_per_launch"] / (imag_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": imag_tflops, "peak": tflops_peak,
+                "unit": "TFLOP/s", "frac": imag_tflops / tflops_peak,
+                "traffic": IMAG_TRAFFIC_BYTES.get(w0.name),
+                "kernel": "prefill_tc_kernel, imagination pass (wam_video_prefill_kv)",
                 "peak_kind": f"{peak_src} bf16 sustained",
-                "flops_per_launch": work["prefill_flops"] / work["prefill_launches"],
-                "ms_per_launch": video_ms / work["prefill_launches"]}
-    roofline_action = {"bound": "hbm", "achieved": action_gbs, "peak": hbm_peak, "unit": "GB/s",
-                       "frac": action_gbs / hbm_peak, "frac_of_8tbs": action_gbs / 8000.0,
-                       "kernel": "wam_action_attn (all 300 calls of the chunk, 80 fused reads)",
-                       "peak_kind": f"{peak_src} copy bandwidth",
-                       "bytes_per_chunk": work["action_bytes"]}
+                "flops_per_launch": work["imag_flops_per_launch"], "ms_per_launch": imag_ms,
+                "video_stage_tflops": work["prefill_flops"] / (video_ms * 1e-3) / 1e12}
+    fused_bytes = work["fused_read_bytes"] + w.n_act * w.H * w.D * (3 * 2 + 4) * w.B
+    fused_gbs = fused_bytes / (fused_ms * 1e-3) / 1e9
+    roofline_action = {"bound": "hbm", "achieved": fused_gbs, "peak": hbm_peak, "unit": "GB/s",
+                       "frac": fused_gbs / hbm_peak,
+                       "kernel": "action_umma_kernel, one fused-cache read (wam_action_attn)",
+                       "peak_kind": f"{peak_src} copy bandwidth", "bytes_per_launch": fused_bytes,
+                       "ms_per_launch": fused_ms,
+                       "action_stage_gbs": work["action_bytes"] / (action_ms * 1e-3) / 1e9}
 
     e2e = None
     if not args.no_e2e:
@@ -417,7 +455,7 @@ def run_mine(args, world, rank, local):
                        "launch": "cuda graph" if graph is not None else "eager",
                        "l2": "inputs larger than L2: ~25 GB of distinct per-layer buffers per chunk",
                        "parallelism": f"replicas x{world}"},
-            "stage_ms": {"video": video_ms, "action": action_ms},
+            "stage_ms": {**st_ms, "video": video_ms},
             "roofline": roofline,
             "roofline_action": roofline_action,
             "cpu_baseline": cpu,

@@ -154,6 +154,7 @@ class ChunkRunner:
                           (lay, dt, 0, F_h, _vp(inp["hist_q"][l]), _vp(inp["hist_k"][l]),
                            _vp(inp["hist_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
                            o_of(self.hist_o, l), o_dt, self._epilogue(l), s)))
+        hist_end = len(calls)
         # a4: imagination passes + Euler on the future latents
         nf = self.x_future.numel()
         for st in range(w.n_video_steps):
@@ -166,6 +167,7 @@ class ChunkRunner:
             ds = float(self.sig_v[st + 1] - self.sig_v[st])
             calls.append((L.wam_flow_euler_step, (nf, _vp(self.x_future),
                                                   _vp(inp["v_future"][st]), ds, s)))
+        imag_end = len(calls)
         # a5: final pass at sigma*, store future K/V (+ complete the fused pairs)
         for l in range(w.L):
             calls.append((L.wam_video_prefill_kv,
@@ -199,9 +201,13 @@ class ChunkRunner:
             ds = float(self.sig_a[i + 1] - self.sig_a[i])
             calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
         self.calls = calls
-        # stage boundaries (call indices): the video stages a3-a6 (prefill kernels plus four
-        # small Euler steps), then the action stages a7-a8
-        self.stages = [("video", 0, video_end), ("action", video_end, len(calls))]
+        # stage boundaries (call indices): the video stages a3 (history), a4 (imagination passes
+        # and four small Euler steps), a5-a6 (final pass, standalone fusion), then the action
+        # stages a7-a8
+        self.stages = [("history", 0, hist_end), ("imagination", hist_end, imag_end),
+                       ("final", imag_end, video_end), ("action", video_end, len(calls))]
+        self.fused_read_call = next(i for i in range(video_end, len(calls))
+                                    if calls[i][0] is L.wam_action_attn and calls[i][1][2] is not None)
         return self
 
     def reset_latents(self) -> None:

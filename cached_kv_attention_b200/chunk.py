@@ -116,7 +116,9 @@ class ChunkRunner:
         self.act_o = [z(B, w.n_act, H, D, dtype=o_dtype) for _ in range(n_a)]
         self.x_future = inputs["x_future"].clone()
         self.x_act = inputs["x_act"].clone()
-        self.sig_v = wam.flow_schedule(w.n_video_steps, w.sigma_star)
+        # one-shot variant (no video step): the cache pass runs at sigma* directly
+        self.sig_v = (wam.flow_schedule(w.n_video_steps, w.sigma_star) if w.n_video_steps > 0
+                      else [w.sigma_star])
         self.sig_a = wam.flow_schedule(w.n_euler_steps, 0.0)
         self.parts = interval_partition(w.L, w.S)
         self.fw = [wam.fuse_weights(lg.cpu().numpy()) for lg in inputs["fuse_logits"]]

@@ -83,6 +83,14 @@ WORKLOADS = {
     "batched4_bf16": Workload("batched4_bf16", B=4, F_h=24, pad_rule="prefix_unif:21", seed=4,
                               **_BF),
 }
+# Interaction-stride variants of the 19.2 s chunk ("世界模型之Faster-WAM详解" §4.3 ablates strides
+# 1, 2, 4, 7, 14): every layer reads its own K/V (S = 1: one-layer intervals), S = 2, S = 7; and
+# the one-shot variant (§3.1: one video pass at sigma* = 1, no imagination step).
+for _s in (1, 2, 7):
+    WORKLOADS[f"stride{_s}_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
+        name=f"stride{_s}_ctx19.2s_bf16", S=_s)
+WORKLOADS["oneshot_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
+    name="oneshot_ctx19.2s_bf16", n_video_steps=0, sigma_star=1.0)
 
 
 def seed_for(seed: int, name: str, *idx: int) -> int:

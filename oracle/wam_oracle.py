@@ -339,8 +339,10 @@ def chunk(inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int, n_video_step
         k_cache[l] = cache_store(k_cache[l], inp["hist_k"][l], pad, T, 0, F_h)
         v_cache[l] = cache_store(v_cache[l], inp["hist_v"][l], pad, T, 0, F_h)
 
-    # a4: imagination passes and Euler steps on the future latents, sigma 1 -> sigma*
-    sig_v = flow_schedule(n_video_steps, sigma_star)
+    # a4: imagination passes and Euler steps on the future latents, sigma 1 -> sigma*.  With no
+    # video step (the one-shot variant: one video pass at sigma* = 1, [FSW] §3.1) the cache pass
+    # follows directly.
+    sig_v = flow_schedule(n_video_steps, sigma_star) if n_video_steps > 0 else None
     x_future = _f64(inp["x_future"])
     for s in range(n_video_steps):
         outs = []

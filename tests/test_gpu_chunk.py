@@ -70,6 +70,28 @@ def test_tiny_fp32_chunk_end_to_end(fusion):
     _compare_chunk(w, r, ref, pad, None, "f32")
 
 
+@pytest.mark.parametrize("variant", [dict(S=1), dict(S=3), dict(n_video_steps=0, sigma_star=1.0)],
+                         ids=["stride1", "stride3", "one_shot"])
+def test_tiny_fp32_chunk_variants(variant):
+    # The interaction-stride and one-shot variants run the same calls with other S / video steps.
+    w = synth.WORKLOADS["tiny_f32"].replace(seed=8, **variant)
+    r, inp64 = _run_chunk(w)
+    pad = synth.pad_mask(w).numpy()
+    ref = _oracle_chunk(w, inp64, pad)
+    _compare_chunk(w, r, ref, pad, None, "f32")
+
+
+def test_bf16_chunk_stride1_768_token_frames():
+    # Every layer reads its own-layer K/V (S = 1) at the 768-token frame shape, two heads checked.
+    w = synth.WORKLOADS["ctx2.4s_bf16"].replace(L=3, S=1, n_video_steps=1, n_euler_steps=2,
+                                                pad_rule="prefix:1", seed=9)
+    r, inp64 = _run_chunk(w)
+    pad = synth.pad_mask(w).numpy()
+    heads = [3, 20]
+    ref = _oracle_chunk(w, inp64, pad, heads=heads)
+    _compare_chunk(w, r, ref, pad, heads, "bf16")
+
+
 def test_tiny_fp32_chunk_padded_and_grouped_future():
     w = synth.WORKLOADS["tiny_f32"].replace(F_h=3, pad_rule="prefix:1", seed=5)
     blocks = [0, 1, 2, 3, 3]

@@ -86,7 +86,9 @@ typedef struct {
  *   last_in_interval:   fused = round(acc + w * K_j) (acc is read, not written)
  * and the same for V.  A one-layer interval sets both flags.  acc_k/acc_v are caller-owned
  * fp32 device scratch [B, N, H, D]; fused_k/fused_v are device [B, N, H, D] of the call's dtype.
- * The per-layer K/V is folded while it is in on-chip memory and never re-read for fusion.
+ * The fold runs inside the prefill kernel from the call's own K/V input (middle layers add
+ * into acc by L2 reductions), so the stored per-layer cache is never re-read for fusion.
+ * Calls that use the same accumulator must not overlap on the GPU.
  */
 typedef struct {
   float weight;
@@ -152,7 +154,9 @@ wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, in
  *                    arrival ticket per (episode, head) (B * H <= 16384); every call that
  *                    completes leaves them at zero, so one workspace serves calls of any layout
  *                    in turn.  Calls that share a workspace must not overlap on the GPU.  May be
- *                    NULL when the size is 0.
+ *                    NULL when the size is 0.  (The tensor-core read of 128-key tiles,
+ *                    T % 128 == 0, merges its partials on chip and leaves the workspace
+ *                    untouched; the size covers the other paths of the same layout.)
  * Action tokens attend to each other bidirectionally.  Returns WAM_ERR_WORKSPACE if the
  * workspace is missing or too small.
  */

@@ -582,6 +582,14 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = bars.tmem_base;
+  // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
+  // the stream may still be finishing (programmatic dependent launch).
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
+    prefetch_tmap(&maps.fk), prefetch_tmap(&maps.fv);
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -894,6 +902,8 @@ constexpr int kSelfPitch = 128 * 2 + 16;
 __global__ void __launch_bounds__(64)
 action_self_kernel(const __grid_constant__ ActionArgs a) {
   __shared__ __align__(16) uint8_t sm[3][32 * kSelfPitch];
+  grid_dependency_wait();  // programmatic dependent launch: inputs ready from here on
+  grid_launch_dependents();
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const unsigned FULL = 0xffffffffu;
@@ -1070,8 +1080,7 @@ static int umma_split(int BH, int dev) {
 
 cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
   if (!a.with_video) {
-    action_self_kernel<<<dim3(a.H, a.B), 64, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(action_self_kernel, dim3(a.H, a.B), dim3(64), 0, s, 0, a);
   }
   const int bn = action_bn(a);
   const bool umma = bn == 128;
@@ -1104,19 +1113,8 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
     ActionArgs ac = a;
     ac.ksplit = umma_split(a.B * a.H, dev);
     if (ac.ksplit < 1) return cudaErrorUnknown;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(a.B * a.H * ac.ksplit));
-    cfg.blockDim = dim3(um::kThreads);
-    cfg.dynamicSmemBytes = um::kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(ac.ksplit);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, action_umma_kernel, ac, maps);
+    return launch_pdl(action_umma_kernel, dim3(unsigned(a.B * a.H * ac.ksplit)), dim3(um::kThreads),
+                      um::kSmemBytes, s, unsigned(ac.ksplit), ac, maps);
   } else if (bn == 128)
     action_tc_kernel<128><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
   else

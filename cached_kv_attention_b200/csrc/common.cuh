@@ -133,6 +133,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the previous kernel on its stream is still running.  It waits here (until
+// that grid has completed and its memory is visible) before its first global memory access,
+// and lets the next kernel start launching as early as possible.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Bounded wait: returns false if the phase never flips; the caller then records
 // WAM_ERR_TIMEOUT in the device error word (args.err) and leaves without waiting further.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {

@@ -297,6 +297,14 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = bars.tmem_base;
+  // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
+  // the stream may still be finishing (programmatic dependent launch).
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&maps.q), prefetch_tmap(&maps.kn), prefetch_tmap(&maps.vn);
+    prefetch_tmap(&maps.kc), prefetch_tmap(&maps.vc);
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -579,8 +587,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   }
   const int QP = (a.T / kBM + 1) / 2;
   const int64_t grid = int64_t(a.fl.n_items) * QP * a.H;
-  prefill_tc_kernel<<<unsigned(grid), kThreads, kSmemBytes, s>>>(a, maps);
-  return cudaGetLastError();
+  return launch_pdl(prefill_tc_kernel, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);
 }
 
 }  // namespace wam

@@ -38,6 +38,8 @@ static int grid_for(int64_t work, int per_block, int cap) {
 // ------------------------------------------------------------------------------ Euler
 __global__ void euler_kernel(int64_t n, float* __restrict__ x, const float* __restrict__ v,
                              float dsigma) {
+  grid_dependency_wait();  // programmatic dependent launch: inputs ready from here on
+  grid_launch_dependents();
   const int64_t n4 = n >> 2;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   const int64_t i0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -55,8 +57,7 @@ __global__ void euler_kernel(int64_t n, float* __restrict__ x, const float* __re
 
 cudaError_t launch_euler(int64_t n, float* x, const float* v, float dsigma, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  euler_kernel<<<grid_for((n + 3) / 4, 256, 148 * 16), 256, 0, s>>>(n, x, v, dsigma);
-  return cudaGetLastError();
+  return launch_pdl(euler_kernel, dim3(grid_for((n + 3) / 4, 256, 148 * 16)), dim3(256), 0, s, 0, n, x, v, dsigma);
 }
 
 // ------------------------------------------------------------------------------ store + fuse

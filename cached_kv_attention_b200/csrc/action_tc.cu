@@ -612,7 +612,7 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       int nk = 0, nv = 0;
       for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
         if ((it & 31u) == 31u && *abort) break;
-        if (nk < n && (nk < kStages || mbar_try_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1))) {
+        if (nk < n && (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1))) {
           const int st = nk % kStages;
           const CUtensorMap* mp;
           int tok;
@@ -622,7 +622,7 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
           tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, h, tok, b);
           ++nk;
         }
-        if (nv < n && (nv < kStages || mbar_try_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))) {
+        if (nv < n && (nv < kStages || mbar_test_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))) {
           const int st = nv % kStages;
           const CUtensorMap* mp;
           int tok;
@@ -648,9 +648,9 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       const uint32_t idS = tc05::idesc_bf16_f32(128, 32, false, false);
       const uint32_t idO = tc05::idesc_bf16_f32(128, 64, true, true);
       auto s_ready = [&](int j) {
-        return mbar_try_wait(&bars.kfull[j % kStages], (j / kStages) & 1) &&
-               (j > 0 || mbar_try_wait(&bars.qfull, 0)) &&
-               (j < 2 || mbar_try_wait(&bars.sfree[j & 1], ((j >> 1) - 1) & 1));
+        return mbar_test_wait(&bars.kfull[j % kStages], (j / kStages) & 1) &&
+               (j > 0 || mbar_test_wait(&bars.qfull, 0)) &&
+               (j < 2 || mbar_test_wait(&bars.sfree[j & 1], ((j >> 1) - 1) & 1));
       };
       auto issue_S = [&](int j) {
         const int st = j % kStages;
@@ -672,8 +672,8 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
         for (uint32_t it = 0;; ++it) {
           if (ns < n && ns <= i + 2 && s_ready(ns)) issue_S(ns++);
           if (ns > i) {
-            v_ready = v_ready || mbar_try_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
-            p_ready = v_ready && mbar_try_wait(&bars.pfull, i & 1);
+            v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
+            p_ready = v_ready && mbar_test_wait(&bars.pfull, i & 1);
             if (p_ready) break;
           }
           if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
@@ -850,32 +850,40 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       const int L = 32 * (warp & 3) + lane;
       const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k;
       const float* part = reinterpret_cast<const float*>(sP);
-      for (int q = r0; q < r1; ++q) {
-        float pm[kMaxSplit], pl_[kMaxSplit], po[kMaxSplit];
+      // four rows at a time, every peer's (m, l, O) loads of them issued before any is used
+      for (int q0 = r0; q0 < r1; q0 += 4) {
+        float pm[4][kMaxSplit], pl_[4][kMaxSplit], po[4][kMaxSplit];
 #pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p) {
-          if (p >= k) continue;
-          pm[p] = ld_peer(&bars.part_m[q], uint32_t(p));
-          pl_[p] = ld_peer(&bars.part_l[q], uint32_t(p));
-          po[p] = ld_peer(part + q * 128 + L, uint32_t(p));
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int p = 0; p < kMaxSplit; ++p) {
+            if (p >= k || q0 + u >= r1) continue;
+            pm[u][p] = ld_peer(&bars.part_m[q0 + u], uint32_t(p));
+            pl_[u][p] = ld_peer(&bars.part_l[q0 + u], uint32_t(p));
+            po[u][p] = ld_peer(part + (q0 + u) * 128 + L, uint32_t(p));
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u;
+          if (q >= r1) continue;
+          float M = -INFINITY;
+#pragma unroll
+          for (int p = 0; p < kMaxSplit; ++p)
+            if (p < k) M = fmaxf(M, pm[u][p]);
+          const float Mu = M == -INFINITY ? 0.f : M;
+          float num = 0.f, den = 0.f;
+#pragma unroll
+          for (int p = 0; p < kMaxSplit; ++p) {
+            if (p >= k) continue;
+            const float wgt = exp2f(pm[u][p] - Mu);
+            num = fmaf(wgt, po[u][p], num);
+            den = fmaf(wgt, pl_[u][p], den);
+          }
+          const float val = den > 0.f ? num / den : 0.f;
+          const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
+          if (a.o_f32) static_cast<float*>(a.o)[off] = val;
+          else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
         }
-        float M = -INFINITY;
-#pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p)
-          if (p < k) M = fmaxf(M, pm[p]);
-        const float Mu = M == -INFINITY ? 0.f : M;
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p) {
-          if (p >= k) continue;
-          const float wgt = exp2f(pm[p] - Mu);
-          num = fmaf(wgt, po[p], num);
-          den = fmaf(wgt, pl_[p], den);
-        }
-        const float val = den > 0.f ? num / den : 0.f;
-        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
-        if (a.o_f32) static_cast<float*>(a.o)[off] = val;
-        else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
       }
     }
     __syncwarp();

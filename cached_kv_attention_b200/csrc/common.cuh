@@ -144,6 +144,18 @@ __device__ __forceinline__ void grid_dependency_wait() {
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// Non-blocking test of a phase (mbarrier.try_wait may suspend the thread for a while when the
+// phase is not complete; a thread that polls several barriers uses this instead).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait: returns false if the phase never flips; the caller then records
 // WAM_ERR_TIMEOUT in the device error word (args.err) and leaves without waiting further.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {

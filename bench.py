@@ -80,7 +80,8 @@ def algorithmic_work(w: synth.Workload, pad: np.ndarray) -> dict:
                 hist_pairs += sum(1 for g in valid if g <= f)
         for f in range(w.F_h, w.F):
             fut_pairs += sum(1 for g in valid if g <= f)
-    n_pass_fut = w.n_video_steps + 1
+    # future-frame passes: the imagination steps and the cache pass, or one per joint step
+    n_pass_fut = w.n_euler_steps if w.joint else w.n_video_steps + 1
     flops_hist = pair * hist_pairs * w.L
     flops_fut = pair * fut_pairs * w.L * n_pass_fut
     act_qkvo = w.n_act * H * D * (3 * 2 + 4) * w.B
@@ -208,9 +209,12 @@ def oracle_sample_seconds(w: synth.Workload, pad: np.ndarray, n_heads: int, n_la
     hq = [g("hq", hist, l) for l in layers]
     hk = [g("hk", hist, l) for l in layers]
     hv = [g("hv", hist, l) for l in layers]
-    iq = [[g("iq", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
-    ik = [[g("ik", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
-    iv = [[g("iv", fut, s, l) for l in layers] for s in range(w.n_video_steps + 1)]
+    # future-frame passes: imagination steps + the cache pass, or one per joint step (the
+    # co-denoising chunk does the same work in another order)
+    n_fut = w.n_euler_steps if w.joint else w.n_video_steps + 1
+    iq = [[g("iq", fut, s, l) for l in layers] for s in range(n_fut)]
+    ik = [[g("ik", fut, s, l) for l in layers] for s in range(n_fut)]
+    iv = [[g("iv", fut, s, l) for l in layers] for s in range(n_fut)]
     aq = [[g("aq", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
     ak = [[g("ak", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
     av = [[g("av", w.n_act, i, l) for l in layers] for i in range(w.n_euler_steps)]
@@ -226,12 +230,13 @@ def oracle_sample_seconds(w: synth.Workload, pad: np.ndarray, n_heads: int, n_la
     rows_f = np.arange(0, fut, row_stride)
     for l in layers:
         O.video_prefill(hq[l], hk[l], hv[l], None, None, pad, None, T, 0, w.F_h, rows=rows_h)
-    sv = O.flow_schedule(w.n_video_steps, w.sigma_star)
-    for s in range(w.n_video_steps + 1):
+    n_ode = n_fut if w.joint else w.n_video_steps
+    sv = O.flow_schedule(n_ode, 0.0 if w.joint else w.sigma_star) if n_ode > 0 else None
+    for s in range(n_fut):
         for l in layers:
             O.video_prefill(iq[s][l], ik[s][l], iv[s][l], kc[l], vc[l], pad, None, T, w.F_h, w.F,
                             rows=rows_f)
-        if s < w.n_video_steps:
+        if s < n_ode:
             xf = O.euler_step(xf, vf, sv[s + 1] - sv[s])
     for l in layers:
         kc[l] = O.cache_store(kc[l], ik[-1][l], pad, T, w.F_h, w.F)
@@ -365,7 +370,7 @@ def run_mine(args, world, rank, local):
 
     ev = {name: (torch.cuda.Event(enable_timing=True, external=True),
                  torch.cuda.Event(enable_timing=True, external=True))
-          for name in ("history", "imagination", "final", "action")}
+          for name, _, _ in runner.stages}
     runner.run()  # first call: one-time per-device set-up outside any capture
     torch.cuda.synchronize()
     wam.device_error()
@@ -406,7 +411,13 @@ def run_mine(args, world, rank, local):
     wam.device_error()
     ms, value = replica_throughput(total_ms / args.steps, world)
     st_ms = {k: statistics.mean(v) for k, v in stage_ms.items()}
-    video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"]
+    if w.joint:  # co-denoising: per joint step a video stage (future passes) and an action stage
+        fut_ms = sum(v for k, v in st_ms.items() if k.startswith("video"))
+        st_ms = {"history": st_ms["history"], "joint_video": fut_ms,
+                 "action": sum(v for k, v in st_ms.items() if k.startswith("action"))}
+        video_ms = st_ms["history"] + fut_ms
+    else:
+        video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"]
     action_ms = st_ms["action"]
     fused_ms = time_fused_read(runner, stream)
 
@@ -427,11 +438,12 @@ def run_mine(args, world, rank, local):
     # (the stage's four Euler launches, ~3 us each, are included).
     # (With no imagination step, the one-shot variant, the final pass stands in: same shape,
     # plus the cache store and fusion epilogue.)
-    pass_name = "imagination" if w.n_video_steps > 0 else "final"
-    n_imag = w.n_video_steps * w.L if w.n_video_steps > 0 else w.L
+    pass_name = ("joint_video" if w.joint else "imagination" if w.n_video_steps > 0 else "final")
+    n_imag = (w.n_euler_steps * w.L if w.joint else
+              w.n_video_steps * w.L if w.n_video_steps > 0 else w.L)
     imag_ms = st_ms[pass_name] / n_imag
     imag_tflops = work["imag_flops_per_launch"] / (imag_ms * 1e-3) / 1e12
-    same_launch = (w.n_video_steps > 0 and
+    same_launch = (w.n_video_steps > 0 and not w.joint and
                    w0.replace(name="ctx19.2s_bf16", S=4) == synth.WORKLOADS["ctx19.2s_bf16"])
     roofline = {"bound": "tensor", "achieved": imag_tflops, "peak": tflops_peak,
                 "unit": "TFLOP/s", "frac": imag_tflops / tflops_peak,
@@ -527,7 +539,7 @@ def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
     for name in ("hist_q", "hist_k", "hist_v"):
         for l, t in enumerate(inp[name]):
             add(name, t, l % 2, runs)
-    for name in ("imag_q", "imag_k", "imag_v", "act_q", "act_k", "act_v"):
+    for name in ("imag_q", "imag_k", "imag_v", "act_q", "act_k", "act_v", "joint_q", "joint_k", "joint_v"):
         for i, row in enumerate(inp[name]):
             for l, t in enumerate(row):
                 add(name, t, (i + l) % 2)

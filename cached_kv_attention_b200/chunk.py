@@ -59,9 +59,16 @@ def make_inputs(w: Workload, device: str = "cpu") -> Dict:
         "imag_q": [[qkv("imag_q", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
         "imag_k": [[qkv("imag_k", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
         "imag_v": [[qkv("imag_v", fut, s, l) for l in range(w.L)] for s in range(w.n_video_steps)],
-        "final_q": [qkv("final_q", fut, l) for l in range(w.L)],
-        "final_k": [qkv("final_k", fut, l) for l in range(w.L)],
-        "final_v": [qkv("final_v", fut, l) for l in range(w.L)],
+        "final_q": [qkv("final_q", fut, l) for l in range(w.L)] if not w.joint else [],
+        "final_k": [qkv("final_k", fut, l) for l in range(w.L)] if not w.joint else [],
+        "final_v": [qkv("final_v", fut, l) for l in range(w.L)] if not w.joint else [],
+        # co-denoising: the future frames' Q/K/V at every joint step
+        "joint_q": [[qkv("joint_q", fut, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)]
+                   if w.joint else [],
+        "joint_k": [[qkv("joint_k", fut, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)]
+                   if w.joint else [],
+        "joint_v": [[qkv("joint_v", fut, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)]
+                   if w.joint else [],
         "fuse_logits": [synth.normal((len(I),), w.seed, "fuse_logits", m)
                         for m, I in enumerate(interval_partition(w.L, w.S))],
         "act_q": [[qkv("act_q", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
@@ -69,7 +76,7 @@ def make_inputs(w: Workload, device: str = "cpu") -> Dict:
         "act_v": [[qkv("act_v", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
         "x_future": synth.normal((B, fut, w.C), w.seed, "x_future", device=device),
         "v_future": [synth.normal((B, fut, w.C), w.seed, "v_future", s, device=device)
-                     for s in range(w.n_video_steps)],
+                     for s in range(w.n_euler_steps if w.joint else w.n_video_steps)],
         "x_act": synth.normal((B, w.n_act, w.A), w.seed, "x_act", device=device),
         "v_act": [synth.normal((B, w.n_act, w.A), w.seed, "v_act", i, device=device)
                   for i in range(w.n_euler_steps)],
@@ -114,6 +121,9 @@ class ChunkRunner:
         self.final_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_h)]
         self.imag_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_i)]
         self.act_o = [z(B, w.n_act, H, D, dtype=o_dtype) for _ in range(n_a)]
+        if w.joint and fusion != "epilogue":
+            raise ValueError("co-denoising chunks fold the fusion into the future passes (epilogue)")
+        self.joint_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_a if w.joint else 0)]
         self.x_future = inputs["x_future"].clone()
         self.x_act = inputs["x_act"].clone()
         # one-shot variant (no video step): the cache pass runs at sigma* directly
@@ -157,6 +167,8 @@ class ChunkRunner:
                            _vp(inp["hist_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
                            o_of(self.hist_o, l), o_dt, self._epilogue(l), s)))
         hist_end = len(calls)
+        if w.joint:
+            return self._prepare_joint(calls, hist_end, lay, dt, o_dt, s, o_of)
         # a4: imagination passes + Euler on the future latents
         nf = self.x_future.numel()
         for st in range(w.n_video_steps):
@@ -209,6 +221,41 @@ class ChunkRunner:
         self.stages = [("history", 0, hist_end), ("imagination", hist_end, imag_end),
                        ("final", imag_end, video_end), ("action", video_end, len(calls))]
         self.fused_read_call = next(i for i in range(video_end, len(calls))
+                                    if calls[i][0] is L.wam_action_attn and calls[i][1][2] is not None)
+        return self
+
+    def _prepare_joint(self, calls, hist_end, lay, dt, o_dt, s, o_of) -> "ChunkRunner":
+        """Co-denoising: at every joint step i the future frames are passed through all layers
+        (their K/V stored into the caches and folded into the fused pairs by the epilogue), then
+        the action layers read, then both latents take one Euler step on the shared schedule."""
+        w, L, inp, F_h, F = self.w, wam.lib, self.inp, self.w.F_h, self.w.F
+        sig = wam.flow_schedule(w.n_euler_steps, 0.0)
+        reader = {j: m for m, j in enumerate(interaction_layers(w.L, w.S))}
+        nf, na = self.x_future.numel(), self.x_act.numel()
+        self.stages = [("history", 0, hist_end)]
+        for i in range(w.n_euler_steps):
+            v0 = len(calls)
+            for l in range(w.L):
+                calls.append((L.wam_video_prefill_kv,
+                              (lay, dt, F_h, F, _vp(inp["joint_q"][i][l]), _vp(inp["joint_k"][i][l]),
+                               _vp(inp["joint_v"][i][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]),
+                               1, o_of(self.joint_o, i * w.L + l), o_dt, self._epilogue(l), s)))
+            a0 = len(calls)
+            for l in range(w.L):
+                m = reader.get(l)
+                fk = _vp(self.fused_k[m]) if m is not None else None
+                fv = _vp(self.fused_v[m]) if m is not None else None
+                calls.append((L.wam_action_attn,
+                              (lay, dt, fk, fv, w.n_act, _vp(inp["act_q"][i][l]),
+                               _vp(inp["act_k"][i][l]), _vp(inp["act_v"][i][l]),
+                               o_of(self.act_o, i * w.L + l), o_dt, _vp(self.workspace),
+                               self.workspace.numel(), s)))
+            ds = float(sig[i + 1] - sig[i])
+            calls.append((L.wam_flow_euler_step, (nf, _vp(self.x_future), _vp(inp["v_future"][i]), ds, s)))
+            calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
+            self.stages += [(f"video{i}", v0, a0), (f"action{i}", a0, len(calls))]
+        self.calls = calls
+        self.fused_read_call = next(i for i in range(hist_end, len(calls))
                                     if calls[i][0] is L.wam_action_attn and calls[i][1][2] is not None)
         return self
 

@@ -48,6 +48,7 @@ class Workload:
     A: int               # action dim (RoboTwin: 14)
     pad_rule: str        # "none" | "prefix:<P>" | "prefix_frac:<pmax>" | "prefix_unif:<Pmax>"
     seed: int
+    joint: bool = False  # co-denoising: the future frames are re-passed at every action step
 
     @property
     def F(self) -> int:
@@ -91,6 +92,11 @@ for _s in (1, 2, 7):
         name=f"stride{_s}_ctx19.2s_bf16", S=_s)
 WORKLOADS["oneshot_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
     name="oneshot_ctx19.2s_bf16", n_video_steps=0, sigma_star=1.0)
+# Co-denoising (CoD, "Long-WAM ... | Summary" App. F: V4/A4): video and actions denoised
+# together in 4 joint steps; every step re-passes the future frames (cache store and fusion)
+# before its action reads.
+WORKLOADS["cod4_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
+    name="cod4_ctx19.2s_bf16", joint=True, n_video_steps=0, n_euler_steps=4, sigma_star=0.0)
 
 
 def seed_for(seed: int, name: str, *idx: int) -> int:

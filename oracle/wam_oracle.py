@@ -49,7 +49,7 @@ __all__ = [
     "block_ids", "video_allowed", "action_key_allowed",
     "masked_attention", "video_prefill", "cache_store",
     "interval_partition", "interaction_layers", "fuse_weights", "fuse_interval",
-    "action_attention", "chunk",
+    "action_attention", "chunk", "chunk_joint",
 ]
 
 
@@ -385,4 +385,65 @@ def chunk(inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int, n_video_step
         out["act_o"].append(outs)
         x_act = euler_step(x_act, inp["v_act"][i], sig_a[i + 1] - sig_a[i])
     out["x_act"] = x_act
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Co-denoising (CoD) chunk            [LW-sum] Fig. 2 and App. F (IDM versus co-denoising,
+#                                     V4/A4); [FSW] §1-2 (Joint-WAM updates the future video
+#                                     and the actions at every denoising step)
+# --------------------------------------------------------------------------------------
+
+def chunk_joint(inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int, n_steps: int, pad,
+                frame_block=None, heads: Optional[Sequence[int]] = None) -> Dict:
+    """One chunk with video and actions denoised together in ``n_steps`` joint steps.
+
+    Reading R10 (the pages give the idea and latencies, not the step order): the history pass
+    runs once; at joint step i every layer first passes the future frames (queries over the
+    cached history and the step's own future K/V), their K/V replace the future frames of the
+    layer's cache, the fused pairs are formed again, then every action layer reads (interaction
+    layers their fused pair), and both latents take one Euler step on one schedule 1 -> 0.
+
+    ``inp`` holds hist_q/k/v[l], joint_q/k/v[i][l] (future frames at step i), fuse_weights[m],
+    act_q/k/v[i][l], x_future, v_future[i], x_act, v_act[i].
+    """
+    F = F_h + F_f
+    B, _, H, D = np.shape(inp["hist_k"][0])
+    N = F * T
+    zeros = np.zeros((B, N, H, D))
+    out: Dict = {"hist_o": [], "joint_o": [], "act_o": []}
+    k_cache = [zeros.copy() for _ in range(L)]
+    v_cache = [zeros.copy() for _ in range(L)]
+    for l in range(L):
+        out["hist_o"].append(video_prefill(inp["hist_q"][l], inp["hist_k"][l], inp["hist_v"][l],
+                                           k_cache[l], v_cache[l], pad, frame_block, T, 0, F_h,
+                                           heads=heads))
+        k_cache[l] = cache_store(k_cache[l], inp["hist_k"][l], pad, T, 0, F_h)
+        v_cache[l] = cache_store(v_cache[l], inp["hist_v"][l], pad, T, 0, F_h)
+    parts = interval_partition(L, S)
+    reader = {j: m for m, j in enumerate(interaction_layers(L, S))}
+    sig = flow_schedule(n_steps, 0.0)
+    x_future, x_act = _f64(inp["x_future"]), _f64(inp["x_act"])
+    for i in range(n_steps):
+        outs = []
+        for l in range(L):
+            outs.append(video_prefill(inp["joint_q"][i][l], inp["joint_k"][i][l],
+                                      inp["joint_v"][i][l], k_cache[l], v_cache[l], pad,
+                                      frame_block, T, F_h, F, heads=heads))
+            k_cache[l] = cache_store(k_cache[l], inp["joint_k"][i][l], pad, T, F_h, F)
+            v_cache[l] = cache_store(v_cache[l], inp["joint_v"][i][l], pad, T, F_h, F)
+        out["joint_o"].append(outs)
+        fused_k = [fuse_interval([k_cache[j] for j in I], inp["fuse_weights"][m]) for m, I in enumerate(parts)]
+        fused_v = [fuse_interval([v_cache[j] for j in I], inp["fuse_weights"][m]) for m, I in enumerate(parts)]
+        outs = []
+        for l in range(L):
+            m = reader.get(l)
+            outs.append(action_attention(inp["act_q"][i][l], inp["act_k"][i][l], inp["act_v"][i][l],
+                                         fused_k[m] if m is not None else None,
+                                         fused_v[m] if m is not None else None, pad, T, heads=heads))
+        out["act_o"].append(outs)
+        x_future = euler_step(x_future, inp["v_future"][i], sig[i + 1] - sig[i])
+        x_act = euler_step(x_act, inp["v_act"][i], sig[i + 1] - sig[i])
+    out.update(k_cache=k_cache, v_cache=v_cache, fused_k=fused_k, fused_v=fused_v,
+               x_future=x_future, x_act=x_act)
     return out

@@ -168,3 +168,41 @@ def test_full_size_stages_sampled(name):
         ref = O.action_attention(to64(qa[b:b + 1]), to64(ka[b:b + 1]), to64(va[b:b + 1]),
                                  kc64[b:b + 1], vc64[b:b + 1], pb, T, heads=heads)
         assert_parity(to64(oa[b:b + 1])[:, :, heads], ref[:, :, heads], "bf16", f"{name} action b{b}")
+
+
+# ----------------------------------------------------------------------------- co-denoising
+
+@pytest.mark.parametrize("name,dtype", [("tiny_f32", "f32"), ("ctx2.4s_bf16", "bf16")])
+def test_joint_chunk(name, dtype):
+    # Co-denoising: every joint step re-passes the future frames (cache store + fusion
+    # epilogue) before its action reads; compared step by step with the oracle's joint chunk.
+    base = synth.WORKLOADS[name]
+    if dtype == "f32":
+        w = base.replace(seed=12, joint=True, n_video_steps=0, n_euler_steps=3)
+        heads = None
+    else:
+        w = base.replace(L=3, S=2, joint=True, n_video_steps=0, n_euler_steps=2,
+                         pad_rule="prefix:1", seed=13)
+        heads = [5, 19]
+    r, inp64 = _run_chunk(w)
+    pad = synth.pad_mask(w).numpy()
+    ref = O.chunk_joint(inp64, L=w.L, S=w.S, T=w.T, F_h=w.F_h, F_f=w.F_f,
+                        n_steps=w.n_euler_steps, pad=pad, heads=heads)
+    hs = list(range(w.H)) if heads is None else heads
+    T, F_h, F = w.T, w.F_h, w.F
+    rows_h, rows_f, rows = valid_rows(pad, T, 0, F_h), valid_rows(pad, T, F_h, F), valid_rows(pad, T, 0, F)
+    for l in range(w.L):
+        assert_parity(to64(r.hist_o[l])[:, :, hs][rows_h], ref["hist_o"][l][:, :, hs][rows_h], dtype, f"hist {l}")
+    for i in range(w.n_euler_steps):
+        for l in range(w.L):
+            assert_parity(to64(r.joint_o[i * w.L + l])[:, :, hs][rows_f], ref["joint_o"][i][l][:, :, hs][rows_f],
+                          dtype, f"joint {i},{l}")
+            assert_parity(to64(r.act_o[i * w.L + l])[:, :, hs], ref["act_o"][i][l][:, :, hs], dtype,
+                          f"joint action {i},{l}")
+    for l in range(w.L):
+        np.testing.assert_array_equal(to64(r.k_cache[l])[rows], ref["k_cache"][l][rows])
+    for m in range(w.M):
+        assert_parity(to64(r.fused_k[m])[rows], ref["fused_k"][m][rows], dtype, f"joint fused K {m}")
+        assert_parity(to64(r.fused_v[m])[rows], ref["fused_v"][m][rows], dtype, f"joint fused V {m}")
+    assert_parity(to64(r.x_future), ref["x_future"], "f32", "joint x_future")
+    assert_parity(to64(r.x_act), ref["x_act"], "f32", "joint x_act")

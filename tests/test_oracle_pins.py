@@ -396,3 +396,65 @@ def test_action_never_changes_video_outputs():
             np.testing.assert_array_equal(x, y)
     for m in range(len(a["fused_k"])):
         np.testing.assert_array_equal(a["fused_k"][m], b["fused_k"][m])
+
+
+# ----------------------------------------------------------------------------- co-denoising
+
+def _joint_inputs(N=3, **kw):
+    inp, ckw, M = _tiny_inputs(Nv=N, Ne=N, **kw)
+    # the joint steps re-use the tiny imagination draws as their future Q/K/V
+    inp["joint_q"], inp["joint_k"], inp["joint_v"] = inp["imag_q"], inp["imag_k"], inp["imag_v"]
+    jkw = {k: ckw[k] for k in ("L", "S", "T", "F_h", "F_f")}
+    return inp, jkw, N
+
+
+def test_joint_chunk_of_one_step_is_the_one_shot_chunk():
+    # One joint step: the history pass, one future pass whose K/V fill the cache, the fused
+    # pairs, one action step and one Euler step 1 -> 0 -- the IDM chunk with no imagination step
+    # whose cache pass takes the same future Q/K/V.
+    inp, jkw, _ = _joint_inputs(N=1)
+    pad = np.array([[1, 0, 0, 0]], np.uint8)
+    joint = O.chunk_joint(inp, n_steps=1, pad=pad, **jkw)
+    idm_inp = dict(inp, final_q=inp["joint_q"][0], final_k=inp["joint_k"][0], final_v=inp["joint_v"][0])
+    idm = O.chunk(idm_inp, n_video_steps=0, n_euler_steps=1, sigma_star=1.0, pad=pad, **jkw)
+    for x, y in zip(joint["hist_o"], idm["hist_o"]):
+        np.testing.assert_array_equal(x, y)
+    for x, y in zip(joint["joint_o"][0], idm["final_o"]):
+        np.testing.assert_array_equal(x, y)
+    for key in ("k_cache", "v_cache", "fused_k", "fused_v"):
+        for x, y in zip(joint[key], idm[key]):
+            np.testing.assert_array_equal(x, y)
+    for x, y in zip(joint["act_o"][0], idm["act_o"][0]):
+        np.testing.assert_array_equal(x, y)
+    np.testing.assert_array_equal(joint["x_act"], idm["x_act"])
+
+
+def test_joint_chunk_steps_only_see_their_own_and_earlier_inputs():
+    inp, jkw, N = _joint_inputs(N=3)
+    pad = np.zeros((1, 4), np.uint8)
+    a = O.chunk_joint(inp, n_steps=N, pad=pad, **jkw)
+    inp2 = dict(inp)
+    inp2["joint_k"] = inp["joint_k"][:2] + [[x + 5.0 for x in inp["joint_k"][2]]]
+    inp2["joint_v"] = inp["joint_v"][:2] + [[x - 1.0 for x in inp["joint_v"][2]]]
+    b = O.chunk_joint(inp2, n_steps=N, pad=pad, **jkw)
+    for i in range(2):
+        for key in ("joint_o", "act_o"):
+            for x, y in zip(a[key][i], b[key][i]):
+                np.testing.assert_array_equal(x, y)
+    # the last step's future K/V are what the caches hold at the end
+    T, Fh = jkw["T"], jkw["F_h"]
+    for l in range(jkw["L"]):
+        np.testing.assert_array_equal(b["k_cache"][l][:, Fh * T:], inp2["joint_k"][2][l])
+
+
+def test_joint_chunk_euler_recovers_the_clean_latents():
+    # With the true flow-matching velocity u = eps - x0 and the start x = eps, the shared
+    # schedule 1 -> 0 brings both latents back to x0 (closed form of the path).
+    inp, jkw, N = _joint_inputs(N=4)
+    r = np.random.default_rng(3)
+    x0f, epsf = r.standard_normal(inp["x_future"].shape), r.standard_normal(inp["x_future"].shape)
+    x0a, epsa = r.standard_normal(inp["x_act"].shape), r.standard_normal(inp["x_act"].shape)
+    inp = dict(inp, x_future=epsf, v_future=[epsf - x0f] * N, x_act=epsa, v_act=[epsa - x0a] * N)
+    out = O.chunk_joint(inp, n_steps=N, pad=np.zeros((1, 4), np.uint8), **jkw)
+    np.testing.assert_allclose(out["x_future"], x0f, atol=1e-13)
+    np.testing.assert_allclose(out["x_act"], x0a, atol=1e-13)

@@ -1,24 +1,23 @@
-// Asymmetric action attention on the tensor cores (bf16, D = 128, T % 64 == 0, n_act <= 32).
-//
-// 32 action queries read the fused video cache of one interaction layer plus their own K/V
-// ("Fast-WAM 精读" SECTION 07; Long-WAM Summary §4.2).  The read is HBM-bound: per key it
-// moves 512 B (K and V, bf16) and does 32 x 4 x 128 FLOP, 32 FLOP/B, above what the fp32
-// pipes can issue at full HBM bandwidth, so the contractions run on mma.sync tensor-core
-// tiles (M = 32 queries) while the loads stream through TMA: Q K^T on bf16 tiles, P V on tf32
-// tiles (the fused cache is already rounded to bf16 once, so P keeps 10 mantissa bits to
-// leave the error budget to the storage rounding).
-//
-// Work split (persistent, balanced): the call's tiles are laid out as, for every (episode b,
-// head h), one action tile (the n_act action keys, zero-padded to 64 and masked) followed by
-// the 64-key tiles of b's valid frames.  The G tiles are cut into P equal runs, one per CTA
-// (P = SM count), so every CTA streams the same amount whatever the padding.  A CTA keeps one
-// online-softmax state per (b, h) run it touches; a (b, h) contained in one CTA writes O
-// directly, otherwise each CTA writes its partial (O, m, l) into the workspace and the last
-// to arrive (atomic ticket) merges all partials by their log-sum-exp and resets the ticket.
-//
-// Tiles hold 128 keys when T % 128 == 0 (2-stage K/V ring), else 64 (4 stages).  Warps 0-7
-// consume (warp w: query rows 16 (w & 1) .., keys (w >> 1) * tile / 4 .. of each tile), warp
-// 8 lane 0 issues TMA loads into the ring and a 2-slot Q buffer.
+// Asymmetric action attention: 32 action queries read the fused video cache of one
+// interaction layer plus their own K/V ("Fast-WAM 精读" SECTION 07; Long-WAM Summary §4.2).
+// The read is HBM-bound: per key it moves 512 B (K and V, bf16) for 32 x 4 x 128 FLOP.
+// Three kernels (bf16, D = 128, n_act <= 32):
+//   action_umma_kernel  T % 128 == 0: tcgen05 tensor cores, one thread-block cluster per
+//                       (episode, head), partials merged in distributed shared memory (below).
+//   action_tc_kernel    T % 64 == 0 otherwise: mma.sync tiles (M = 32 queries), Q K^T on bf16
+//                       and P V on tf32 (P keeps 10 mantissa bits; the fused cache is already
+//                       rounded to bf16 once).  Persistent and balanced: the call's tiles (per
+//                       (episode b, head h) one action tile, the n_act action keys zero-padded
+//                       to 64 and masked, then the 64-key tiles of b's valid frames) are cut
+//                       into P equal runs, one per CTA (P = SM count).  A CTA keeps one
+//                       online-softmax state per (b, h) run it touches; a (b, h) contained in
+//                       one CTA writes O directly, otherwise each CTA writes its partial
+//                       (O, m, l) into the workspace and the last to arrive (atomic ticket)
+//                       merges them by their log-sum-exp and resets the ticket.  Warps 0-7
+//                       consume (warp w: query rows 16 (w & 1) .., keys (w >> 1) * 16 .. of
+//                       each tile), warp 8 lane 0 issues TMA loads into a 4-stage ring and a
+//                       2-slot Q buffer.
+//   action_self_kernel  layers outside the interaction set (action keys only).
 #include "launch.h"
 #include "tcgen05.cuh"
 
@@ -1109,9 +1108,7 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 32) return cudaErrorInvalidDevice;
   if (!(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(action_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, um::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -1123,10 +1120,9 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
     if (ac.ksplit < 1) return cudaErrorUnknown;
     return launch_pdl(action_umma_kernel, dim3(unsigned(a.B * a.H * ac.ksplit)), dim3(um::kThreads),
                       um::kSmemBytes, s, unsigned(ac.ksplit), ac, maps);
-  } else if (bn == 128)
-    action_tc_kernel<128><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
-  else
-    action_tc_kernel<64><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
+  }
+  // 64-key tiles (T % 128 != 0): the mma.sync kernel
+  action_tc_kernel<64><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);
   return cudaGetLastError();
 }
 

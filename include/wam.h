@@ -156,8 +156,7 @@ wam_status wam_fuse_interval_kv(const wam_video_layout* layout, wam_dtype dt, in
  *                    in turn.  Calls that share a workspace must not overlap on the GPU.  May be
  *                    NULL when the size is 0.  (The tensor-core read of 128-key tiles,
  *                    T % 128 == 0, merges its partials on chip and leaves the workspace
- *                    untouched; the size reported is the same for every layout so one
- *                    buffer sized once serves all calls.)
+ *                    untouched; the size query does not depend on which path will run.)
  * Action tokens attend to each other bidirectionally.  Returns WAM_ERR_WORKSPACE if the
  * workspace is missing or too small.
  */

@@ -49,7 +49,7 @@ __all__ = [
     "block_ids", "video_allowed", "action_key_allowed",
     "masked_attention", "video_prefill", "cache_store",
     "interval_partition", "interaction_layers", "fuse_weights", "fuse_interval",
-    "action_attention", "chunk", "chunk_joint",
+    "action_attention", "chunk", "chunk_joint", "chunk_stream",
 ]
 
 
@@ -339,6 +339,20 @@ def chunk(inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int, n_video_step
         k_cache[l] = cache_store(k_cache[l], inp["hist_k"][l], pad, T, 0, F_h)
         v_cache[l] = cache_store(v_cache[l], inp["hist_v"][l], pad, T, 0, F_h)
 
+    rest = chunk_after_history(inp, k_cache, v_cache, L=L, S=S, T=T, F_h=F_h, F_f=F_f,
+                               n_video_steps=n_video_steps, n_euler_steps=n_euler_steps,
+                               sigma_star=sigma_star, pad=pad, frame_block=frame_block, heads=heads)
+    rest["hist_o"] = out["hist_o"]
+    return rest
+
+
+def chunk_after_history(inp: Dict, k_cache, v_cache, *, L: int, S: int, T: int, F_h: int,
+                        F_f: int, n_video_steps: int, n_euler_steps: int, sigma_star: float, pad,
+                        frame_block=None, heads: Optional[Sequence[int]] = None) -> Dict:
+    """Stages a4 -> a8 of ``chunk`` given the per-layer caches of the history frames (the
+    lists are updated in place with the future frames)."""
+    F = F_h + F_f
+    out: Dict = {"imag_o": [], "final_o": [], "act_o": []}
     # a4: imagination passes and Euler steps on the future latents, sigma 1 -> sigma*.  With no
     # video step (the one-shot variant: one video pass at sigma* = 1, [FSW] §3.1) the cache pass
     # follows directly.
@@ -447,3 +461,54 @@ def chunk_joint(inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int, n_step
     out.update(k_cache=k_cache, v_cache=v_cache, fused_k=fused_k, fused_v=fused_v,
                x_future=x_future, x_act=x_act)
     return out
+
+
+# --------------------------------------------------------------------------------------
+# Streamed chunk: the history window kept across chunks     [LW-sum] §4.2 and App. B.2
+#                 (observed-video K/V computed once and reused; the conditions under which a
+#                 reused cache stays valid); [LW-src] §05 (streaming encoding of new frames)
+# --------------------------------------------------------------------------------------
+
+def chunk_stream(prev: Dict, inp: Dict, *, L: int, S: int, T: int, F_h: int, F_f: int,
+                 n_video_steps: int, n_euler_steps: int, sigma_star: float, pad,
+                 frame_block=None, heads: Optional[Sequence[int]] = None) -> Dict:
+    """The next chunk of an episode whose history window slid by one frame.
+
+    Reading R11: between chunks one observation frame arrives; the window keeps F_h frames, so
+    every cached frame moves one position earlier and the oldest leaves it (``pad`` is this
+    chunk's padding: the frames the previous chunk held at f + 1 are the ones valid at f).  The
+    per-layer caches and the fused pairs of the surviving frames are the previous chunk's,
+    shifted; only the newest frame (F_h - 1) is passed through the layers (queries over the
+    cached window and itself), stored and folded.  The imagination, cache and action stages
+    then run as in ``chunk``.
+
+    ``prev`` is a previous chunk's output (its k_cache and v_cache are used; the fused pairs of
+    the surviving frames are sums over those caches, so forming them again from the shifted
+    caches equals shifting them); ``inp`` holds new_q/k/v[l] ([B, T, H, D], the newest frame)
+    and the imagination, final, fusion and action inputs of ``chunk``.  Returns the same keys as
+    ``chunk`` with hist_o[l] the newest frame's output ([B, T, H, D]).
+    """
+    F = F_h + F_f
+    pad = np.asarray(pad)
+    shift = lambda x: np.concatenate([x[:, T:F_h * T], np.zeros_like(x[:, :T]), x[:, F_h * T:]], axis=1)
+    keep = lambda x: np.where(_row_valid(pad, T, F)[:, :, None, None], x, 0.0)
+    k_cache = [keep(shift(x)) for x in prev["k_cache"]]
+    v_cache = [keep(shift(x)) for x in prev["v_cache"]]
+    out: Dict = {"hist_o": [], "imag_o": [], "final_o": [], "act_o": []}
+    for l in range(L):
+        out["hist_o"].append(video_prefill(inp["new_q"][l], inp["new_k"][l], inp["new_v"][l],
+                                           k_cache[l], v_cache[l], pad, frame_block, T, F_h - 1,
+                                           F_h, heads=heads))
+        k_cache[l] = cache_store(k_cache[l], inp["new_k"][l], pad, T, F_h - 1, F_h)
+        v_cache[l] = cache_store(v_cache[l], inp["new_v"][l], pad, T, F_h - 1, F_h)
+    rest = chunk_after_history(inp, k_cache, v_cache, L=L, S=S, T=T, F_h=F_h, F_f=F_f,
+                               n_video_steps=n_video_steps, n_euler_steps=n_euler_steps,
+                               sigma_star=sigma_star, pad=pad, frame_block=frame_block, heads=heads)
+    rest["hist_o"] = out["hist_o"]
+    return rest
+
+
+def _row_valid(pad, T: int, F: int) -> np.ndarray:
+    """[B, F*T] True on the rows of non-padding frames."""
+    pad = np.asarray(pad)
+    return np.repeat(pad[:, :F] == 0, T, axis=1)

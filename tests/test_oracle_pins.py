@@ -458,3 +458,37 @@ def test_joint_chunk_euler_recovers_the_clean_latents():
     out = O.chunk_joint(inp, n_steps=N, pad=np.zeros((1, 4), np.uint8), **jkw)
     np.testing.assert_allclose(out["x_future"], x0f, atol=1e-13)
     np.testing.assert_allclose(out["x_act"], x0a, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- streamed chunks
+
+@pytest.mark.parametrize("p_prev,p_next", [(2, 1), (0, 0)], ids=["window_grows", "window_full"])
+def test_streamed_chunk_equals_the_chunk_recomputed_over_the_slid_window(p_prev, p_next):
+    # The previous chunk's caches shifted by one frame plus one pass of the newest frame give
+    # exactly the chunk computed from scratch over the slid window (whose history inputs are
+    # the previous ones moved one frame earlier, the oldest dropped, the newest appended).
+    inp, kw, M = _tiny_inputs(Fh=4)
+    L, T, Fh, Ff = kw["L"], kw["T"], kw["F_h"], kw["F_f"]
+    F = Fh + Ff
+    pad_prev = np.array([[1] * p_prev + [0] * (F - p_prev)], np.uint8)
+    pad_next = np.array([[1] * p_next + [0] * (F - p_next)], np.uint8)
+    prev = O.chunk(inp, pad=pad_prev, **kw)
+    r = np.random.default_rng(11)
+    new = {n: [r.standard_normal((1, T) + inp["hist_k"][0].shape[2:]) for _ in range(L)] for n in ("q", "k", "v")}
+    step = dict(inp, new_q=new["q"], new_k=new["k"], new_v=new["v"])
+    got = O.chunk_stream(prev, step, pad=pad_next, **kw)
+    slid = dict(inp)
+    for n in ("q", "k", "v"):
+        slid["hist_" + n] = [np.concatenate([inp["hist_" + n][l][:, T:], new[n][l]], axis=1) for l in range(L)]
+    want = O.chunk(slid, pad=pad_next, **kw)
+    for l in range(L):
+        np.testing.assert_allclose(got["hist_o"][l], want["hist_o"][l][:, (Fh - 1) * T:], atol=1e-13)
+    for key in ("k_cache", "v_cache", "fused_k", "fused_v"):
+        for x, y in zip(got[key], want[key]):
+            np.testing.assert_allclose(x, y, atol=1e-13)
+    for key in ("imag_o", "act_o"):
+        for xs, ys in zip(got[key], want[key]):
+            for x, y in zip(xs, ys):
+                np.testing.assert_allclose(x, y, atol=1e-13)
+    for x, y in zip(got["final_o"], want["final_o"]):
+        np.testing.assert_allclose(x, y, atol=1e-13)

@@ -76,7 +76,7 @@ def algorithmic_work(w: synth.Workload, pad: np.ndarray) -> dict:
         valid = [f for f in range(w.F) if not pad[b, f]]
         valid_keys += len(valid) * T
         for f in range(w.F_h):
-            if not pad[b, f]:
+            if not pad[b, f] and (not w.slide or f == w.F_h - 1):  # sliding window: newest only
                 hist_pairs += sum(1 for g in valid if g <= f)
         for f in range(w.F_h, w.F):
             fut_pairs += sum(1 for g in valid if g <= f)
@@ -226,7 +226,7 @@ def oracle_sample_seconds(w: synth.Workload, pad: np.ndarray, n_heads: int, n_la
     t0 = time.perf_counter()
     kc = [O.cache_store(np.zeros((w.B, N, n_heads, D)), hk[l], pad, T, 0, w.F_h) for l in layers]
     vc = [O.cache_store(np.zeros((w.B, N, n_heads, D)), hv[l], pad, T, 0, w.F_h) for l in layers]
-    rows_h = np.arange(0, hist, row_stride)
+    rows_h = np.arange((w.F_h - 1) * T if w.slide else 0, hist, row_stride)
     rows_f = np.arange(0, fut, row_stride)
     for l in layers:
         O.video_prefill(hq[l], hk[l], hv[l], None, None, pad, None, T, 0, w.F_h, rows=rows_h)
@@ -371,6 +371,8 @@ def run_mine(args, world, rank, local):
     ev = {name: (torch.cuda.Event(enable_timing=True, external=True),
                  torch.cuda.Event(enable_timing=True, external=True))
           for name, _, _ in runner.stages}
+    if w.slide:
+        runner.prime()  # the state the first streamed chunk continues from
     runner.run()  # first call: one-time per-device set-up outside any capture
     torch.cuda.synchronize()
     wam.device_error()
@@ -409,7 +411,8 @@ def run_mine(args, world, rank, local):
         for k, (a, b) in ev.items():
             stage_ms[k].append(a.elapsed_time(b))
     wam.device_error()
-    ms, value = replica_throughput(total_ms / args.steps, world)
+    # a run is one chunk, or two streamed chunks in the sliding-window mode
+    ms, value = replica_throughput(total_ms / args.steps / runner.chunks_per_run, world)
     st_ms = {k: statistics.mean(v) for k, v in stage_ms.items()}
     if w.joint:  # co-denoising: per joint step a video stage (future passes) and an action stage
         fut_ms = sum(v for k, v in st_ms.items() if k.startswith("video"))
@@ -417,7 +420,7 @@ def run_mine(args, world, rank, local):
                  "action": sum(v for k, v in st_ms.items() if k.startswith("action"))}
         video_ms = st_ms["history"] + fut_ms
     else:
-        video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"]
+        video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"] + st_ms.get("copy", 0.0)
     action_ms = st_ms["action"]
     fused_ms = time_fused_read(runner, stream)
 
@@ -536,9 +539,9 @@ def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
                     prev = f
     else:
         runs = None
-    for name in ("hist_q", "hist_k", "hist_v"):
+    for name in (("new_q", "new_k", "new_v") if w.slide else ("hist_q", "hist_k", "hist_v")):
         for l, t in enumerate(inp[name]):
-            add(name, t, l % 2, runs)
+            add(name, t, l % 2, None if w.slide else runs)
     for name in ("imag_q", "imag_k", "imag_v", "act_q", "act_k", "act_v", "joint_q", "joint_k", "joint_v"):
         for i, row in enumerate(inp[name]):
             for l, t in enumerate(row):
@@ -570,9 +573,10 @@ def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
+    ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps / runner.chunks_per_run, world)
+    cpr = runner.chunks_per_run
     return {"value": world * 1000.0 / ms, "unit": "chunks/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "h2d_bytes_per_step": h2d // cpr, "d2h_bytes_per_step": d2h // cpr,
             "note": "inputs in pinned host memory; non-padding frames of every Q/K/V tensor "
                     "copied host->device each step, x_act read back"}
 

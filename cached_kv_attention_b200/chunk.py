@@ -74,6 +74,10 @@ def make_inputs(w: Workload, device: str = "cpu") -> Dict:
         "act_q": [[qkv("act_q", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
         "act_k": [[qkv("act_k", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
         "act_v": [[qkv("act_v", w.n_act, i, l) for l in range(w.L)] for i in range(w.n_euler_steps)],
+        # sliding window: the newest history frame of a streamed chunk
+        "new_q": [qkv("new_q", T, l) for l in range(w.L)] if w.slide else [],
+        "new_k": [qkv("new_k", T, l) for l in range(w.L)] if w.slide else [],
+        "new_v": [qkv("new_v", T, l) for l in range(w.L)] if w.slide else [],
         "x_future": synth.normal((B, fut, w.C), w.seed, "x_future", device=device),
         "v_future": [synth.normal((B, fut, w.C), w.seed, "v_future", s, device=device)
                      for s in range(w.n_euler_steps if w.joint else w.n_video_steps)],
@@ -107,10 +111,19 @@ class ChunkRunner:
         self.layout = wam.VideoLayout(B, H, D, T, F, self.pad, frame_block)
         dev = torch.device(device)
         z = lambda *s, dtype=dt: torch.zeros(s, dtype=dtype, device=dev)
-        self.k_cache = [z(B, N, H, D) for _ in range(w.L)]
-        self.v_cache = [z(B, N, H, D) for _ in range(w.L)]
-        self.fused_k = [z(B, N, H, D) for _ in range(w.M)]
-        self.fused_v = [z(B, N, H, D) for _ in range(w.M)]
+        # per-layer caches and fused pairs; the sliding-window mode keeps two sets used in turn
+        self._sets = [([z(B, N, H, D) for _ in range(w.L)], [z(B, N, H, D) for _ in range(w.L)],
+                       [z(B, N, H, D) for _ in range(w.M)], [z(B, N, H, D) for _ in range(w.M)])
+                      for _ in range(2 if w.slide else 1)]
+        self._use_set(0)
+        self.chunks_per_run = 1
+        if w.slide:
+            if fusion != "epilogue":
+                raise ValueError("the sliding-window mode folds the fusion into its passes (epilogue)")
+            P = int(self.pad[0, :w.F_h].sum())
+            if not (np.all(self.pad[:, :P] == 1) and np.all(self.pad[:, P:] == 0) and P < w.F_h):
+                raise ValueError("the sliding-window mode needs the same padding prefix in every episode")
+            self.slide_pad = P
         self.acc_k = z(B, N, H, D, dtype=torch.float32)
         self.acc_v = z(B, N, H, D, dtype=torch.float32)
         hist, fut = w.F_h * T, w.F_f * T
@@ -121,6 +134,7 @@ class ChunkRunner:
         self.final_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_h)]
         self.imag_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_i)]
         self.act_o = [z(B, w.n_act, H, D, dtype=o_dtype) for _ in range(n_a)]
+        self.new_o = [z(B, T, H, D, dtype=o_dtype) for _ in range(n_h if w.slide else 0)]
         if w.joint and fusion != "epilogue":
             raise ValueError("co-denoising chunks fold the fusion into the future passes (epilogue)")
         self.joint_o = [z(B, fut, H, D, dtype=o_dtype) for _ in range(n_a if w.joint else 0)]
@@ -149,26 +163,50 @@ class ChunkRunner:
         return e.ref
 
     def prepare(self, stream=None) -> "ChunkRunner":
-        w, L = self.w, wam.lib
+        w = self.w
         s = ctypes.c_void_p(wam._stream(stream))
         lay = self.layout.ref
         dt = wam.BF16 if w.dtype == "bf16" else wam.F32
         o_dt = wam.F32 if self.hist_o[0].dtype == torch.float32 else dt
-        inp, F_h, F = self.inp, w.F_h, w.F
-        calls = []
 
         def o_of(lst, idx):
             return _vp(lst[idx % len(lst)])
 
-        # a3: history prefill with the cache store (+ fusion epilogue)
-        for l in range(w.L):
-            calls.append((L.wam_video_prefill_kv,
-                          (lay, dt, 0, F_h, _vp(inp["hist_q"][l]), _vp(inp["hist_k"][l]),
-                           _vp(inp["hist_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
-                           o_of(self.hist_o, l), o_dt, self._epilogue(l), s)))
-        hist_end = len(calls)
+        if w.slide:
+            return self._prepare_slide(lay, dt, o_dt, s, o_of)
+        calls = []
+        hist_end = self._history_calls(calls, lay, dt, o_dt, s, o_of)
         if w.joint:
             return self._prepare_joint(calls, hist_end, lay, dt, o_dt, s, o_of)
+        imag_end, video_end = self._rest_calls(calls, lay, dt, o_dt, s, o_of)
+        self.calls = calls
+        # stage boundaries (call indices): the video stages a3 (history), a4 (imagination passes
+        # and four small Euler steps), a5-a6 (final pass, standalone fusion), then the action
+        # stages a7-a8
+        self.stages = [("history", 0, hist_end), ("imagination", hist_end, imag_end),
+                       ("final", imag_end, video_end), ("action", video_end, len(calls))]
+        self.fused_read_call = self._first_fused_read(calls, video_end)
+        return self
+
+    @staticmethod
+    def _first_fused_read(calls, start):
+        return next(i for i in range(start, len(calls))
+                    if calls[i][0] is wam.lib.wam_action_attn and calls[i][1][2] is not None)
+
+    def _history_calls(self, calls, lay, dt, o_dt, s, o_of) -> int:
+        """a3: history prefill with the cache store (+ fusion epilogue), all history frames."""
+        w, L, inp = self.w, wam.lib, self.inp
+        for l in range(w.L):
+            calls.append((L.wam_video_prefill_kv,
+                          (lay, dt, 0, w.F_h, _vp(inp["hist_q"][l]), _vp(inp["hist_k"][l]),
+                           _vp(inp["hist_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
+                           o_of(self.hist_o, l), o_dt, self._epilogue(l), s)))
+        return len(calls)
+
+    def _rest_calls(self, calls, lay, dt, o_dt, s, o_of):
+        """a4-a8 on the current buffer set; returns the call indices where the final pass and
+        the action stages start."""
+        w, L, inp, F_h, F = self.w, wam.lib, self.inp, self.w.F_h, self.w.F
         # a4: imagination passes + Euler on the future latents
         nf = self.x_future.numel()
         for st in range(w.n_video_steps):
@@ -214,15 +252,54 @@ class ChunkRunner:
                                self.workspace.numel(), s)))
             ds = float(self.sig_a[i + 1] - self.sig_a[i])
             calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
-        self.calls = calls
-        # stage boundaries (call indices): the video stages a3 (history), a4 (imagination passes
-        # and four small Euler steps), a5-a6 (final pass, standalone fusion), then the action
-        # stages a7-a8
-        self.stages = [("history", 0, hist_end), ("imagination", hist_end, imag_end),
-                       ("final", imag_end, video_end), ("action", video_end, len(calls))]
-        self.fused_read_call = next(i for i in range(video_end, len(calls))
-                                    if calls[i][0] is L.wam_action_attn and calls[i][1][2] is not None)
+        return imag_end, video_end
+
+    def _use_set(self, k: int) -> None:
+        self.k_cache, self.v_cache, self.fused_k, self.fused_v = self._sets[k]
+
+    def _prepare_slide(self, lay, dt, o_dt, s, o_of) -> "ChunkRunner":
+        """History window kept across chunks: ``prime_calls`` fill buffer set 1 with a full chunk;
+        one run is two streamed chunks (set 1 -> 0, then 0 -> 1), each moving the surviving
+        frames' caches and fused pairs one frame earlier into the other set, passing only the
+        newest frame through the layers, then the imagination, cache and action stages."""
+        w, L, inp, F_h, P = self.w, wam.lib, self.inp, self.w.F_h, self.slide_pad
+        self._use_set(1)
+        prime = []
+        self._history_calls(prime, lay, dt, o_dt, s, o_of)
+        self._rest_calls(prime, lay, dt, o_dt, s, o_of)
+        self.prime_calls = prime
+        calls, stages = [], []
+        for k in (0, 1):
+            src, dst = self._sets[1 - k], self._sets[k]
+            self._use_set(k)
+            tensors = [(a, b) for sa, sb in zip(src, dst) for a, b in zip(sa, sb)]
+            sp = (ctypes.c_void_p * len(tensors))(*[a.data_ptr() for a, _ in tensors])
+            dp = (ctypes.c_void_p * len(tensors))(*[b.data_ptr() for _, b in tensors])
+            self._keep += [sp, dp]
+            c0 = len(calls)
+            calls.append((L.wam_copy_frames, (lay, dt, len(tensors), sp, dp, P + 1, P, F_h - 1 - P, s)))
+            h0 = len(calls)
+            for l in range(w.L):
+                calls.append((L.wam_video_prefill_kv,
+                              (lay, dt, F_h - 1, F_h, _vp(inp["new_q"][l]), _vp(inp["new_k"][l]),
+                               _vp(inp["new_v"][l]), _vp(self.k_cache[l]), _vp(self.v_cache[l]), 1,
+                               o_of(self.new_o, l), o_dt, self._epilogue(l), s)))
+            h1 = len(calls)
+            imag_end, video_end = self._rest_calls(calls, lay, dt, o_dt, s, o_of)
+            if k == 0:
+                stages = [("copy", c0, h0), ("history", h0, h1), ("imagination", h1, imag_end),
+                          ("final", imag_end, video_end), ("action", video_end, len(calls))]
+                self.fused_read_call = self._first_fused_read(calls, video_end)
+        self.calls, self.stages, self.chunks_per_run = calls, stages, 2
         return self
+
+    def prime(self) -> None:
+        """Sliding-window mode: fill buffer set 1 with one full chunk (the state the first
+        streamed chunk continues from)."""
+        for fn, args in self.prime_calls:
+            st = fn(*args)
+            if st:
+                wam.check(st)
 
     def _prepare_joint(self, calls, hist_end, lay, dt, o_dt, s, o_of) -> "ChunkRunner":
         """Co-denoising: at every joint step i the future frames are passed through all layers
@@ -265,26 +342,25 @@ class ChunkRunner:
         self.x_act.copy_(self.inp["x_act"])
 
     def run(self, events: Optional[Dict] = None, stream=None) -> None:
-        """Issue the chunk.  ``events`` maps a stage name to (start, end) CUDA events that are
-        recorded on ``stream`` around that stage (also inside a graph capture when the events
-        are external)."""
-        if not events:
-            for fn, args in self.calls:
-                st = fn(*args)
-                if st:
-                    wam.check(st)
-            return
-        stream = torch.cuda.current_stream() if stream is None else stream
-        for name, i0, i1 in self.stages:
-            ev = events.get(name)
-            if ev:
-                ev[0].record(stream)
-            for fn, args in self.calls[i0:i1]:
-                st = fn(*args)
-                if st:
-                    wam.check(st)
-            if ev:
-                ev[1].record(stream)
+        """Issue the prepared calls (one chunk, or two in the sliding-window mode).  ``events``
+        maps a stage name to (start, end) CUDA events that are recorded on ``stream`` around
+        that stage (also inside a graph capture when the events are external)."""
+        marks: Dict[int, List] = {}
+        if events:
+            stream = torch.cuda.current_stream() if stream is None else stream
+            for name, i0, i1 in self.stages:
+                ev = events.get(name)
+                if ev:
+                    marks.setdefault(i0, []).append(ev[0])
+                    marks.setdefault(i1, []).append(ev[1])
+        for i, (fn, args) in enumerate(self.calls):
+            for e in marks.get(i, ()):
+                e.record(stream)
+            st = fn(*args)
+            if st:
+                wam.check(st)
+        for e in marks.get(len(self.calls), ()):
+            e.record(stream)
 
     # ------------------------------------------------------------------ counts
     def launches_per_chunk(self) -> int:

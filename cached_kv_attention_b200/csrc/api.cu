@@ -262,6 +262,44 @@ wam_status wam_flow_euler_step(int64_t n, float* x, const float* v, float dsigma
                      "wam_flow_euler_step");
 }
 
+wam_status wam_copy_frames(const wam_video_layout* layout, wam_dtype dt, int32_t n,
+                           const void* const* src, void* const* dst, int32_t f_src,
+                           int32_t f_dst, int32_t n_frames, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(dt, "dt"));
+  if (n < 1 || n > WAM_MAX_COPY_TENSORS)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n must be in [1, %d] (got %d)", WAM_MAX_COPY_TENSORS, n);
+  if (!src || !dst) return fail(WAM_ERR_INVALID_ARGUMENT, "src or dst is NULL");
+  if (n_frames < 0 || f_src < 0 || f_dst < 0 || f_src + n_frames > g.F || f_dst + n_frames > g.F)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "frames [%d, %d) -> [%d, %d) outside [0, %d)", f_src,
+                f_src + n_frames, f_dst, f_dst + n_frames, g.F);
+  const size_t es = dt == WAM_BF16 ? 2 : 4;
+  const size_t frame_bytes = size_t(g.T) * g.H * g.D * es;
+  const size_t tensor_bytes = size_t(g.B) * g.F * frame_bytes;
+  static thread_local wam::CopyArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int j = 0; j < n; ++j) {
+    if (!src[j] || !dst[j])
+      return fail(WAM_ERR_INVALID_ARGUMENT, "src[%d] or dst[%d] is NULL", j, j);
+    if (!aligned16(src[j]) || !aligned16(dst[j]))
+      return fail(WAM_ERR_INVALID_ARGUMENT, "src[%d] or dst[%d] is not 16-byte aligned", j, j);
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(src[j]), d0 = reinterpret_cast<uintptr_t>(dst[j]);
+    if (s0 < d0 + tensor_bytes && d0 < s0 + tensor_bytes)
+      return fail(WAM_ERR_INVALID_ARGUMENT, "src[%d] and dst[%d] overlap", j, j);
+    a.src[j] = src[j];
+    a.dst[j] = dst[j];
+  }
+  if (n_frames == 0) return ok();
+  a.n = n, a.B = g.B;
+  a.ep_vec = int64_t(g.F) * frame_bytes / 16;
+  a.src_vec = int64_t(f_src) * frame_bytes / 16;
+  a.dst_vec = int64_t(f_dst) * frame_bytes / 16;
+  a.n_vec = int64_t(n_frames) * frame_bytes / 16;
+  return cuda_status(wam::launch_copy_frames(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_copy_frames");
+}
+
 wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt, int32_t f_begin,
                                 int32_t f_end, const void* q, const void* k_new,
                                 const void* v_new, void* k_cache, void* v_cache,

@@ -77,6 +77,16 @@ struct ActionArgs {
   FrameLists fl;
 };
 
+struct CopyArgs {
+  const void* src[WAM_MAX_COPY_TENSORS];
+  void* dst[WAM_MAX_COPY_TENSORS];
+  int32_t n, B;
+  int64_t ep_vec;    // 16-byte vectors of one episode's tensor (F*T*H*D*es / 16)
+  int64_t src_vec;   // first vector copied within an episode
+  int64_t dst_vec;
+  int64_t n_vec;     // vectors copied per (tensor, episode)
+};
+
 struct FuseArgs {
   const void* k[WAM_MAX_FUSE_LAYERS];
   const void* v[WAM_MAX_FUSE_LAYERS];

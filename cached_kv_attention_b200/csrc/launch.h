@@ -11,6 +11,7 @@ namespace wam {
 cudaError_t launch_euler(int64_t n, float* x, const float* v, float dsigma, cudaStream_t s);
 cudaError_t launch_store_fuse(const PrefillArgs& a, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_fuse(const FuseArgs& a, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_copy_frames(const CopyArgs& a, cudaStream_t s);
 cudaError_t launch_debug_mask(const PrefillArgs& a, uint8_t* mask, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_action_simt(const ActionArgs& a, int D, bool bf16, cudaStream_t s);

@@ -60,6 +60,29 @@ cudaError_t launch_euler(int64_t n, float* x, const float* v, float dsigma, cuda
   return launch_pdl(euler_kernel, dim3(grid_for((n + 3) / 4, 256, 148 * 16)), dim3(256), 0, s, 0, n, x, v, dsigma);
 }
 
+// ------------------------------------------------------------------------------ frame copies
+// blockIdx.y = tensor pair j * B + episode b; a grid-stride loop over the 16-byte vectors of
+// the copied frames (contiguous within an episode).
+__global__ void copy_frames_kernel(const __grid_constant__ CopyArgs a) {
+  grid_dependency_wait();  // programmatic dependent launch: inputs ready from here on
+  grid_launch_dependents();
+  const int j = int(blockIdx.y) / a.B, b = int(blockIdx.y) % a.B;
+  const uint4* src = static_cast<const uint4*>(a.src[j]) + int64_t(b) * a.ep_vec + a.src_vec;
+  uint4* dst = static_cast<uint4*>(a.dst[j]) + int64_t(b) * a.ep_vec + a.dst_vec;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.n_vec;
+       i += int64_t(gridDim.x) * blockDim.x)
+    dst[i] = __ldcs(src + i);  // streamed once: evict-first
+}
+
+cudaError_t launch_copy_frames(const CopyArgs& a, cudaStream_t s) {
+  if (a.n_vec == 0) return cudaSuccess;
+  const int64_t pairs = int64_t(a.n) * a.B;
+  const int64_t per_pair = (a.n_vec + 255) / 256;
+  const int64_t want = (148 * 8 + pairs - 1) / pairs;  // ~8 blocks per SM over all pairs
+  const unsigned gx = unsigned(per_pair < want ? per_pair : (want < 1 ? 1 : want));
+  return launch_pdl(copy_frames_kernel, dim3(gx, unsigned(pairs)), dim3(256), 0, s, 0, a);
+}
+
 // ------------------------------------------------------------------------------ store + fuse
 // Copies the new K/V of every valid query frame into the cache and applies the fusion
 // epilogue (acc = w K | acc += w K | fused = round(acc + w K)).  grid (chunks, items, 2).

@@ -49,6 +49,7 @@ class Workload:
     pad_rule: str        # "none" | "prefix:<P>" | "prefix_frac:<pmax>" | "prefix_unif:<Pmax>"
     seed: int
     joint: bool = False  # co-denoising: the future frames are re-passed at every action step
+    slide: bool = False  # history window kept across chunks: only the newest frame is passed
 
     @property
     def F(self) -> int:
@@ -97,6 +98,10 @@ WORKLOADS["oneshot_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
 # before its action reads.
 WORKLOADS["cod4_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
     name="cod4_ctx19.2s_bf16", joint=True, n_video_steps=0, n_euler_steps=4, sigma_star=0.0)
+# The 19.2 s chunk with the history window kept across chunks (steady state: each chunk one
+# new frame in, the oldest of the 5 valid frames out).
+WORKLOADS["slide_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
+    name="slide_ctx19.2s_bf16", slide=True)
 
 
 def seed_for(seed: int, name: str, *idx: int) -> int:

@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "wam_action_attn": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp],
         "wam_action_attn_workspace_size": [lay, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)],
         "wam_flow_euler_step": [i64, vp, vp, f32, vp],
+        "wam_copy_frames": [lay, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp],
         "wam_flow_schedule": [i32, f64, f64, ctypes.POINTER(f64)],
         "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
         "wam_debug_video_mask": [lay, i32, i32, vp, vp],
@@ -87,7 +88,8 @@ def exported_names() -> list:
     return ["wam_video_prefill_kv", "wam_fuse_interval_kv", "wam_action_attn",
             "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
             "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
-            "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size"]
+            "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size",
+            "wam_copy_frames"]
 
 
 def check(status: int) -> None:
@@ -182,6 +184,16 @@ def fuse_interval_kv(layout: VideoLayout, k_layers, v_layers, weights, f_begin: 
     w = (ctypes.c_float * n)(*[float(x) for x in weights])
     check(lib.wam_fuse_interval_kv(layout.ref, _dtype(fused_k), n, kp, vp, w, f_begin, f_end,
                                    _ptr(fused_k), _ptr(fused_v), _stream(stream)))
+
+
+def copy_frames(layout: VideoLayout, src, dst, f_src: int, f_dst: int, n_frames: int,
+                stream=None) -> None:
+    """Frames [f_src, f_src + n_frames) of every src tensor to [f_dst, ...) of its dst."""
+    n = len(src)
+    sp = (ctypes.c_void_p * n)(*[_ptr(t) for t in src])
+    dp = (ctypes.c_void_p * n)(*[_ptr(t) for t in dst])
+    check(lib.wam_copy_frames(layout.ref, _dtype(src[0]), n, sp, dp, f_src, f_dst, n_frames,
+                              _stream(stream)))
 
 
 def action_attn_workspace_size(layout: VideoLayout, dtype: torch.dtype, n_act: int,

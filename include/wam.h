@@ -46,6 +46,7 @@ typedef struct CUstream_st* wam_stream_t; /* the same handle as cudaStream_t */
 #define WAM_MAX_FRAMES 256
 #define WAM_MAX_EPISODE_FRAMES 1024
 #define WAM_MAX_FUSE_LAYERS 16
+#define WAM_MAX_COPY_TENSORS 128
 
 typedef enum {
   WAM_OK = 0,
@@ -181,6 +182,24 @@ wam_status wam_action_attn_workspace_size(const wam_video_layout* layout, wam_dt
  */
 wam_status wam_flow_euler_step(int64_t n, float* x, const float* v, float dsigma,
                                wam_stream_t stream);
+
+/*
+ * Move whole frames of per-layer K/V tensors from one buffer set to another, for a history
+ * window kept across chunks ("Long-WAM ... | Summary" §4.2: the observed-video K/V is
+ * computed once and reused; one frame arrives per chunk, so the window slides and every kept
+ * frame moves to an earlier position).  For each pair j < n and every episode b:
+ *   dst[j][b, (f_dst + i) * T + t, :, :] = src[j][b, (f_src + i) * T + t, :, :]
+ *   for 0 <= i < n_frames, 0 <= t < T.
+ *   src, dst  host arrays of n device pointers [B, F*T, H, D] (dtype dt), 16-byte aligned;
+ *             src[j] and dst[j] must not overlap (keep the window in two buffer sets used in
+ *             turn).  1 <= n <= WAM_MAX_COPY_TENSORS.
+ *   frames    0 <= f_src, f_dst and f_src + n_frames, f_dst + n_frames <= F; n_frames == 0
+ *             launches nothing.
+ * Padding is not consulted: whole frames are copied.
+ */
+wam_status wam_copy_frames(const wam_video_layout* layout, wam_dtype dt, int32_t n,
+                           const void* const* src, void* const* dst, int32_t f_src,
+                           int32_t f_dst, int32_t n_frames, wam_stream_t stream);
 
 /*
  * wam_video_prefill_kv with the fusion epilogue, for callers that cannot allocate device memory

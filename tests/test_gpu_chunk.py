@@ -206,3 +206,52 @@ def test_joint_chunk(name, dtype):
         assert_parity(to64(r.fused_v[m])[rows], ref["fused_v"][m][rows], dtype, f"joint fused V {m}")
     assert_parity(to64(r.x_future), ref["x_future"], "f32", "joint x_future")
     assert_parity(to64(r.x_act), ref["x_act"], "f32", "joint x_act")
+
+
+# ----------------------------------------------------------------------------- sliding window
+
+@pytest.mark.parametrize("name,dtype", [("tiny_f32", "f32"), ("ctx2.4s_bf16", "bf16")])
+def test_sliding_window_chunks(name, dtype):
+    # A full chunk primes buffer set 1; one run streams two chunks (set 1 -> 0, then 0 -> 1),
+    # each moving the kept frames one position earlier (wam_copy_frames) and passing only the
+    # newest frame.  Compared with the oracle's streamed chunks continuing from its full chunk.
+    base = synth.WORKLOADS[name]
+    if dtype == "f32":
+        w = base.replace(F_h=3, pad_rule="prefix:1", slide=True, seed=14)
+        heads = None
+    else:
+        w = base.replace(F_h=4, L=3, S=2, n_video_steps=1, n_euler_steps=2, pad_rule="prefix:1",
+                         slide=True, seed=15)
+        heads = [2, 21]
+    inp_cpu = C.make_inputs(w, "cpu")
+    inp = {k: _tree(v, lambda t: t.cuda()) for k, v in inp_cpu.items()}
+    r = C.ChunkRunner(w, inp, distinct_out=True).prepare()
+    r.prime()
+    r.run()
+    wam.device_error()
+    inp64 = {k: _tree(v, to64) for k, v in inp_cpu.items()}
+    inp64["fuse_weights"] = [O.fuse_weights(lg) for lg in inp64.pop("fuse_logits")]
+    pad = synth.pad_mask(w).numpy()
+    kw = dict(L=w.L, S=w.S, T=w.T, F_h=w.F_h, F_f=w.F_f, n_video_steps=w.n_video_steps,
+              n_euler_steps=w.n_euler_steps, sigma_star=w.sigma_star, pad=pad, heads=heads)
+    prime = O.chunk(inp64, **kw)
+    first = O.chunk_stream(prime, inp64, **kw)
+    second = O.chunk_stream(first, inp64, **kw)
+    hs = list(range(w.H)) if heads is None else heads
+    rows = valid_rows(pad, w.T, 0, w.F)
+    rows_f = valid_rows(pad, w.T, w.F_h, w.F)
+    for k_set, ref in ((0, first), (1, second)):
+        kc, vc, fk, fv = r._sets[k_set]
+        for l in range(w.L):
+            np.testing.assert_array_equal(to64(kc[l])[rows], ref["k_cache"][l][rows])
+            np.testing.assert_array_equal(to64(vc[l])[rows], ref["v_cache"][l][rows])
+        for m in range(w.M):
+            assert_parity(to64(fk[m])[rows], ref["fused_k"][m][rows], dtype, f"slide fused K {k_set},{m}")
+            assert_parity(to64(fv[m])[rows], ref["fused_v"][m][rows], dtype, f"slide fused V {k_set},{m}")
+    for l in range(w.L):   # the outputs hold the second streamed chunk's
+        assert_parity(to64(r.new_o[l])[:, :, hs], second["hist_o"][l][:, :, hs], dtype, f"slide newest {l}")
+        assert_parity(to64(r.final_o[l])[:, :, hs][rows_f], second["final_o"][l][:, :, hs][rows_f], dtype,
+                      f"slide final {l}")
+        for i in range(w.n_euler_steps):
+            assert_parity(to64(r.act_o[i * w.L + l])[:, :, hs], second["act_o"][i][l][:, :, hs], dtype,
+                          f"slide action {i},{l}")

@@ -146,3 +146,21 @@ def test_error_message_is_thread_local_and_cleared():
     out = (ctypes.c_double * 3)()
     assert L.wam_flow_schedule(2, 0.5, 1.0, out) == 0
     assert _msg() == ""
+
+
+def test_copy_frames_rejects_bad_arguments():
+    lay = _lay(B=1, H=2, D=64, T=16, F=4)
+    nbytes = 4 * 16 * 2 * 64 * 4          # one fp32 tensor [1, F*T, H, D]
+    a, b = FAKE, FAKE + 4 * nbytes
+    pair = lambda x: (ctypes.c_void_p * 1)(x)
+    call = lambda n=1, s=pair(a), d=pair(b), fs=1, fd=0, nf=3: L.wam_copy_frames(
+        lay.ref, wam.F32, n, s, d, fs, fd, nf, None)
+    assert call(n=0) == 1 and "n must be" in _msg()
+    assert call(n=129) == 1 and "n must be" in _msg()
+    assert call(fs=2, nf=3) == 1 and "outside" in _msg()
+    assert call(fd=-1) == 1 and "outside" in _msg()
+    assert call(nf=-1) == 1 and "outside" in _msg()
+    assert call(d=pair(a + nbytes // 2)) == 1 and "overlap" in _msg()
+    assert call(d=pair(b + 4)) == 1 and "aligned" in _msg()
+    assert call(s=pair(0)) == 1 and "NULL" in _msg()
+    assert call(nf=0) == 0                   # nothing to copy: valid, launches nothing

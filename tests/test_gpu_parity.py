@@ -370,3 +370,20 @@ def test_prefill_tensor_core_large_logit_jumps(big_frame):
     wam.video_prefill_kv(lay, 0, F, q, k, v, torch.zeros_like(k), torch.zeros_like(v), o)
     ref = O.video_prefill(to64(q), to64(k), to64(v), None, None, np.zeros((1, F)), None, T, 0, F)
     assert_parity(to64(o), ref, "bf16", f"logit jumps, big frame {big_frame}")
+
+
+# ----------------------------------------------------------------------------- frame copies
+
+@pytest.mark.parametrize("tdt", [torch.bfloat16, torch.float32])
+def test_copy_frames_moves_whole_frames_of_every_episode(tdt):
+    B, H, D, T, F = 2, 3, 64, 16, 5
+    lay = wam.VideoLayout(B, H, D, T, F)
+    src = [dev_normal((B, F * T, H, D), 81, "src", j, dtype=tdt) for j in range(3)]
+    dst = [torch.full_like(x, SENTINEL) for x in src]
+    wam.copy_frames(lay, src, dst, 2, 1, 3)          # frames 2..4 -> 1..3
+    torch.cuda.synchronize()
+    for x, y in zip(src, dst):
+        assert torch.equal(y[:, T:4 * T], x[:, 2 * T:5 * T])
+        assert torch.all(y[:, :T] == SENTINEL) and torch.all(y[:, 4 * T:] == SENTINEL)
+    wam.copy_frames(lay, src, dst, 0, 0, 0)          # nothing to copy
+    torch.cuda.synchronize()

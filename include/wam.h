@@ -51,7 +51,7 @@ typedef struct CUstream_st* wam_stream_t; /* the same handle as cudaStream_t */
 typedef enum {
   WAM_OK = 0,
   WAM_ERR_INVALID_ARGUMENT = 1, /* a null pointer, bad size, misaligned pointer, bad range */
-  WAM_ERR_UNSUPPORTED = 2,      /* a valid request this build has no kernel for */
+  WAM_ERR_UNSUPPORTED = 2,      /* a valid request the library has no kernel for */
   WAM_ERR_CUDA = 3,             /* a CUDA runtime error while configuring or launching */
   WAM_ERR_WORKSPACE = 4,        /* a workspace that is missing or too small */
   WAM_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up (wam_device_error) */
@@ -264,7 +264,7 @@ wam_status wam_device_error(int32_t clear);
 /* Thread-local message of the last failing call on this thread ("" if none). */
 const char* wam_last_error(void);
 
-/* ABI version of this build: major * 10000 + minor * 100 + patch. */
+/* ABI version of the library: major * 10000 + minor * 100 + patch. */
 int32_t wam_version(void);
 
 #ifdef __cplusplus

@@ -64,6 +64,7 @@ struct Bars {
   uint64_t done;
   uint32_t tmem_base;
   int abort;
+  int unit_next;  // next unclaimed unit of the store + fusion pool
 };
 
 constexpr int kSmemBytes = 1024 + (2 + kKStages + kVStages) * kTile + int(sizeof(Bars)) + 64;
@@ -84,64 +85,83 @@ __device__ __forceinline__ void red_add_v4(float* acc, float a0, float a1, float
                : "memory");
 }
 
-// Store the CTA's own new K or V rows into the layer's cache and fold them into the fusion
-// accumulator, straight from the call's input (64 threads, `rows` tokens from row0_in of the
-// input to row0_out of the cache).  The first layer of an interval writes w x, a middle layer
-// adds w x by L2 reductions (nothing to wait for), the last reads the sum and writes the fused
-// bf16 pair.  Each thread keeps 4 chunks of 8 elements in flight (more measured slower).
-__device__ __forceinline__ void store_fuse_rows(const PrefillArgs& a, const void* in_base,
+// One unit of the cache store + fusion epilogue: 8 consecutive own token rows of the new K or V
+// (128 chunks of 8 elements, 4 per lane of one warp; row0_in is the unit's first row in the
+// call's input, row0_out in the cache).  The rows are copied into the layer's cache and folded
+// into the fusion accumulator: the first layer of an interval writes w x, a middle layer adds
+// w x by L2 reductions (nothing to wait for), the last reads the sum and writes the fused bf16
+// pair.  4 chunks in flight per lane (8 measured slower).
+__device__ __forceinline__ void store_fuse_unit(const PrefillArgs& a, const void* in_base,
                                                 void* store_base, float* acc_base,
                                                 void* fused_base, int64_t row0_in,
-                                                int64_t row0_out, int rows, int h, int t) {
+                                                int64_t row0_out, int h, int lane) {
   constexpr int kU = 4;
-  const int chunks = rows * 16;
   const bool need_acc = a.fuse_on && !a.fuse_first && a.fuse_last;
   const bool middle = a.fuse_on && !a.fuse_first && !a.fuse_last;
-  for (int c0 = t; c0 < chunks; c0 += 64 * kU) {
-    uint4 raw[kU];
-    float4 p0[kU], p1[kU];
-    int64_t off[kU];
+  uint4 raw[kU];
+  float4 p0[kU], p1[kU];
+  int64_t off[kU];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int c = c0 + 64 * u, r = c >> 4, cc = (c & 15) * 8;
-      if (c >= chunks) continue;
-      raw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(in_base) +
-                                               ((row0_in + r) * a.H + h) * 128 + cc);
-      off[u] = ((row0_out + r) * a.H + h) * 128 + cc;
-      if (need_acc) {
-        p0[u] = *reinterpret_cast<const float4*>(acc_base + off[u]);
-        p1[u] = *reinterpret_cast<const float4*>(acc_base + off[u] + 4);
-      }
+  for (int u = 0; u < kU; ++u) {
+    const int c = lane + 32 * u, r = c >> 4, cc = (c & 15) * 8;
+    raw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(in_base) +
+                                             ((row0_in + r) * a.H + h) * 128 + cc);
+    off[u] = ((row0_out + r) * a.H + h) * 128 + cc;
+    if (need_acc) {
+      p0[u] = *reinterpret_cast<const float4*>(acc_base + off[u]);
+      p1[u] = *reinterpret_cast<const float4*>(acc_base + off[u] + 4);
     }
+  }
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      if (c0 + 64 * u >= chunks) continue;
-      if (store_base)
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(store_base) + off[u]) = raw[u];
-      if (!a.fuse_on) continue;
-      const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
-      float s[8];
-      if (need_acc) {
-        const float p[8] = {p0[u].x, p0[u].y, p0[u].z, p0[u].w, p1[u].x, p1[u].y, p1[u].z, p1[u].w};
+  for (int u = 0; u < kU; ++u) {
+    if (store_base)
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(store_base) + off[u]) = raw[u];
+    if (!a.fuse_on) continue;
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+    float s[8];
+    if (need_acc) {
+      const float p[8] = {p0[u].x, p0[u].y, p0[u].z, p0[u].w, p1[u].x, p1[u].y, p1[u].z, p1[u].w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = fmaf(a.fuse_w, __bfloat162float(x[j]), p[j]);
-      } else {
+      for (int j = 0; j < 8; ++j) s[j] = fmaf(a.fuse_w, __bfloat162float(x[j]), p[j]);
+    } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = a.fuse_w * __bfloat162float(x[j]);
-      }
-      if (middle) {
-        red_add_v4(acc_base + off[u], s[0], s[1], s[2], s[3]);
-        red_add_v4(acc_base + off[u] + 4, s[4], s[5], s[6], s[7]);
-      } else if (a.fuse_last) {
-        uint4 v;
-        v.x = pack_bf16(s[0], s[1]), v.y = pack_bf16(s[2], s[3]);
-        v.z = pack_bf16(s[4], s[5]), v.w = pack_bf16(s[6], s[7]);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(fused_base) + off[u]) = v;
-      } else {
-        *reinterpret_cast<float4*>(acc_base + off[u]) = make_float4(s[0], s[1], s[2], s[3]);
-        *reinterpret_cast<float4*>(acc_base + off[u] + 4) = make_float4(s[4], s[5], s[6], s[7]);
-      }
+      for (int j = 0; j < 8; ++j) s[j] = a.fuse_w * __bfloat162float(x[j]);
     }
+    if (middle) {
+      red_add_v4(acc_base + off[u], s[0], s[1], s[2], s[3]);
+      red_add_v4(acc_base + off[u] + 4, s[4], s[5], s[6], s[7]);
+    } else if (a.fuse_last) {
+      uint4 v;
+      v.x = pack_bf16(s[0], s[1]), v.y = pack_bf16(s[2], s[3]);
+      v.z = pack_bf16(s[4], s[5]), v.w = pack_bf16(s[6], s[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(fused_base) + off[u]) = v;
+    } else {
+      *reinterpret_cast<float4*>(acc_base + off[u]) = make_float4(s[0], s[1], s[2], s[3]);
+      *reinterpret_cast<float4*>(acc_base + off[u] + 4) = make_float4(s[4], s[5], s[6], s[7]);
+    }
+  }
+}
+
+// The CTA's store + fusion work as a pool of units (K units first, then V), claimed one at a
+// time through a shared-memory counter by whole warps: the helper warps from the start, each
+// softmax warp once its output is written, so a CTA with few key tiles does not wait on two
+// warps for its epilogue.  `rows` (a multiple of 8) own tokens from row_in / row_out.
+__device__ __forceinline__ void store_fuse_pool(const PrefillArgs& a, int* next, int rows,
+                                                int64_t row_in, int64_t row_out, int h,
+                                                int lane) {
+  if (a.k_store == nullptr && !a.fuse_on) return;
+  const int per = rows / 8;
+  for (;;) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(next, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= 2 * per) break;
+    if (u < per)
+      store_fuse_unit(a, a.k_new, a.k_store, a.acc_k, a.fused_k, row_in + 8 * u,
+                      row_out + 8 * u, h, lane);
+    else
+      store_fuse_unit(a, a.v_new, a.v_store, a.acc_v, a.fused_v, row_in + 8 * (u - per),
+                      row_out + 8 * (u - per), h, lane);
   }
 }
 
@@ -287,6 +307,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     }
     mbar_init(&bars.done, 1);
     bars.abort = 0;
+    bars.unit_next = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -392,18 +413,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       }
       tc05::mma_commit(&bars.done);  // arrives once every MMA issued above has completed
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ cache store + fusion
-    // The CTA's own tokens, read from the call's new K/V while the attention loop runs.
-    const int t = threadIdx.x - 64;
-    if (a.k_store != nullptr || a.fuse_on) {
-      const int64_t N = int64_t(a.F) * a.T, qtok = int64_t(a.f_end - a.f_begin) * a.T;
-      const int64_t row_in = int64_t(b) * qtok + qtok0;
-      const int64_t row_out = int64_t(b) * N + int64_t(f) * a.T + qp * 2 * kBM;
-      store_fuse_rows(a, a.k_new, a.k_store, a.acc_k, a.fused_k, row_in, row_out, nq * kBN, h, t);
-      store_fuse_rows(a, a.v_new, a.v_store, a.acc_v, a.fused_v, row_in, row_out, nq * kBN, h, t);
-    }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax, one row per thread
     // tcgen05.ld / tcgen05.st are warp-collective: every decision in front of one is voted
     // across the warp, so all 32 lanes always execute them together.
@@ -546,6 +556,16 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         }
       }
     }
+  }
+  if (warp >= 2) {
+    // ------------------------------------------------------------ cache store + fusion
+    // The CTA's own tokens, read from the call's new K/V: the helper warps start at once, while
+    // the attention loop runs; each softmax warp joins once its output is written (converged:
+    // every branch in the softmax is warp-uniform).
+    // first own token row in the call's new K/V and in the layer's cache
+    const int64_t own_in = int64_t(b) * (int64_t(a.f_end - a.f_begin) * a.T) + qtok0;
+    const int64_t own_out = int64_t(b) * (int64_t(a.F) * a.T) + int64_t(f) * a.T + qp * 2 * kBM;
+    store_fuse_pool(a, &bars.unit_next, nq * kBM, own_in, own_out, h, lane);
   }
 
   // ------------------------------------------------------------ teardown

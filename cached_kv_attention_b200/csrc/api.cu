@@ -6,7 +6,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
 #include <string>
 #include <vector>
 
@@ -174,6 +176,62 @@ wam_status check_range(const Geo& g, int f_begin, int f_end) {
 
 // Tensor-core eligibility of a bf16 video/action call.
 bool tc_video_ok(const Geo& g, wam_dtype dt) { return dt == WAM_BF16 && g.D == 128 && g.T % 128 == 0; }
+
+// Launch order of the tensor-core prefill's work items (one resident CTA per SM; the CTAs of
+// an item are consecutive blocks).  The block scheduler hands blocks to SMs in index order
+// as SMs free up, and a pass holds only a few CTAs per SM, so longest-first can end in a wave
+// of short CTAs on a mostly idle GPU.  Candidates are longest-first and, for each class of
+// equal key-frame count, that class moved right behind the longest class or to the end; each
+// is scored by replaying that dispatch with a cost of (key tiles + a fixed 5-tile prologue
+// and epilogue) per CTA.  The cheapest order is kept, longest-first on ties.  Results do not
+// depend on the order: every CTA writes only its own rows.
+void order_items_for_tc(const Geo& g, wam::FrameLists& fl) {
+  constexpr int kOverheadTiles = 5;
+  constexpr int64_t kMaxReplayBlocks = 60000;  // bound on host work per call
+  const int n = fl.n_items, sms = sm_count();
+  const int tpf = g.T / 128, QP = (g.T / 128 + 1) / 2;
+  const int64_t per_item = int64_t(QP) * g.H;
+  if (n < 2 || sms <= 0 || int64_t(n) * per_item <= sms) return;  // one wave: any order
+  std::vector<int> nk;                          // classes, longest first (items are sorted)
+  std::vector<std::vector<uint32_t>> members;
+  for (int i = 0; i < n; ++i) {
+    const int k = wam::item_nk(fl.item[i]);
+    if (nk.empty() || nk.back() != k) nk.push_back(k), members.emplace_back();
+    members.back().push_back(fl.item[i]);
+  }
+  const int C = int(nk.size());
+  if (C < 2 || int64_t(2 * C - 1) * n * per_item > kMaxReplayBlocks) return;
+  auto makespan = [&](const std::vector<int>& order) {
+    std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> free_at;
+    for (int i = 0; i < sms; ++i) free_at.push(0);
+    int64_t end = 0;
+    for (int c : order) {
+      const int64_t cost = int64_t(nk[c]) * tpf + kOverheadTiles;
+      for (int64_t m = int64_t(members[c].size()) * per_item; m > 0; --m) {
+        const int64_t e = free_at.top() + cost;
+        free_at.pop();
+        free_at.push(e);
+        end = std::max(end, e);
+      }
+    }
+    return end;
+  };
+  std::vector<int> best(C);
+  for (int c = 0; c < C; ++c) best[c] = c;
+  int64_t best_t = makespan(best);
+  const std::vector<int> lpt = best;
+  for (int c = 1; c < C; ++c)
+    for (int where : {1, C - 1}) {
+      std::vector<int> o = lpt;
+      o.erase(o.begin() + c);
+      o.insert(o.begin() + where, c);
+      const int64_t t = makespan(o);
+      if (t < best_t) best_t = t, best = o;
+    }
+  int i = 0;
+  for (int c : best)
+    for (uint32_t it : members[c]) fl.item[i++] = it;
+}
 bool tc_action_ok(const Geo& g, wam_dtype dt, int n_act) {
   return dt == WAM_BF16 && g.D == 128 && g.T % 64 == 0 && n_act <= 32;
 }
@@ -352,6 +410,7 @@ wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf16 = dt == WAM_BF16;
   if (tc_video_ok(g, dt)) {
+    order_items_for_tc(g, a.fl);
     cudaError_t e = wam::launch_prefill_tc(a, s);
     if (e != cudaErrorNotSupported) return cuda_status(e, "wam_video_prefill_kv (tensor cores)");
   }

@@ -502,16 +502,22 @@ __device__ __forceinline__ bool softmax_any(bool v) {
       : "memory");
   return r != 0;
 }
-// Every thread of every CTA of the cluster; shared-memory writes before it are visible after.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
 // A float in CTA `peer`'s shared memory at the offset of `local` in this CTA's.
 __device__ __forceinline__ float ld_peer(const float* local, uint32_t peer) {
   uint32_t pa;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(pa) : "r"(smem_u32(local)), "r"(peer));
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(pa) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_peer4(const float* local, uint32_t peer) {
+  uint32_t pa;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(pa) : "r"(smem_u32(local)), "r"(peer));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(pa)
+               : "memory");
   return v;
 }
 // After the call lane q holds the max (or sum) over the warp's lanes of v[q]; v is clobbered.
@@ -844,49 +850,79 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   if (k > 1) {
     // ---------------------------------------------------------------- merge over the cluster
     __syncwarp();
-    cluster_sync_all();  // every CTA's partial is in its shared memory
-    if (warp >= 2) {
-      const int L = 32 * (warp & 3) + lane;
+    // Every CTA's partial is in its shared memory after this barrier.  Only the softmax warps
+    // wrote it, so only they arrive with release semantics: a release arrive of the TMA and MMA
+    // warps measured ~2 us on B200 and held up the whole cluster.
+    if (warp >= 2)
+      asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+    else
+      asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+    {
+      // One query row per half-warp (all 6 warps; at most 2 rows each, a rank has <= 16), 8
+      // columns per lane: every peer's (m, l) and its 32 bytes of the partial row are loaded
+      // before any is used (one round trip per row).  The CTA arrives on the closing cluster
+      // barrier once its peer reads are done and only then stores O.  That arrive is relaxed:
+      // it orders nothing, it only says that this thread's peer loads, whose values it has
+      // already consumed, can no longer touch a peer's shared memory.
+      const int hw = threadIdx.x >> 4, c0 = 8 * (threadIdx.x & 15);
       const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k;
       const float* part = reinterpret_cast<const float*>(sP);
-      // four rows at a time, every peer's (m, l, O) loads of them issued before any is used
-      for (int q0 = r0; q0 < r1; q0 += 4) {
-        float pm[4][kMaxSplit], pl_[4][kMaxSplit], po[4][kMaxSplit];
+      float val[2][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+      for (int rr = 0; rr < 2; ++rr) {
+        const int q = r0 + hw + rr * (um::kThreads / 16);
+        if (q >= r1) continue;
+        float pm[kMaxSplit], pl_[kMaxSplit];
+        float4 pa[kMaxSplit], pb[kMaxSplit];
 #pragma unroll
-          for (int p = 0; p < kMaxSplit; ++p) {
-            if (p >= k || q0 + u >= r1) continue;
-            pm[u][p] = ld_peer(&bars.part_m[q0 + u], uint32_t(p));
-            pl_[u][p] = ld_peer(&bars.part_l[q0 + u], uint32_t(p));
-            po[u][p] = ld_peer(part + (q0 + u) * 128 + L, uint32_t(p));
-          }
+        for (int p = 0; p < kMaxSplit; ++p) {
+          if (p >= k) continue;
+          pm[p] = ld_peer(&bars.part_m[q], uint32_t(p));
+          pl_[p] = ld_peer(&bars.part_l[q], uint32_t(p));
+          pa[p] = ld_peer4(part + q * 128 + c0, uint32_t(p));
+          pb[p] = ld_peer4(part + q * 128 + c0 + 4, uint32_t(p));
+        }
+        float M = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = q0 + u;
-          if (q >= r1) continue;
-          float M = -INFINITY;
+        for (int p = 0; p < kMaxSplit; ++p)
+          if (p < k) M = fmaxf(M, pm[p]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
 #pragma unroll
-          for (int p = 0; p < kMaxSplit; ++p)
-            if (p < k) M = fmaxf(M, pm[u][p]);
-          const float Mu = M == -INFINITY ? 0.f : M;
-          float num = 0.f, den = 0.f;
+        for (int p = 0; p < kMaxSplit; ++p) {
+          if (p >= k) continue;
+          const float wgt = exp2f(pm[p] - Mu);
+          den = fmaf(wgt, pl_[p], den);
+          num[0] = fmaf(wgt, pa[p].x, num[0]), num[1] = fmaf(wgt, pa[p].y, num[1]);
+          num[2] = fmaf(wgt, pa[p].z, num[2]), num[3] = fmaf(wgt, pa[p].w, num[3]);
+          num[4] = fmaf(wgt, pb[p].x, num[4]), num[5] = fmaf(wgt, pb[p].y, num[5]);
+          num[6] = fmaf(wgt, pb[p].z, num[6]), num[7] = fmaf(wgt, pb[p].w, num[7]);
+        }
 #pragma unroll
-          for (int p = 0; p < kMaxSplit; ++p) {
-            if (p >= k) continue;
-            const float wgt = exp2f(pm[u][p] - Mu);
-            num = fmaf(wgt, po[u][p], num);
-            den = fmaf(wgt, pl_[u][p], den);
-          }
-          const float val = den > 0.f ? num / den : 0.f;
-          const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
-          if (a.o_f32) static_cast<float*>(a.o)[off] = val;
-          else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
+        for (int e = 0; e < 8; ++e) val[rr][e] = den > 0.f ? num[e] / den : 0.f;
+      }
+      __syncwarp();
+      asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");  // peer reads done
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int q = r0 + hw + rr * (um::kThreads / 16);
+        if (q >= r1) continue;
+        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + c0;
+        if (a.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
+          dst[0] = make_float4(val[rr][0], val[rr][1], val[rr][2], val[rr][3]);
+          dst[1] = make_float4(val[rr][4], val[rr][5], val[rr][6], val[rr][7]);
+        } else {
+          uint4 u;
+          u.x = pack_bf16(val[rr][0], val[rr][1]), u.y = pack_bf16(val[rr][2], val[rr][3]);
+          u.z = pack_bf16(val[rr][4], val[rr][5]), u.w = pack_bf16(val[rr][6], val[rr][7]);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off) = u;
         }
       }
+      // no CTA leaves while a peer may still read its shared memory
+      asm volatile("barrier.cluster.wait;" ::: "memory");
     }
-    __syncwarp();
-    cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
   }
 
   // ---------------------------------------------------------------- teardown

@@ -321,10 +321,13 @@ IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 79.2e6}
 def time_fused_read(runner, stream, n=20) -> float:
     """Mean device time (ms) of one fused-cache action read of the prepared chunk.  The call is
     captured once in a CUDA graph; each sample replays it right after a 256 MB write that
-    flushes the L2 (and keeps the GPU busy while the replay is submitted), with CUDA events
-    around the replay alone."""
+    flushes the L2 and a 256 MB read of another buffer, which evicts the write's dirty lines
+    (otherwise the timed read also pays for writing them back) and keeps the GPU busy while
+    the replay is submitted, with CUDA events around the replay alone."""
     fn, args = runner.calls[runner.fused_read_call]
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    clean = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    total = torch.zeros((), dtype=torch.float32, device="cuda")
     st = fn(*args)  # the call once outside capture (one-time per-device set-up)
     if st:
         raise RuntimeError(f"fused read call failed: {st}")
@@ -337,6 +340,7 @@ def time_fused_read(runner, stream, n=20) -> float:
     ts = []
     for i in range(n + 3):
         flush.fill_(float(i))
+        torch.sum(clean, dim=0, out=total)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -345,7 +349,7 @@ def time_fused_read(runner, stream, n=20) -> float:
         torch.cuda.synchronize()
         if i >= 3:
             ts.append(a.elapsed_time(b))
-    del g
+    del g, flush, clean, total
     return statistics.mean(ts)
 
 

@@ -185,10 +185,10 @@ bool tc_video_ok(const Geo& g, wam_dtype dt) { return dt == WAM_BF16 && g.D == 1
 // is scored by replaying that dispatch with a cost of (key tiles + a fixed 5-tile prologue
 // and epilogue) per CTA.  The cheapest order is kept, longest-first on ties.  Results do not
 // depend on the order: every CTA writes only its own rows.
-void order_items_for_tc(const Geo& g, wam::FrameLists& fl) {
+void order_items_for_tc(const Geo& g, wam::FrameLists& fl, int sms) {
   constexpr int kOverheadTiles = 5;
   constexpr int64_t kMaxReplayBlocks = 60000;  // bound on host work per call
-  const int n = fl.n_items, sms = sm_count();
+  const int n = fl.n_items;
   const int tpf = g.T / 128, QP = (g.T / 128 + 1) / 2;
   const int64_t per_item = int64_t(QP) * g.H;
   if (n < 2 || sms <= 0 || int64_t(n) * per_item <= sms) return;  // one wave: any order
@@ -410,7 +410,7 @@ wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf16 = dt == WAM_BF16;
   if (tc_video_ok(g, dt)) {
-    order_items_for_tc(g, a.fl);
+    order_items_for_tc(g, a.fl, sm_count());
     cudaError_t e = wam::launch_prefill_tc(a, s);
     if (e != cudaErrorNotSupported) return cuda_status(e, "wam_video_prefill_kv (tensor cores)");
   }
@@ -550,6 +550,30 @@ wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin,
   fill_items(g, f_begin, f_end, a.fl);
   return cuda_status(wam::launch_debug_mask(a, mask, reinterpret_cast<cudaStream_t>(stream)),
                      "wam_debug_video_mask");
+}
+
+wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
+                                   int32_t n_sms, int32_t* episode, int32_t* frame,
+                                   int32_t* n_key_frames, int32_t* n_items) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_range(g, f_begin, f_end));
+  if (!episode || !frame || !n_key_frames || !n_items)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "an output pointer is NULL");
+  if (g.T % 128 != 0)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "T = %d is not a multiple of 128", g.T);
+  static thread_local wam::PrefillArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fill_vlists(g, a.fl);
+  fill_items(g, f_begin, f_end, a.fl);
+  order_items_for_tc(g, a.fl, n_sms);
+  for (int i = 0; i < a.fl.n_items; ++i) {
+    episode[i] = wam::item_b(a.fl.item[i]);
+    frame[i] = wam::item_f(a.fl.item[i]);
+    n_key_frames[i] = wam::item_nk(a.fl.item[i]);
+  }
+  *n_items = a.fl.n_items;
+  return WAM_OK;
 }
 
 wam_status wam_device_error(int32_t clear) {

@@ -17,7 +17,7 @@ __all__ = [
     "video_prefill_kv", "fuse_interval_kv", "action_attn", "flow_euler_step",
     "flow_schedule", "fuse_weights", "debug_video_mask", "device_error", "exported_names",
     "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS", "action_attn_workspace_size",
-    "action_workspace",
+    "action_workspace", "debug_prefill_order",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
@@ -65,6 +65,8 @@ def _load() -> ctypes.CDLL:
         "wam_flow_schedule": [i32, f64, f64, ctypes.POINTER(f64)],
         "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
         "wam_debug_video_mask": [lay, i32, i32, vp, vp],
+        "wam_debug_prefill_order": [lay, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                    ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "wam_device_error": [i32],
         "wam_video_prefill_kv_fuse_noalloc": [lay, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp,
                                               i32, f32, i32, i32, vp, vp, vp],
@@ -89,7 +91,7 @@ def exported_names() -> list:
             "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
             "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
             "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size",
-            "wam_copy_frames"]
+            "wam_copy_frames", "wam_debug_prefill_order"]
 
 
 def check(status: int) -> None:
@@ -261,6 +263,18 @@ def debug_video_mask(layout: VideoLayout, f_begin: int, f_end: int, stream=None)
                        device="cuda")
     check(lib.wam_debug_video_mask(layout.ref, f_begin, f_end, _ptr(mask), _stream(stream)))
     return mask
+
+
+def debug_prefill_order(layout: VideoLayout, f_begin: int, f_end: int, n_sms: int):
+    """Work items of a tensor-core prefill call over [f_begin, f_end) in launch order for a
+    device of n_sms SMs (host only): int32 arrays (episode, frame, n_key_frames)."""
+    cap = max(layout.B * (f_end - f_begin), 1)
+    ep, fr, nk = (np.zeros(cap, dtype=np.int32) for _ in range(3))
+    n = ctypes.c_int32(0)
+    P = ctypes.POINTER(ctypes.c_int32)
+    check(lib.wam_debug_prefill_order(layout.ref, f_begin, f_end, n_sms, ep.ctypes.data_as(P),
+                                      fr.ctypes.data_as(P), nk.ctypes.data_as(P), ctypes.byref(n)))
+    return ep[:n.value], fr[:n.value], nk[:n.value]
 
 
 def device_error(clear: bool = True) -> None:

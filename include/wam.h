@@ -255,6 +255,22 @@ wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin,
                                 uint8_t* mask, wam_stream_t stream);
 
 /*
+ * The work items of a bf16, D = 128 tensor-core prefill call over frames [f_begin, f_end)
+ * (T % 128 == 0), in the order the call launches them on a device with n_sms SMs; host only,
+ * no GPU needed.  An item is one valid query frame of one episode with the number of valid
+ * key frames it reads; it runs as ceil(T / 256) x H consecutive CTAs, one resident per SM.
+ * The order starts from longest first; each class of equal key-frame count is also tried right
+ * behind the longest class and at the end, every candidate is scored by replaying in-order
+ * dispatch of its CTAs onto n_sms SMs (cost per CTA: key tiles + 5), and the cheapest is
+ * kept (longest first on ties; n_sms <= 0, or a single wave, keeps longest first).
+ *   episode, frame, n_key_frames: host int32 arrays with room for B * (f_end - f_begin);
+ *   *n_items receives the number of items written.
+ */
+wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
+                                   int32_t n_sms, int32_t* episode, int32_t* frame,
+                                   int32_t* n_key_frames, int32_t* n_items);
+
+/*
  * Synchronise the current device and report its error word: WAM_OK, or WAM_ERR_TIMEOUT when
  * a kernel's bounded wait on an mbarrier gave up (the kernel then skipped its remaining work
  * and returned without faulting).  clear != 0 resets the word.  Host-blocking.

@@ -1,0 +1,104 @@
+"""Launch order of the tensor-core prefill's work items (host logic, CPU only).
+
+The library picks the order in which a prefill call's work items (one valid query frame of one
+episode) are launched by replaying the block scheduler's in-order dispatch onto one CTA per SM.
+These tests read that order through `wam_debug_prefill_order` and check it against an
+independent count of each item's key frames, against longest-first, and against a replay of
+the dispatch written here."""
+
+import heapq
+
+import numpy as np
+import pytest
+
+from cached_kv_attention_b200 import synth, wam
+
+B200_SMS = 148
+
+
+def layout_of(name, T=None):
+    w = synth.WORKLOADS[name]
+    if T is not None:
+        w = w.replace(T=T)
+    return w, wam.VideoLayout(w.B, w.H, w.D, w.T, w.F, synth.pad_mask(w).numpy())
+
+
+def key_frames(w, b, f):
+    """Valid frames an item of frame f reads: every non-padding frame up to f (one frame per
+    attention block, the layouts' default)."""
+    pad = synth.pad_mask(w).numpy()
+    return int(sum(1 for u in range(f + 1) if not pad[b, u]))
+
+
+def makespan(nk, w, sms):
+    """In-order dispatch of every item's CTAs (ceil(T / 256) x H each, cost key tiles + 5) onto
+    `sms` SMs, each CTA to the SM that frees first; returns when the last one ends."""
+    per_item = (w.T // 128 + 1) // 2 * w.H
+    free = [0] * sms
+    end = 0
+    for k in nk:
+        cost = int(k) * (w.T // 128) + 5
+        for _ in range(per_item):
+            t = heapq.heappop(free) + cost
+            heapq.heappush(free, t)
+            end = max(end, t)
+    return end
+
+
+RANGES = {
+    "history": lambda w: (0, w.F_h),
+    "imagination": lambda w: (w.F_h, w.F),
+    "all": lambda w: (0, w.F),
+}
+
+
+@pytest.mark.parametrize("name", ["ctx19.2s_bf16", "ctx2.4s_bf16", "ctx38.4s_bf16", "batched4_bf16"])
+@pytest.mark.parametrize("rng", sorted(RANGES))
+@pytest.mark.parametrize("sms", [0, 16, B200_SMS, 1000])
+def test_order_is_a_permutation_no_worse_than_longest_first(name, rng, sms):
+    w, lay = layout_of(name)
+    f0, f1 = RANGES[rng](w)
+    ep, fr, nk = wam.debug_prefill_order(lay, f0, f1, sms)
+    ep0, fr0, nk0 = wam.debug_prefill_order(lay, f0, f1, 0)
+    pad = synth.pad_mask(w).numpy()
+    # every valid query frame of every episode exactly once, with its key-frame count
+    want = sorted((b, f) for b in range(w.B) for f in range(f0, f1) if not pad[b, f])
+    assert sorted(zip(ep.tolist(), fr.tolist())) == want
+    for b, f, k in zip(ep, fr, nk):
+        assert k == key_frames(w, int(b), int(f))
+    # n_sms = 0 is longest first (ties in episode, frame order); any other order is a
+    # permutation of it that the dispatch replay scores no worse
+    assert np.all(np.diff(nk0) <= 0)
+    assert sorted(zip(ep0.tolist(), fr0.tolist(), nk0.tolist())) == \
+        sorted(zip(ep.tolist(), fr.tolist(), nk.tolist()))
+    if sms > 0:
+        assert makespan(nk, w, sms) <= makespan(nk0, w, sms)
+
+
+def test_history_pass_of_the_19_2s_chunk_on_148_sms():
+    # 5 valid history frames (19 of 24 padded): items of 5, 4, 3, 2, 1 key frames, 72 CTAs
+    # each on 148 SMs.  Longest first leaves the 72 one-frame CTAs in a last wave; the order
+    # picked runs the two-frame items right behind the five-frame ones.
+    w, lay = layout_of("ctx19.2s_bf16")
+    ep, fr, nk = wam.debug_prefill_order(lay, 0, w.F_h, B200_SMS)
+    assert nk.tolist() == [5, 2, 4, 3, 1]
+    assert fr.tolist() == [23, 20, 22, 21, 19] and ep.tolist() == [0] * 5
+    assert makespan(nk, w, B200_SMS) < makespan(sorted(nk, reverse=True), w, B200_SMS)
+
+
+def test_single_wave_keeps_longest_first():
+    # the two imagined frames: 2 x 72 = 144 CTAs fit on 148 SMs at once
+    w, lay = layout_of("ctx19.2s_bf16")
+    ep, fr, nk = wam.debug_prefill_order(lay, w.F_h, w.F, B200_SMS)
+    n_hist = w.F_h - int(synth.pad_mask(w).numpy()[0].sum())  # 5 valid history frames
+    assert nk.tolist() == [n_hist + 2, n_hist + 1]  # each imagined frame also reads the ones before it
+    assert fr.tolist() == [w.F - 1, w.F - 2]
+
+
+def test_rejects_layouts_without_a_tensor_core_prefill():
+    w, lay = layout_of("ctx19.2s_bf16", T=64)
+    with pytest.raises(wam.WamError):
+        wam.debug_prefill_order(lay, 0, w.F_h, B200_SMS)
+    w, lay = layout_of("ctx19.2s_bf16")
+    with pytest.raises(wam.WamError):
+        wam.debug_prefill_order(lay, 3, 2, B200_SMS)

@@ -19,7 +19,7 @@ Sources (page title, section):
             (greeksharifa.github.io), §3.1-3.3, §4.2, App. B.2
   [FSW]     "世界模型之Faster-WAM详解" (171host.com), §3.1-3.4
 
-Readings taken where the pages leave a step open (each is also listed in the design doc):
+Readings taken where the pages leave a step open:
   R1  schedule warp phi = identity (shift 1); the rescale that lands on sigma* is the affine
       map sigma = sigma* + (1 - sigma*) * phi(u), the only affine map pinning both ends.
   R2  one attention block = one latent frame unless ``frame_block`` groups frames.

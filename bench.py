@@ -312,9 +312,9 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------------------ this library
 
-# DRAM bytes (read + write) of one imagination-pass prefill launch, from one ncu capture of
-# the same kernel (profiles/prefill_tc_ctx19.2s_imagination.md); the stride variants launch
-# the identical imagination pass, other workloads report None.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one imagination-pass prefill
+# launch, from one ncu capture of the same kernel (`bench.py --profile-call future`); the
+# stride variants launch the identical imagination pass, other workloads report None.
 IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 80.3e6}
 
 

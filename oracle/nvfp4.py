@@ -28,13 +28,15 @@ float32).  Values are decoded to float64.
 
 from __future__ import annotations
 
-from typing import Tuple
+from typing import Optional, Tuple
 
 import numpy as np
 
+from oracle.wam_oracle import action_attention
+
 __all__ = [
     "E2M1_MAGNITUDES", "e2m1_decode", "e2m1_encode", "e4m3_values", "e4m3_decode",
-    "e4m3_encode", "quantize", "dequantize", "BLOCK",
+    "e4m3_encode", "quantize", "dequantize", "BLOCK", "quantize_cache", "action_attention_nvfp4",
 ]
 
 BLOCK = 16
@@ -138,3 +140,21 @@ def dequantize(codes, s_b_codes, s_g) -> np.ndarray:
     vals = e2m1_decode(codes).reshape(codes.shape[:-1] + (D // BLOCK, BLOCK))
     scale = e4m3_decode(s_b_codes) * np.float64(s_g)
     return (vals * scale[..., None]).reshape(codes.shape)
+
+
+def quantize_cache(x, pad, T: int) -> Tuple[np.ndarray, np.ndarray, np.float32]:
+    """NVFP4 encoding of a fused K or V cache [B, F*T, H, D] over its valid frames.  Rows of
+    padded frames are never read (reading R3), so they take no part in the tensor's amax and
+    encode as 0, whatever they hold."""
+    x = np.asarray(x, dtype=_F32)
+    valid = ~np.repeat(np.asarray(pad).astype(bool), T, axis=1)  # [B, F*T]
+    return quantize(np.where(valid[:, :, None, None], x, _F32(0)))
+
+
+def action_attention_nvfp4(qa, ka, va, fk, fv, pad, T: int,
+                           scale: Optional[float] = None, heads=None) -> np.ndarray:
+    """The action read over an NVFP4 fused pair: ``fk`` and ``fv`` are (codes, block scale
+    codes, s_g) as ``quantize_cache`` returns them; the cache enters the attention as its
+    decoded float64 values, everything else as in the bf16 read."""
+    return action_attention(qa, ka, va, dequantize(*fk), dequantize(*fv), pad, T,
+                            scale=scale, heads=heads)

@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 from oracle import nvfp4 as Q
+from oracle import wam_oracle as O
 
 RNG = np.random.default_rng(20241202)
 
@@ -116,3 +117,40 @@ def test_zero_tensor_and_zero_block():
 def test_storage_is_about_3_6_times_smaller_than_bf16():
     bits = 4 + 8 / Q.BLOCK  # one E2M1 per element, one E4M3 per 16 (the per-tensor FP32 is negligible)
     assert abs(16 / bits - 3.6) < 0.05
+
+
+def test_cache_encoding_ignores_padded_frames():
+    B, F, T, H, D = 2, 3, 4, 2, 32
+    pad = np.array([[1, 0, 0], [0, 0, 1]], dtype=np.uint8)
+    x = bf16_exact(RNG.standard_normal((B, F * T, H, D)).astype(np.float32))
+    y = x.copy()
+    rows = np.repeat(pad.astype(bool), T, axis=1)
+    y[rows] = np.float32(np.nan)  # whatever a padded frame holds
+    y[0, 0, 0, 0] = np.float32(1e30)
+    cx, sx, gx = Q.quantize_cache(x, pad, T)
+    cy, sy, gy = Q.quantize_cache(y, pad, T)
+    assert gx == gy and np.array_equal(cx, cy) and np.array_equal(sx, sy)
+    assert not cx[rows].any() and not sx[rows].any()
+    # valid rows alone: the same as encoding the tensor with padded rows zeroed
+    z = np.where(rows[:, :, None, None], np.float32(0), x)
+    assert np.array_equal(Q.quantize(z)[0], cx)
+
+
+def test_nvfp4_read_of_a_grid_exact_cache_is_the_bf16_read():
+    # a fused pair whose values are already NVFP4 values decodes to itself, so the NVFP4 read
+    # must equal the plain read of the same values
+    B, F, T, H, D, n = 1, 2, 4, 2, 32, 3
+    pad = np.array([[0, 0]], dtype=np.uint8)
+    grid = Q.e2m1_decode(np.arange(16))
+    def cache():
+        codes = RNG.integers(0, 16, size=(B, F * T, H, D))
+        codes[..., ::16] = 7
+        s_b = 2.0 ** RNG.integers(-3, 3, size=(B, F * T, H, D // 16))
+        s_b[0, 0, 0, 0] = 448.0  # the tensor's largest block: s_g = 2^-10
+        v = grid[codes].reshape(B, F * T, H, D // 16, 16) * s_b[..., None] * 2.0 ** -10
+        return v.reshape(B, F * T, H, D).astype(np.float32)
+    fk, fv = cache(), cache()
+    qa, ka, va = (bf16_exact(RNG.standard_normal((B, n, H, D)).astype(np.float32)) for _ in range(3))
+    got = Q.action_attention_nvfp4(qa, ka, va, Q.quantize_cache(fk, pad, T), Q.quantize_cache(fv, pad, T), pad, T)
+    want = O.action_attention(qa, ka, va, fk, fv, pad, T)
+    assert np.array_equal(got, want)

@@ -54,8 +54,9 @@ def e2m1_decode(codes) -> np.ndarray:
 def _nearest_even(y: np.ndarray, table: np.ndarray) -> np.ndarray:
     """Index into the ascending non-negative ``table`` of the value nearest to |y|, ties to
     the even index (the code whose lowest mantissa bit is 0); beyond the last entry the last
-    index (saturation).  Distances are exact in float64 for these short tables."""
-    a = np.abs(np.asarray(y, dtype=np.float64)).reshape(-1)
+    index (saturation: |y| is first clamped to the last entry, so that distances from a huge
+    |y| cannot round to a false tie).  Distances are exact in float64 for these short tables."""
+    a = np.minimum(np.abs(np.asarray(y, dtype=np.float64)).reshape(-1), table[-1])
     idx = np.empty(a.shape, dtype=np.int64)
     even_col = (np.arange(table.size) % 2 == 0)[None, :]
     for s in range(0, a.size, 1 << 18):

@@ -32,7 +32,7 @@ def test_e2m1_codes_decode_as_their_bit_fields():
 
 @pytest.mark.parametrize("y, want", [
     (0.0, 0.0), (0.2, 0.0), (0.25, 0.0), (0.26, 0.5), (0.75, 1.0), (1.25, 1.0), (1.75, 2.0),
-    (2.5, 2.0), (3.5, 4.0), (5.0, 4.0), (5.01, 6.0), (6.0, 6.0), (6.5, 6.0), (1e9, 6.0),
+    (2.5, 2.0), (3.5, 4.0), (5.0, 4.0), (5.01, 6.0), (6.0, 6.0), (6.5, 6.0), (1e9, 6.0), (1e30, 6.0),
     (-1.3, -1.5), (-0.75, -1.0), (-5.0, -4.0), (-7.0, -6.0),
 ])
 def test_e2m1_rounds_to_nearest_ties_to_even_and_saturates(y, want):
@@ -59,7 +59,7 @@ def test_e4m3_values_are_the_formats():
 
 def test_e4m3_rounding_matches_binade_rounding():
     x = np.concatenate([np.exp(RNG.uniform(np.log(1e-4), np.log(500.0), 20000)),
-                        [2.0 ** -10, 448.0, 464.0, 1e6, 0.0]]).astype(np.float32)
+                        [2.0 ** -10, 448.0, 464.0, 1e6, 1e30, 0.0]]).astype(np.float32)
     xd = x.astype(np.float64)
     e = np.floor(np.log2(np.maximum(xd, 2.0 ** -30)))
     step = 2.0 ** (np.maximum(e, -6) - 3)  # 3 mantissa bits; subnormal spacing below 2^-6

@@ -29,7 +29,7 @@ __host__ __device__ inline int item_nk(uint32_t it) { return int(it >> 21); }
 
 struct FrameLists {
   int32_t n_items;                               // prefill / store: valid query frames
-  uint32_t item[WAM_MAX_EPISODE_FRAMES];         // longest-first (descending nk)
+  uint32_t item[WAM_MAX_EPISODE_FRAMES];         // launch order (order_items_for_tc in api.cu)
   uint16_t vlist[WAM_MAX_EPISODE_FRAMES];        // valid frames of episode b at [b*F, ...)
   uint16_t nvalid[WAM_MAX_EPISODE_FRAMES];       // number of valid frames of episode b
 };

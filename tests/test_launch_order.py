@@ -102,3 +102,21 @@ def test_rejects_layouts_without_a_tensor_core_prefill():
     w, lay = layout_of("ctx19.2s_bf16")
     with pytest.raises(wam.WamError):
         wam.debug_prefill_order(lay, 3, 2, B200_SMS)
+
+
+def test_repeated_and_alternating_calls_give_the_same_orders():
+    # the library keeps its last answer for a repeated work list; alternating layouts and SM
+    # counts must still get each one's own order
+    cases = [("ctx19.2s_bf16", 0, B200_SMS), ("batched4_bf16", 0, B200_SMS),
+             ("ctx19.2s_bf16", 0, 16), ("ctx38.4s_bf16", 0, B200_SMS)]
+    first = {}
+    for name, f0, sms in cases:
+        w, lay = layout_of(name)
+        first[(name, sms)] = [a.tolist() for a in wam.debug_prefill_order(lay, f0, w.F_h, sms)]
+    for _ in range(2):
+        for name, f0, sms in cases + cases[::-1]:
+            w, lay = layout_of(name)
+            got = [a.tolist() for a in wam.debug_prefill_order(lay, f0, w.F_h, sms)]
+            assert got == first[(name, sms)]
+            again = [a.tolist() for a in wam.debug_prefill_order(lay, f0, w.F_h, sms)]
+            assert again == got

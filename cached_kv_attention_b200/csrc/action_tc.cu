@@ -18,6 +18,8 @@
 //                       each tile), warp 8 lane 0 issues TMA loads into a 4-stage ring and a
 //                       2-slot Q buffer.
 //   action_self_kernel  layers outside the interaction set (action keys only).
+#include <mutex>
+
 #include "launch.h"
 #include "tcgen05.cuh"
 
@@ -1092,8 +1094,11 @@ size_t action_tc_workspace_bytes(int BH, int max_parts) {
 // portable cluster size) while all B*H clusters still fit on the GPU at once.  The number of
 // co-resident clusters of each size is asked of the runtime once per device.
 static int umma_split(int BH, int dev) {
+  // Filled and read under one lock, so a second host thread never sees a half-filled table.
   static int max_clusters[32][um::kMaxSplit + 1];
   static bool known[32];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
   if (!known[dev]) {
     for (int k = 1; k <= um::kMaxSplit; ++k) {
       cudaLaunchConfig_t cfg = {};
@@ -1140,16 +1145,14 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
   } else {
     maps.fk = maps.ka, maps.fv = maps.va;
   }
-  static unsigned configured = 0;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 32) return cudaErrorInvalidDevice;
-  if (!(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(action_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, um::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured |= 1u << dev;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
+  // Set on every call (a host-side attribute write, no device work): nothing cached here can
+  // go stale across devices, threads or a device reset.
+  cudaError_t e = cudaFuncSetAttribute(action_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(action_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, um::kSmemBytes);
+  if (e != cudaSuccess) return e;
   if (umma) {
     ActionArgs ac = a;
     ac.ksplit = umma_split(a.B * a.H, dev);

@@ -2,6 +2,7 @@
 // per-launch work lists from the host padding mask and attention blocks, and dispatch to the
 // tensor-core or CUDA-core kernels.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -23,19 +24,15 @@ namespace {
 
 thread_local std::string g_last_error;
 
-// Address of the error word on the current device (looked up once per device).
+// Address of the error word on the current device, looked up on every call: an address kept
+// from an earlier call could belong to a context that a device reset has since replaced.
 int* device_error_word() {
-  static int* addr[64] = {};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_wam_device_error) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_wam_device_error) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return addr[dev];
+  return static_cast<int*>(p);
 }
 
 wam_status fail(wam_status st, const char* fmt, ...) {
@@ -138,17 +135,18 @@ void fill_items(const Geo& g, int f_begin, int f_end, wam::FrameLists& fl) {
   std::copy(items.begin(), items.end(), fl.item);
 }
 
-// SM count of the current device (looked up once per device).
+// SM count of the current device (looked up once per device; concurrent first calls may both
+// look it up and store the same value).
 int sm_count() {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (!cached[dev]) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 wam_status check_range(const Geo& g, int f_begin, int f_end) {

@@ -19,7 +19,6 @@ cudaError_t launch_action_simt(const ActionArgs& a, int D, bool bf16, cudaStream
 // Tensor-core paths (bf16, D = 128).  Return cudaErrorNotSupported when the shape has no
 // tensor-core kernel; the caller then takes the CUDA-core path.
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);   // tcgen05 + TMEM
-cudaError_t launch_prefill_mma(const PrefillArgs& a, cudaStream_t s);  // mma.sync tiles
 cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s);
 int action_tc_total_tiles(const ActionArgs& a);
 int action_tc_max_parts(const ActionArgs& a, int P, int G);

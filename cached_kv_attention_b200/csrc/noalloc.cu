@@ -8,7 +8,6 @@
 // entry point keeps the accumulator in a file-scope device array instead, so the caller passes
 // only its inputs and outputs.  It runs exactly the same kernels as wam_video_prefill_kv.
 #include <cstdio>
-#include <mutex>
 
 #include "launch.h"
 
@@ -19,30 +18,20 @@ static __device__ __align__(256) float g_noalloc_fuse_acc[2 * size_t(WAM_NOALLOC
 
 namespace {
 
-// Device address of the accumulator, looked up once per device with that device current.
+// Device address of the accumulator on the current device.  It is looked up on every call
+// (cudaGetSymbolAddress allocates nothing): an address kept from an earlier call could belong
+// to a context that a device reset has since replaced.
 float* noalloc_acc_address(wam_status* st) {
-  static float* addr[64] = {};
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= 64) {
-    *st = wam::record_error(WAM_ERR_CUDA, "wam_video_prefill_kv_fuse_noalloc: no current device");
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_fuse_acc);
+  if (e != cudaSuccess || !p) {
+    char msg[256];
+    snprintf(msg, sizeof(msg), "wam_video_prefill_kv_fuse_noalloc: cudaGetSymbolAddress: %s",
+             cudaGetErrorString(e));
+    *st = wam::record_error(WAM_ERR_CUDA, msg);
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_fuse_acc);
-    if (e != cudaSuccess || !p) {
-      char msg[256];
-      snprintf(msg, sizeof(msg), "wam_video_prefill_kv_fuse_noalloc: cudaGetSymbolAddress: %s",
-               cudaGetErrorString(e));
-      *st = wam::record_error(WAM_ERR_CUDA, msg);
-      return nullptr;
-    }
-    addr[dev] = static_cast<float*>(p);
-  }
-  return addr[dev];
+  return static_cast<float*>(p);
 }
 
 }  // namespace
@@ -54,10 +43,13 @@ extern "C" wam_status wam_video_prefill_kv_fuse_noalloc(
     void* fused_k, void* fused_v, wam_stream_t stream) {
   if (!layout)
     return wam::record_error(WAM_ERR_INVALID_ARGUMENT, "layout is NULL");
-  const long long need = (long long)layout->B * layout->F * layout->T * layout->H * layout->D;
   if (layout->B < 1 || layout->F < 1 || layout->T < 1 || layout->H < 1 || layout->D < 1)
     return wam::record_error(WAM_ERR_INVALID_ARGUMENT, "B, F, T, H and D must be >= 1");
-  if (need > (long long)WAM_NOALLOC_FUSE_ACC_ELEMS) {
+  // A one-layer interval (first and last) writes the fused pair directly and never touches
+  // the accumulator, so only calls that do are held to the array's size.
+  const bool uses_acc = !(first_in_interval && last_in_interval);
+  const long long need = (long long)layout->B * layout->F * layout->T * layout->H * layout->D;
+  if (uses_acc && need > (long long)WAM_NOALLOC_FUSE_ACC_ELEMS) {
     char msg[256];
     snprintf(msg, sizeof(msg),
              "wam_video_prefill_kv_fuse_noalloc: B*F*T*H*D = %lld exceeds the static accumulator "

@@ -597,14 +597,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   } else {
     maps.kc = maps.kn, maps.vc = maps.vn;
   }
-  static unsigned configured = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 32) return cudaErrorInvalidDevice;
-  if (!(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured |= 1u << dev;
-  }
+  // Set on every call (a host-side attribute write, no device work): nothing cached here can
+  // go stale across devices, threads or a device reset.
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int QP = (a.T / kBM + 1) / 2;
   const int64_t grid = int64_t(a.fl.n_items) * QP * a.H;
   return launch_pdl(prefill_tc_kernel, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);

@@ -214,8 +214,11 @@ wam_status wam_copy_frames(const wam_video_layout* layout, wam_dtype dt, int32_t
  *   - Limit: B * F * T * H * D <= WAM_NOALLOC_FUSE_ACC_ELEMS (about 4.2 million elements, for
  *     K and for V); larger layouts return WAM_ERR_UNSUPPORTED and launch nothing.  The array
  *     (2 x 16 MiB) is held on every GPU that loads the library until the process exits.
- *   - The first call on a device looks the array's address up (cudaGetSymbolAddress): make
- *     that first call before any stream capture.
+ *   - Every call looks the array's address up on the current device (cudaGetSymbolAddress,
+ *     which allocates nothing).  The first call on a device may also load the library's
+ *     device code there: make that first call before any stream capture.
+ *   - A one-layer interval (first_in_interval and last_in_interval) never touches the array
+ *     and is not held to the limit.
  *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - Every call shares the one array, which keeps what the last call left in it: a middle or
  *     last call of an interval reads what the previous call of that interval accumulated, and

@@ -44,7 +44,7 @@ METRIC = "action chunks/s at 19.2 s context (1 B200); % HBM / tensor-core roofli
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default="ctx19.2s_bf16", choices=sorted(synth.WORKLOADS))
@@ -52,11 +52,15 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="issue the chunk eagerly")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--profile-call", default=None, choices=["history", "future", "action"],
                     help="launch one stage call of the workload --repeat times and exit "
                          "(a small case for ncu captures; prints nothing)")
     ap.add_argument("--repeat", type=int, default=3)
+    ap.add_argument("--processes", type=int, default=2,
+                    help="at N = 1, repeat the timed steps in this many processes in all and report "
+                         "each one's median step time")
+    ap.add_argument("--child", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
 
 
@@ -87,8 +91,11 @@ def algorithmic_work(w: synth.Workload, pad: np.ndarray) -> dict:
     act_qkvo = w.n_act * H * D * (3 * 2 + 4) * w.B
     reads = w.M * w.n_euler_steps
     calls = w.L * w.n_euler_steps
-    action_bytes = valid_keys * H * D * 2 * 2 * reads + act_qkvo * calls
-    fused_read_bytes = valid_keys * H * D * 2 * 2  # one fused pair read
+    # bytes of one fused K or V row of one head: bf16, or NVFP4 (D / 2 bytes of E2M1 codes and
+    # D / 16 E4M3 block scales)
+    row = D * 2 if w.kv_format == "bf16" else D // 2 + D // 16
+    fused_read_bytes = valid_keys * H * row * 2  # one fused pair read (K and V)
+    action_bytes = fused_read_bytes * reads + act_qkvo * calls
     return {
         "imag_flops_per_launch": pair * fut_pairs,
         "prefill_flops": flops_hist + flops_fut,
@@ -274,6 +281,67 @@ def cpu_baseline(w: synth.Workload, pad: np.ndarray, seed: int) -> dict:
                       f"({sec:.1f} s of fp64 CPU work), extrapolated x{scale:.0f} to a whole chunk"}
 
 
+def parity_sample(w: synth.Workload, pad: np.ndarray) -> dict:
+    """Parity of this library against the oracle on a sample of the workload: the same chunk
+    (frames, padding, schedules, Euler steps) on 1 head and 4 layers (one fusion interval read
+    by layer 3), run through the chunk runner and through the oracle's chunk on the same seeded
+    inputs.  Per stage: the worst max|err| / max|ref| and the worst mean relative error
+    sum|err| / sum|ref| over the stage's output tensors."""
+    from cached_kv_attention_b200 import chunk as C
+    from oracle import wam_oracle as O
+    if w.slide:
+        return None
+    ws = w.replace(name=w.name + "_parity", H=1, L=4, seed=w.seed + 77)
+
+    def tree(x, fn):
+        return [tree(y, fn) for y in x] if isinstance(x, list) else fn(x)
+
+    to64 = lambda t: t.float().cpu().double().numpy()
+    inp_cpu = C.make_inputs(ws, "cpu")
+    inp = {k: tree(v, lambda t: t.cuda()) for k, v in inp_cpu.items()}
+    r = C.ChunkRunner(ws, inp, pad=pad, distinct_out=True).prepare()
+    r.run()
+    torch.cuda.synchronize()
+    inp64 = {k: tree(v, to64) for k, v in inp_cpu.items()}
+    inp64["fuse_weights"] = [O.fuse_weights(x) for x in inp64.pop("fuse_logits")]
+    kw = dict(L=ws.L, S=ws.S, T=ws.T, F_h=ws.F_h, F_f=ws.F_f, pad=pad)
+    if ws.joint:
+        ref = O.chunk_joint(inp64, n_steps=ws.n_euler_steps, **kw)
+    else:
+        ref = O.chunk(inp64, n_video_steps=ws.n_video_steps, n_euler_steps=ws.n_euler_steps,
+                      sigma_star=ws.sigma_star, **kw)
+    rows = lambda f0, f1: np.repeat(~pad[:, f0:f1].astype(bool), ws.T, axis=1)
+    out = {}
+
+    def add(stage, got, want, mask=None):
+        got, want = to64(got), np.asarray(want)
+        if mask is not None:
+            got, want = got[mask], want[mask]
+        err = np.abs(got - want)
+        mx = float(err.max() / max(np.abs(want).max(), 1e-300))
+        mean = float(err.sum() / max(np.abs(want).sum(), 1e-300))
+        o = out.setdefault(stage, {"max_rel": 0.0, "mean_rel": 0.0})
+        o["max_rel"], o["mean_rel"] = max(o["max_rel"], mx), max(o["mean_rel"], mean)
+
+    for l in range(ws.L):
+        add("history", r.hist_o[l], ref["hist_o"][l], rows(0, ws.F_h))
+        if not ws.joint:
+            add("final", r.final_o[l], ref["final_o"][l], rows(ws.F_h, ws.F))
+            for s_ in range(ws.n_video_steps):
+                add("imagination", r.imag_o[s_ * ws.L + l], ref["imag_o"][s_][l], rows(ws.F_h, ws.F))
+    reader = set(C.interaction_layers(ws.L, ws.S))
+    for i in range(ws.n_euler_steps):
+        for l in range(ws.L):
+            add("fused read" if l in reader else "self-only read", r.act_o[i * ws.L + l], ref["act_o"][i][l])
+    for m in range(ws.M):
+        add("fused pairs", r.fused_k[m], ref["fused_k"][m], rows(0, ws.F))
+        add("fused pairs", r.fused_v[m], ref["fused_v"][m], rows(0, ws.F))
+    add("x_act", r.x_act, ref["x_act"])
+    return {"sample": f"the chunk on 1/{w.H} heads and 4/{w.L} layers (one fusion interval)",
+            "bounds": {"bf16": {"max_rel": 1e-2, "mean_rel": 2e-3}, "f32": {"max_rel": 1e-5}},
+            "stages": out}
+
+
 # ------------------------------------------------------------------------------ reference arm
 
 def run_reference(args, world, rank):
@@ -393,18 +461,22 @@ def run_mine(args, world, rank, local):
         step()
     torch.cuda.synchronize()
     stage_ms = {k: [] for k in ev}
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    # one event between consecutive steps: the whole region for the mean, each step for the median
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for _ in range(args.steps):
+        marks[0].record(stream)
+        for i in range(args.steps):
             step()
-        t_end.record(stream)
+            marks[i + 1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = marks[0].elapsed_time(marks[-1])
+    step_times = [marks[i].elapsed_time(marks[i + 1]) / runner.chunks_per_run for i in range(args.steps)]
+    if args.child:
+        print(json.dumps({"median_ms": statistics.median(step_times)}), flush=True)
+        return
     # Stage events are re-recorded by every step: read the last timed step's stage times,
     # then time up to 10 more steps one by one for the stage averages.
     for k, (a, b) in ev.items():
@@ -424,7 +496,8 @@ def run_mine(args, world, rank, local):
                  "action": sum(v for k, v in st_ms.items() if k.startswith("action"))}
         video_ms = st_ms["history"] + fut_ms
     else:
-        video_ms = st_ms["history"] + st_ms["imagination"] + st_ms["final"] + st_ms.get("copy", 0.0)
+        video_ms = (st_ms["history"] + st_ms["imagination"] + st_ms["final"] + st_ms.get("copy", 0.0) +
+                    st_ms.get("quantize", 0.0))
     action_ms = st_ms["action"]
     fused_ms = time_fused_read(runner, stream)
 
@@ -463,18 +536,27 @@ def run_mine(args, world, rank, local):
     fused_gbs = fused_bytes / (fused_ms * 1e-3) / 1e9
     roofline_action = {"bound": "hbm", "achieved": fused_gbs, "peak": hbm_peak, "unit": "GB/s",
                        "frac": fused_gbs / hbm_peak,
-                       "kernel": "action_umma_kernel, one fused-cache read (wam_action_attn)",
+                       "kernel": ("action_nvfp4_kernel, one NVFP4 fused-cache read (wam_action_attn_nvfp4)"
+                                  if w.kv_format == "nvfp4" else
+                                  "action_split_kernel, one fused-cache read (wam_action_attn)"),
                        "peak_kind": f"{peak_src} copy bandwidth", "bytes_per_launch": fused_bytes,
                        "ms_per_launch": fused_ms,
                        "action_stage_gbs": work["action_bytes"] / (action_ms * 1e-3) / 1e9}
+
+    protocol = {"warmup": args.warmup, "samples": args.steps,
+                "median_ms_per_process": [statistics.median(step_times)],
+                "mean_ms": total_ms / args.steps / runner.chunks_per_run}
+    if rank == 0 and world == 1 and args.processes > 1:
+        protocol["median_ms_per_process"] += other_process_medians(args, args.processes - 1)
 
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(args, w, runner, inp, step, pad, world)
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, pad, seed=7)
+        parity = parity_sample(w, pad)
 
     if rank == 0:
         line = {
@@ -486,14 +568,16 @@ def run_mine(args, world, rank, local):
                        "F_h": w.F_h, "F_f": w.F_f, "pad_frames": int(pad.sum()),
                        "valid_keys": work["valid_keys"], "n_act": w.n_act,
                        "n_video_steps": w.n_video_steps, "n_euler_steps": w.n_euler_steps,
-                       "fusion_stride": w.S, "fusion": args.fusion,
+                       "fusion_stride": w.S, "fusion": args.fusion, "fused_cache": w.kv_format,
                        "launch": "cuda graph" if graph is not None else "eager",
                        "l2": "inputs larger than L2: ~25 GB of distinct per-layer buffers per chunk",
                        "parallelism": f"replicas x{world}"},
             "stage_ms": {**st_ms, "video": video_ms},
+            "protocol": protocol,
             "roofline": roofline,
             "roofline_action": roofline_action,
             "cpu_baseline": cpu,
+            "parity": parity,
             "e2e": e2e,
             "gpu_launches": launches * args.steps,
             "clocks": clocks.summary(),
@@ -501,6 +585,23 @@ def run_mine(args, world, rank, local):
         print(json.dumps(line), flush=True)
     if graph is not None:
         del graph
+
+
+def other_process_medians(args, n: int) -> list:
+    """Median step time (ms) of the same timed steps in n more processes, run one after another
+    (the pages time 5 warm-ups + 30 samples in two processes and report medians)."""
+    out = []
+    for _ in range(n):
+        cmd = [sys.executable, os.path.abspath(__file__), "--steps", str(args.steps), "--warmup",
+               str(args.warmup), "--workload", args.workload, "--fusion", args.fusion, "--child"]
+        if args.no_graph:
+            cmd.append("--no-graph")
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+        if r.returncode != 0 or not lines:
+            raise RuntimeError(f"bench child process failed (rc {r.returncode}): {r.stderr[-2000:]}")
+        out.append(json.loads(lines[-1])["median_ms"])
+    return out
 
 
 def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
@@ -561,28 +662,52 @@ def measure_e2e(args, w, runner, inp, step, pad, world) -> dict:
     h2d = sum(d.numel() * d.element_size() for d, _ in copies)
     out_host = torch.empty(runner.x_act.shape, dtype=torch.float32, pin_memory=True)
     d2h = out_host.numel() * 4
+    # Step i + 1's inputs cross PCIe on a copy stream into a staging set while step i's chunk
+    # runs; each step then moves its staged inputs into the chunk's buffers (device to device,
+    # on the compute stream) before replaying the chunk.
+    staged = [torch.empty_like(d) for d, _ in copies]
+    copy_stream = torch.cuda.Stream()
 
-    def one():
-        for d, h in copies:
-            d.copy_(h, non_blocking=True)
-        step()
-        out_host.copy_(runner.x_act, non_blocking=True)
+    def h2d_into_staging():
+        with torch.cuda.stream(copy_stream):
+            for (_, h), s_ in zip(copies, staged):
+                s_.copy_(h, non_blocking=True)
+        e = torch.cuda.Event()
+        e.record(copy_stream)
+        return e
 
-    one()
-    torch.cuda.synchronize()
+    def run(n_steps):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        copy_stream.wait_event(start)
+        ready = h2d_into_staging()
+        for i in range(n_steps):
+            stream.wait_event(ready)
+            for (d, _), s_ in zip(copies, staged):
+                d.copy_(s_, non_blocking=True)
+            free = torch.cuda.Event()
+            free.record(stream)
+            if i + 1 < n_steps:
+                copy_stream.wait_event(free)
+                ready = h2d_into_staging()
+            step()
+            out_host.copy_(runner.x_act, non_blocking=True)
+        end.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    run(1)
     barrier(world)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.e2e_steps):
-        one()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps / runner.chunks_per_run, world)
+    total = run(args.e2e_steps)
+    ms = max_over_ranks(total / args.e2e_steps / runner.chunks_per_run, world)
     cpr = runner.chunks_per_run
     return {"value": world * 1000.0 / ms, "unit": "chunks/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d // cpr, "d2h_bytes_per_step": d2h // cpr,
-            "note": "inputs in pinned host memory; non-padding frames of every Q/K/V tensor "
-                    "copied host->device each step, x_act read back"}
+            "note": "inputs in pinned host memory; the non-padding frames of every Q/K/V tensor, "
+                    "the velocities and initial noise copied host->device every step (timed), on "
+                    "a copy stream overlapping the previous step's chunk, then moved into the "
+                    "chunk's buffers; x_act read back every step"}
 
 
 def profile_call(args):

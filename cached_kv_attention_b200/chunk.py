@@ -20,7 +20,7 @@ capture the whole chunk.
 from __future__ import annotations
 
 import ctypes
-from typing import Dict, List, Optional
+from typing import Callable, Dict, List, Optional
 
 import numpy as np
 import torch
@@ -42,15 +42,18 @@ def interaction_layers(L: int, S: int) -> List[int]:
     return [I[-1] for I in interval_partition(L, S)]
 
 
-def make_inputs(w: Workload, device: str = "cpu") -> Dict:
-    """Seeded inputs of one chunk (see ``synth``); drawn on ``device``."""
+def make_inputs(w: Workload, device: str = "cpu", post: Optional[Callable] = None) -> Dict:
+    """Seeded inputs of one chunk (see ``synth``); drawn on ``device``.  ``post``, if given,
+    is applied to each Q/K/V tensor as soon as it is drawn and its result is stored instead
+    (for example a copy to the GPU, so a full-size chunk never holds every draw at once)."""
     dt = synth.torch_dtype(w)
     B, H, D, T = w.B, w.H, w.D, w.T
     hist, fut = w.F_h * T, w.F_f * T
+    keep = post if post is not None else (lambda t: t)
 
     def qkv(name, tokens, *idx):
-        return synth.normal((B, tokens, H, D), w.seed, name, *idx, std=w.qkv_std, dtype=dt,
-                            device=device)
+        return keep(synth.normal((B, tokens, H, D), w.seed, name, *idx, std=w.qkv_std, dtype=dt,
+                                 device=device))
 
     inp = {
         "hist_q": [qkv("hist_q", hist, l) for l in range(w.L)],
@@ -148,6 +151,11 @@ class ChunkRunner:
         self.fw = [wam.fuse_weights(lg.cpu().numpy()) for lg in inputs["fuse_logits"]]
         ws_bytes = wam.action_attn_workspace_size(self.layout, dt, w.n_act, True)
         self.workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        self.nvfp4 = None
+        if w.kv_format == "nvfp4":
+            if w.joint or w.slide or fusion != "epilogue" or w.dtype != "bf16":
+                raise ValueError("the NVFP4 fused cache is built for the bf16 IDM chunk with the fusion epilogue")
+            self.nvfp4 = wam.Nvfp4Cache(self.layout, 2 * w.M, device=dev.index)
         self.calls: List = []
         self._keep: List = []
 
@@ -184,14 +192,18 @@ class ChunkRunner:
         # and four small Euler steps), a5-a6 (final pass, standalone fusion), then the action
         # stages a7-a8
         self.stages = [("history", 0, hist_end), ("imagination", hist_end, imag_end),
-                       ("final", imag_end, video_end), ("action", video_end, len(calls))]
+                       ("final", imag_end, video_end)]
+        if self.action_start > video_end:
+            self.stages.append(("quantize", video_end, self.action_start))
+        self.stages.append(("action", self.action_start, len(calls)))
         self.fused_read_call = self._first_fused_read(calls, video_end)
         return self
 
     @staticmethod
     def _first_fused_read(calls, start):
         return next(i for i in range(start, len(calls))
-                    if calls[i][0] is wam.lib.wam_action_attn and calls[i][1][2] is not None)
+                    if calls[i][0] is wam.lib.wam_action_attn_nvfp4 or
+                    (calls[i][0] is wam.lib.wam_action_attn and calls[i][1][2] is not None))
 
     def _history_calls(self, calls, lay, dt, o_dt, s, o_of) -> int:
         """a3: history prefill with the cache store (+ fusion epilogue), all history frames."""
@@ -237,17 +249,36 @@ class ChunkRunner:
                               (lay, dt, len(I), kp, vp, wt, 0, F, _vp(self.fused_k[m]),
                                _vp(self.fused_v[m]), s)))
         video_end = len(calls)
+        # low-precision fused cache: every fused pair encoded once, after the final pass
+        q = self.nvfp4
+        if q is not None:
+            tensors = [t for m in range(w.M) for t in (self.fused_k[m], self.fused_v[m])]
+            arr = lambda ts: (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+            fp, cp, sp = arr(tensors), arr(q.codes), arr(q.scales)
+            self._keep += [fp, cp, sp]
+            calls.append((L.wam_fused_to_nvfp4, (lay, len(tensors), fp, cp, sp, _vp(q.s_g),
+                                                 _vp(q.workspace), q.workspace.numel(), s)))
+        self.action_start = len(calls)
         # a7 + a8: action denoising
         reader = {j: m for m, j in enumerate(interaction_layers(w.L, w.S))}
         na = self.x_act.numel()
         for i in range(w.n_euler_steps):
             for l in range(w.L):
                 m = reader.get(l)
+                qa_, ka_, va_ = (_vp(inp[k][i][l]) for k in ("act_q", "act_k", "act_v"))
+                if q is not None and m is not None:
+                    sg = q.s_g.data_ptr()
+                    calls.append((L.wam_action_attn_nvfp4,
+                                  (lay, _vp(q.codes[2 * m]), _vp(q.scales[2 * m]),
+                                   ctypes.c_void_p(sg + 8 * m), _vp(q.codes[2 * m + 1]),
+                                   _vp(q.scales[2 * m + 1]), ctypes.c_void_p(sg + 8 * m + 4), w.n_act,
+                                   qa_, ka_, va_, o_of(self.act_o, i * w.L + l), o_dt,
+                                   _vp(self.workspace), self.workspace.numel(), s)))
+                    continue
                 fk = _vp(self.fused_k[m]) if m is not None else None
                 fv = _vp(self.fused_v[m]) if m is not None else None
                 calls.append((L.wam_action_attn,
-                              (lay, dt, fk, fv, w.n_act, _vp(inp["act_q"][i][l]),
-                               _vp(inp["act_k"][i][l]), _vp(inp["act_v"][i][l]),
+                              (lay, dt, fk, fv, w.n_act, qa_, ka_, va_,
                                o_of(self.act_o, i * w.L + l), o_dt, _vp(self.workspace),
                                self.workspace.numel(), s)))
             ds = float(self.sig_a[i + 1] - self.sig_a[i])

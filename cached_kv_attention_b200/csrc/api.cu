@@ -552,6 +552,57 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const v
   return cuda_status(wam::launch_action_simt(a, g.D, dt == WAM_BF16, s), "wam_action_attn");
 }
 
+wam_status wam_action_attn_nvfp4(const wam_video_layout* layout, const void* k_codes,
+                                 const void* k_scales, const float* k_sg, const void* v_codes,
+                                 const void* v_scales, const float* v_sg, int32_t n_act,
+                                 const void* qa, const void* ka, const void* va, void* o,
+                                 wam_dtype o_dt, void* workspace, size_t ws_bytes,
+                                 wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  WAM_CHECK(check_dtype(o_dt, "o_dt"));
+  if (g.D != 128 || g.T % 128 != 0)
+    return fail(WAM_ERR_UNSUPPORTED, "wam_action_attn_nvfp4 needs D = 128 and T %% 128 == 0 (got D = %d, T = %d)",
+                g.D, g.T);
+  if (n_act < 1 || n_act > 32)
+    return fail(WAM_ERR_UNSUPPORTED, "wam_action_attn_nvfp4 needs 1 <= n_act <= 32 (got %d)", n_act);
+  WAM_NONNULL_ALIGNED(k_codes);
+  WAM_NONNULL_ALIGNED(k_scales);
+  WAM_NONNULL_ALIGNED(v_codes);
+  WAM_NONNULL_ALIGNED(v_scales);
+  if (!k_sg || !v_sg) return fail(WAM_ERR_INVALID_ARGUMENT, "k_sg or v_sg is NULL");
+  if ((reinterpret_cast<uintptr_t>(k_sg) & 3u) || (reinterpret_cast<uintptr_t>(v_sg) & 3u))
+    return fail(WAM_ERR_INVALID_ARGUMENT, "k_sg or v_sg is not 4-byte aligned");
+  WAM_NONNULL_ALIGNED(qa);
+  WAM_NONNULL_ALIGNED(ka);
+  WAM_NONNULL_ALIGNED(va);
+  WAM_NONNULL_ALIGNED(o);
+  static thread_local wam::ActionArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.qa = qa, a.ka = ka, a.va = va, a.o = o;
+  a.k_codes = static_cast<const uint8_t*>(k_codes), a.k_scales = static_cast<const uint8_t*>(k_scales);
+  a.v_codes = static_cast<const uint8_t*>(v_codes), a.v_scales = static_cast<const uint8_t*>(v_scales);
+  a.k_sg = k_sg, a.v_sg = v_sg;
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.n_act = n_act;
+  a.o_f32 = o_dt == WAM_F32;
+  a.with_video = 1;
+  a.scale_log2 = float(wam::kLog2e / std::sqrt(double(g.D)));
+  a.err = device_error_word();
+  fill_vlists(g, a.fl);
+  size_t need = 0;
+  WAM_CHECK(action_plan(a, &need));
+  if (need) {
+    if (!workspace || ws_bytes < need)
+      return fail(WAM_ERR_WORKSPACE, "wam_action_attn_nvfp4: workspace of %zu bytes needed (got %zu)", need,
+                  workspace ? ws_bytes : size_t(0));
+    if (!aligned16(workspace)) return fail(WAM_ERR_INVALID_ARGUMENT, "workspace is not 16-byte aligned");
+    a.ws_count = static_cast<int*>(workspace);
+    a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + wam::kTicketBytes);
+  }
+  return cuda_status(wam::launch_action_nvfp4(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_action_attn_nvfp4");
+}
+
 wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
                                 uint8_t* mask, wam_stream_t stream) {
   Geo g;
@@ -589,6 +640,63 @@ wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_beg
   }
   *n_items = a.fl.n_items;
   return WAM_OK;
+}
+
+wam_status wam_nvfp4_workspace_size(int32_t n, size_t* bytes) {
+  if (n < 1 || n > WAM_MAX_NVFP4_TENSORS)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n must be in [1, %d] (got %d)", WAM_MAX_NVFP4_TENSORS, n);
+  if (!bytes) return fail(WAM_ERR_INVALID_ARGUMENT, "bytes is NULL");
+  *bytes = size_t(n) * wam::kNvfp4MaxSlices * sizeof(float);
+  return ok();
+}
+
+wam_status wam_fused_to_nvfp4(const wam_video_layout* layout, int32_t n, const void* const* fused,
+                              void* const* codes, void* const* scales, float* s_g,
+                              void* workspace, size_t ws_bytes, wam_stream_t stream) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  if (n < 1 || n > WAM_MAX_NVFP4_TENSORS)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "n must be in [1, %d] (got %d)", WAM_MAX_NVFP4_TENSORS, n);
+  if (!fused || !codes || !scales) return fail(WAM_ERR_INVALID_ARGUMENT, "fused, codes or scales is NULL");
+  WAM_NONNULL_ALIGNED(s_g);
+  size_t need = 0;
+  WAM_CHECK(wam_nvfp4_workspace_size(n, &need));
+  if (!workspace || ws_bytes < need)
+    return fail(WAM_ERR_WORKSPACE, "wam_fused_to_nvfp4: workspace of %zu bytes needed (got %zu)", need,
+                workspace ? ws_bytes : size_t(0));
+  if (!aligned16(workspace)) return fail(WAM_ERR_INVALID_ARGUMENT, "workspace is not 16-byte aligned");
+  static thread_local wam::Nvfp4Args a;
+  std::memset(&a, 0, sizeof(a));
+  for (int j = 0; j < n; ++j) {
+    if (!fused[j] || !codes[j] || !scales[j])
+      return fail(WAM_ERR_INVALID_ARGUMENT, "fused[%d], codes[%d] or scales[%d] is NULL", j, j, j);
+    if (!aligned16(fused[j]) || !aligned16(codes[j]) || !aligned16(scales[j]))
+      return fail(WAM_ERR_INVALID_ARGUMENT, "fused[%d], codes[%d] or scales[%d] is not 16-byte aligned", j, j, j);
+    a.src[j] = fused[j], a.codes[j] = codes[j], a.scales[j] = scales[j];
+  }
+  a.s_g = s_g;
+  a.ws = static_cast<float*>(workspace);
+  a.n = n, a.B = g.B, a.H = g.H, a.D = g.D, a.T = g.T, a.F = g.F;
+  a.frame_elems = int64_t(g.T) * g.H * g.D;
+  std::vector<uint32_t> items;
+  for (int b = 0; b < g.B; ++b)
+    for (int f = 0; f < g.F; ++f)
+      if (!g.pad[size_t(b) * g.F + f]) items.push_back(wam::pack_item(b, f, 0));
+  a.fl.n_items = int32_t(items.size());
+  std::copy(items.begin(), items.end(), a.fl.item);
+  return cuda_status(wam::launch_nvfp4_encode(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_fused_to_nvfp4");
+}
+
+wam_status wam_debug_wait_timeout(int32_t polls, wam_stream_t stream) {
+  if (polls < 1 || uint32_t(polls) > wam::kWaitSpinLimit)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "polls must be in [1, %u] (got %d)",
+                unsigned(wam::kWaitSpinLimit), polls);
+  int* err = device_error_word();
+  if (!err) return fail(WAM_ERR_CUDA, "wam_debug_wait_timeout: no device error word");
+  return cuda_status(wam::launch_wait_timeout(uint32_t(polls), err,
+                                              reinterpret_cast<cudaStream_t>(stream)),
+                     "wam_debug_wait_timeout");
 }
 
 wam_status wam_device_error(int32_t clear) {

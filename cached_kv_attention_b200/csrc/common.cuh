@@ -74,7 +74,29 @@ struct ActionArgs {
   int32_t ksplit;     // CTAs (one thread-block cluster) per (episode, head) of the cluster read
   float scale_log2;
   int* err;
+  // NVFP4 fused pair (wam_action_attn_nvfp4; null otherwise): head-major codes [B, H, N, 64],
+  // E4M3 block scales [B, H, N, 8] and the device tensor scale of K and of V
+  const uint8_t* k_codes;
+  const uint8_t* k_scales;
+  const uint8_t* v_codes;
+  const uint8_t* v_scales;
+  const float* k_sg;
+  const float* v_sg;
   FrameLists fl;
+};
+
+// NVFP4 encoding of n fused tensors (nvfp4.cu).  ws holds kNvfp4MaxSlices |x| maxima per
+// tensor between the two launches.
+constexpr int kNvfp4MaxSlices = 1024;
+struct Nvfp4Args {
+  const void* src[WAM_MAX_NVFP4_TENSORS];  // bf16 [B, N, H, D]
+  void* codes[WAM_MAX_NVFP4_TENSORS];      // [B, H, N, D / 2]
+  void* scales[WAM_MAX_NVFP4_TENSORS];     // [B, H, N, D / 16]
+  float* s_g;                              // [n]
+  float* ws;                               // [n][kNvfp4MaxSlices]
+  int32_t n, B, H, D, T, F, slices;
+  int64_t frame_elems;                     // T * H * D
+  FrameLists fl;                           // items: the valid (b, f) frames
 };
 
 struct CopyArgs {
@@ -166,12 +188,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: returns false if the phase never flips; the caller then records
-// WAM_ERR_TIMEOUT in the device error word (args.err) and leaves without waiting further.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitSpinLimit; ++i)
+// Bounded wait: returns false if the phase never flips within `limit` polls; the caller then
+// records WAM_ERR_TIMEOUT in the device error word (args.err) and leaves without waiting
+// further.  The kernels use kWaitSpinLimit; wam_debug_wait_timeout passes a short limit.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_bounded(bar, parity, kWaitSpinLimit);
 }
 
 // 4-D tiled TMA load global -> shared, completion counted on an mbarrier (no multicast).

@@ -15,11 +15,14 @@ cudaError_t launch_copy_frames(const CopyArgs& a, cudaStream_t s);
 cudaError_t launch_debug_mask(const PrefillArgs& a, uint8_t* mask, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_action_simt(const ActionArgs& a, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_wait_timeout(uint32_t polls, int* err, cudaStream_t s);
+cudaError_t launch_nvfp4_encode(Nvfp4Args& a, cudaStream_t s);
 
 // Tensor-core paths (bf16, D = 128).  Return cudaErrorNotSupported when the shape has no
 // tensor-core kernel; the caller then takes the CUDA-core path.
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);   // tcgen05 + TMEM
 cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s);
+cudaError_t launch_action_nvfp4(const ActionArgs& a, cudaStream_t s);  // T % 128 == 0, bf16 action inputs
 int action_tc_total_tiles(const ActionArgs& a);
 int action_tc_max_parts(const ActionArgs& a, int P, int G);
 size_t action_tc_workspace_bytes(int BH, int max_parts);

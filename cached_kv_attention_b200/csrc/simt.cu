@@ -35,6 +35,28 @@ static int grid_for(int64_t work, int per_block, int cap) {
   return g < 1 ? 1 : int(g);
 }
 
+// ------------------------------------------------------------------------------ bounded wait
+// A wait that runs out, on purpose: one warp waits on an mbarrier that nothing arrives on,
+// with a short poll limit, and reports WAM_ERR_TIMEOUT through the device error word as the
+// attention kernels do when one of their waits gives up.  It holds no TMA, tensor-core or
+// tensor-memory work, so giving up leaves nothing in flight.
+__global__ void wait_timeout_kernel(uint32_t polls, int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool done = mbar_wait_bounded(&bar, 0, polls);  // phase 0 never completes
+  if (!__any_sync(0xffffffffu, done) && threadIdx.x == 0 && err)
+    atomicExch(err, int(WAM_ERR_TIMEOUT));
+}
+
+cudaError_t launch_wait_timeout(uint32_t polls, int* err, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(polls, err);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------------------ Euler
 __global__ void euler_kernel(int64_t n, float* __restrict__ x, const float* __restrict__ v,
                              float dsigma) {

@@ -50,6 +50,8 @@ class Workload:
     seed: int
     joint: bool = False  # co-denoising: the future frames are re-passed at every action step
     slide: bool = False  # history window kept across chunks: only the newest frame is passed
+    kv_format: str = "bf16"  # fused pairs read by the action layers: "bf16", or "nvfp4" (encoded
+                             # from the bf16 pairs once the final pass has completed them)
 
     @property
     def F(self) -> int:
@@ -86,9 +88,10 @@ WORKLOADS = {
                               **_BF),
 }
 # Interaction-stride variants of the 19.2 s chunk ("世界模型之Faster-WAM详解" §4.3 ablates strides
-# 1, 2, 4, 7, 14): every layer reads its own K/V (S = 1: one-layer intervals), S = 2, S = 7; and
-# the one-shot variant (§3.1: one video pass at sigma* = 1, no imagination step).
-for _s in (1, 2, 7):
+# 1, 2, 4, 7, 14): every layer reads its own K/V (S = 1: one-layer intervals), S = 2, S = 7,
+# S = 14 (intervals {0-13}, {14-27}, {28, 29}); and the one-shot variant (§3.1: one video pass
+# at sigma* = 1, no imagination step).
+for _s in (1, 2, 7, 14):
     WORKLOADS[f"stride{_s}_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
         name=f"stride{_s}_ctx19.2s_bf16", S=_s)
 WORKLOADS["oneshot_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
@@ -102,6 +105,11 @@ WORKLOADS["cod4_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
 # new frame in, the oldest of the 5 valid frames out).
 WORKLOADS["slide_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
     name="slide_ctx19.2s_bf16", slide=True)
+# The 19.2 s chunk with a low-precision fused cache ("Long-WAM: 机器人操作模型的长历史..." §四: the
+# LongLive-2.0 KV cache is NVFP4): the 8 fused pairs are encoded after the final pass and every
+# interaction read decodes them.
+WORKLOADS["nvfp4_ctx19.2s_bf16"] = WORKLOADS["ctx19.2s_bf16"].replace(
+    name="nvfp4_ctx19.2s_bf16", kv_format="nvfp4")
 
 
 def seed_for(seed: int, name: str, *idx: int) -> int:

@@ -17,7 +17,8 @@ __all__ = [
     "video_prefill_kv", "fuse_interval_kv", "action_attn", "flow_euler_step",
     "flow_schedule", "fuse_weights", "debug_video_mask", "device_error", "exported_names",
     "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS", "action_attn_workspace_size",
-    "action_workspace", "debug_prefill_order",
+    "action_workspace", "debug_prefill_order", "debug_wait_timeout",
+    "nvfp4_workspace_size", "fused_to_nvfp4", "Nvfp4Cache", "action_attn_nvfp4",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
@@ -68,6 +69,12 @@ def _load() -> ctypes.CDLL:
         "wam_debug_prefill_order": [lay, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
                                     ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "wam_device_error": [i32],
+        "wam_debug_wait_timeout": [i32, vp],
+        "wam_nvfp4_workspace_size": [i32, ctypes.POINTER(ctypes.c_size_t)],
+        "wam_fused_to_nvfp4": [lay, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                               vp, vp, ctypes.c_size_t, vp],
+        "wam_action_attn_nvfp4": [lay, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, i32, vp,
+                                  ctypes.c_size_t, vp],
         "wam_video_prefill_kv_fuse_noalloc": [lay, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp,
                                               i32, f32, i32, i32, vp, vp, vp],
     }
@@ -91,7 +98,8 @@ def exported_names() -> list:
             "wam_flow_euler_step", "wam_flow_schedule", "wam_fuse_weights",
             "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
             "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size",
-            "wam_copy_frames", "wam_debug_prefill_order"]
+            "wam_copy_frames", "wam_debug_prefill_order", "wam_debug_wait_timeout",
+            "wam_nvfp4_workspace_size", "wam_fused_to_nvfp4", "wam_action_attn_nvfp4"]
 
 
 def check(status: int) -> None:
@@ -275,6 +283,58 @@ def debug_prefill_order(layout: VideoLayout, f_begin: int, f_end: int, n_sms: in
     check(lib.wam_debug_prefill_order(layout.ref, f_begin, f_end, n_sms, ep.ctypes.data_as(P),
                                       fr.ctypes.data_as(P), nk.ctypes.data_as(P), ctypes.byref(n)))
     return ep[:n.value], fr[:n.value], nk[:n.value]
+
+
+def nvfp4_workspace_size(n: int) -> int:
+    out = ctypes.c_size_t(0)
+    check(lib.wam_nvfp4_workspace_size(int(n), ctypes.byref(out)))
+    return out.value
+
+
+class Nvfp4Cache:
+    """Device buffers of NVFP4-encoded fused tensors of one layout: per tensor the codes
+    [B, H, N, D / 2] and E4M3 block scales [B, H, N, D / 16] (uint8, head-major), and one fp32
+    tensor scale each in ``s_g`` [n]."""
+
+    def __init__(self, layout: VideoLayout, n: int, device=None):
+        B, H, N, D = layout.B, layout.H, layout.N, layout.D
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+        self.codes = [torch.zeros((B, H, N, D // 2), dtype=torch.uint8, device=dev) for _ in range(n)]
+        self.scales = [torch.zeros((B, H, N, D // 16), dtype=torch.uint8, device=dev) for _ in range(n)]
+        self.s_g = torch.zeros(n, dtype=torch.float32, device=dev)
+        self.workspace = torch.zeros(nvfp4_workspace_size(n), dtype=torch.uint8, device=dev)
+
+
+def fused_to_nvfp4(layout: VideoLayout, fused, cache: Nvfp4Cache, stream=None) -> None:
+    """NVFP4-encode the bf16 fused tensors ``fused`` (a list) into ``cache``."""
+    n = len(fused)
+    fp = (ctypes.c_void_p * n)(*[_ptr(t) for t in fused])
+    cp = (ctypes.c_void_p * n)(*[_ptr(t) for t in cache.codes[:n]])
+    sp = (ctypes.c_void_p * n)(*[_ptr(t) for t in cache.scales[:n]])
+    check(lib.wam_fused_to_nvfp4(layout.ref, n, fp, cp, sp, _ptr(cache.s_g), _ptr(cache.workspace),
+                                 cache.workspace.numel(), _stream(stream)))
+
+
+def action_attn_nvfp4(layout: VideoLayout, cache: Nvfp4Cache, k_index: int, v_index: int, qa, ka,
+                      va, o, workspace=None, stream=None) -> None:
+    """The action read over the NVFP4 fused pair held in ``cache`` at tensors k_index / v_index."""
+    n_act = qa.shape[1]
+    if workspace is None:
+        need = action_attn_workspace_size(layout, torch.bfloat16, n_act, True)
+        workspace = action_workspace(need, qa.device.index)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    sg = cache.s_g.data_ptr()
+    check(lib.wam_action_attn_nvfp4(layout.ref, _ptr(cache.codes[k_index]), _ptr(cache.scales[k_index]),
+                                    sg + 4 * k_index, _ptr(cache.codes[v_index]),
+                                    _ptr(cache.scales[v_index]), sg + 4 * v_index, n_act, _ptr(qa),
+                                    _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _ptr(workspace), ws_bytes,
+                                    _stream(stream)))
+
+
+def debug_wait_timeout(polls: int = 10000, stream=None) -> None:
+    """Launch a wait that gives up after ``polls`` polls and records WAM_ERR_TIMEOUT in the
+    device error word (read it with ``device_error``)."""
+    check(lib.wam_debug_wait_timeout(int(polls), _stream(stream)))
 
 
 def device_error(clear: bool = True) -> None:

@@ -47,6 +47,7 @@ typedef struct CUstream_st* wam_stream_t; /* the same handle as cudaStream_t */
 #define WAM_MAX_EPISODE_FRAMES 1024
 #define WAM_MAX_FUSE_LAYERS 16
 #define WAM_MAX_COPY_TENSORS 128
+#define WAM_MAX_NVFP4_TENSORS 64
 
 typedef enum {
   WAM_OK = 0,
@@ -235,6 +236,49 @@ wam_status wam_video_prefill_kv_fuse_noalloc(const wam_video_layout* layout, wam
                                              int32_t last_in_interval,
                                              void* fused_k, void* fused_v, wam_stream_t stream);
 
+/*
+ * Low-precision fused cache: NVFP4 encoding of fused K or V tensors ("Long-WAM: 机器人操作模型
+ * 的长历史..." §四: the LongLive-2.0 stack keeps its KV cache block-wise in NVFP4, about 3.6x
+ * smaller; "Long-WAM ... | Summary" §4.2: Long-WAM itself keeps BF16).  The pages name the
+ * format, not its parameters; this library takes NVIDIA's public NVFP4:
+ *   elements E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one E4M3 scale per 16 consecutive
+ *   elements along D, one fp32 scale per tensor s_g = amax / (6 * 448) over the tensor's
+ *   non-padding frames; x ~ e2m1 * e4m3 * s_g.  Codes are chosen in fp32 (IEEE division and
+ *   products), rounded to nearest even and saturated; zero takes the +0 code.
+ *   fused   host array of n device pointers, bf16 [B, N, H, D] (the stored fused pairs)
+ *   codes   host array of n device pointers, uint8 [B, H, N, D / 2]: head-major (one 128-key
+ *           tile of one head is one contiguous run), element 2i in the low nibble of byte i
+ *   scales  host array of n device pointers, uint8 [B, H, N, D / 16]: E4M3 codes
+ *   s_g     device float [n]: each tensor's scale
+ *   workspace device scratch of wam_nvfp4_workspace_size(n) bytes, 16-byte aligned
+ * Rows of padding frames are not read and their codes and scales are not written.  Two kernels
+ * on `stream`; 1 <= n <= WAM_MAX_NVFP4_TENSORS; D % 16 == 0 (D in {64, 128}); bf16 only.
+ */
+wam_status wam_nvfp4_workspace_size(int32_t n, size_t* bytes);
+wam_status wam_fused_to_nvfp4(const wam_video_layout* layout, int32_t n, const void* const* fused,
+                              void* const* codes, void* const* scales, float* s_g,
+                              void* workspace, size_t ws_bytes, wam_stream_t stream);
+
+/*
+ * The asymmetric action read of wam_action_attn over an NVFP4 fused pair (as wam_fused_to_nvfp4
+ * writes it): O = softmax(Q_a [K_video; K_a]^T / sqrt(D)) [V_video; V_a] with the video keys and
+ * values taken as their decoded values e2m1 * e4m3 * s_g.
+ *   k_codes, k_scales, v_codes, v_scales  device [B, H, N, 64] and [B, H, N, 8] (D = 128)
+ *   k_sg, v_sg   device float: the tensors' scales (4-byte aligned)
+ *   qa, ka, va   device bf16 [B, n_act, H, 128], 1 <= n_act <= 32; o device [B, n_act, H, 128]
+ *                (o_dt WAM_F32 or WAM_BF16)
+ *   workspace    as for wam_action_attn (wam_action_attn_workspace_size with dt = WAM_BF16)
+ * T % 128 == 0.  The tiles are decoded exactly into fp16 and the matrix products run on fp16
+ * operands with fp32 accumulation (the action Q/K/V are rounded to fp16 once: they must lie
+ * within fp16's range, |x| < 65504); P is carried as two fp16 terms.
+ */
+wam_status wam_action_attn_nvfp4(const wam_video_layout* layout, const void* k_codes,
+                                 const void* k_scales, const float* k_sg, const void* v_codes,
+                                 const void* v_scales, const float* v_sg, int32_t n_act,
+                                 const void* qa, const void* ka, const void* va, void* o,
+                                 wam_dtype o_dt, void* workspace, size_t ws_bytes,
+                                 wam_stream_t stream);
+
 /* ---- host helpers (no GPU work) ---------------------------------------------------------- */
 
 /*
@@ -272,6 +316,16 @@ wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin,
 wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
                                    int32_t n_sms, int32_t* episode, int32_t* frame,
                                    int32_t* n_key_frames, int32_t* n_items);
+
+/*
+ * Failure-detection check: launches one warp that waits on a shared-memory mbarrier nothing
+ * arrives on, giving up after `polls` polls (1 <= polls <= 2^24, the attention kernels'
+ * own limit), and then records WAM_ERR_TIMEOUT in the device error word exactly as an
+ * attention kernel does when one of its bounded waits gives up.  The kernel holds no TMA,
+ * tensor-core or tensor-memory work and returns normally; wam_device_error() then reports
+ * the timeout, and the device stays usable.  Asynchronous on `stream`.
+ */
+wam_status wam_debug_wait_timeout(int32_t polls, wam_stream_t stream);
 
 /*
  * Synchronise the current device and report its error word: WAM_OK, or WAM_ERR_TIMEOUT when

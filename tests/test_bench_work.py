@@ -43,7 +43,9 @@ def test_action_bytes_are_the_masks_valid_keys(name):
     t = 2
     video_keys = int(O.action_key_allowed(pad, t, w.n_act)[:, : w.F * t].sum()) * (w.T // t)
     assert work["valid_keys"] == video_keys
-    assert work["fused_read_bytes"] == video_keys * w.H * w.D * 2 * 2
+    # one head's K or V row: bf16, or NVFP4's 4-bit codes plus one 8-bit scale per 16 elements
+    row = w.D * 2 if w.kv_format == "bf16" else w.D * 4 // 8 + w.D // 16 * 1
+    assert work["fused_read_bytes"] == video_keys * w.H * row * 2
     reads = len(O.interaction_layers(w.L, w.S)) * w.n_euler_steps
     assert work["action_reads"] == reads
     qkvo = w.B * w.n_act * w.H * w.D * (3 * 2 + 4)  # bf16 Q, K, V in; fp32 O out

@@ -70,8 +70,9 @@ def test_tiny_fp32_chunk_end_to_end(fusion):
     _compare_chunk(w, r, ref, pad, None, "f32")
 
 
-@pytest.mark.parametrize("variant", [dict(S=1), dict(S=3), dict(n_video_steps=0, sigma_star=1.0)],
-                         ids=["stride1", "stride3", "one_shot"])
+@pytest.mark.parametrize("variant", [dict(S=1), dict(S=3), dict(L=16, S=14),
+                                     dict(n_video_steps=0, sigma_star=1.0)],
+                         ids=["stride1", "stride3", "stride14_L16", "one_shot"])
 def test_tiny_fp32_chunk_variants(variant):
     # The interaction-stride and one-shot variants run the same calls with other S / video steps.
     w = synth.WORKLOADS["tiny_f32"].replace(seed=8, **variant)
@@ -255,3 +256,63 @@ def test_sliding_window_chunks(name, dtype):
         for i in range(w.n_euler_steps):
             assert_parity(to64(r.act_o[i * w.L + l])[:, :, hs], second["act_o"][i][l][:, :, hs], dtype,
                           f"slide action {i},{l}")
+
+
+# ----------------------------------------------------------------------------- bench config
+
+@pytest.mark.slow
+def test_bench_config_chunk_end_to_end_sampled_heads():
+    """The whole ctx19.2s_bf16 chunk the benchmark times: 30 layers, history prefill with the
+    fusion epilogue, 4 imagination passes, the final cache pass folding 8 intervals (the last
+    one {28, 29}), 80 fused reads of 5376 keys and 220 self-only reads, both Euler chains.
+    Every stage output, cache and fused pair is compared with the oracle's chunk on two heads
+    (attention and fusion are independent per head, so the oracle runs on those heads alone);
+    the Euler states depend on no head and are compared whole."""
+    w = synth.WORKLOADS["ctx19.2s_bf16"]
+    heads = [4, 19]
+    pad = synth.pad_mask(w).numpy()
+
+    def both(t):  # the device copy, and the sampled heads widened for the oracle
+        return t.cuda(), to64(t[:, :, heads])
+
+    pairs = C.make_inputs(w, "cpu", post=both)
+    inp = {k: _tree(v, lambda p: p[0] if isinstance(p, tuple) else p.cuda()) for k, v in pairs.items()}
+    inp64 = {k: _tree(v, lambda p: p[1] if isinstance(p, tuple) else to64(p)) for k, v in pairs.items()}
+    del pairs
+    inp64["fuse_weights"] = [O.fuse_weights(lg) for lg in inp64.pop("fuse_logits")]
+    r = C.ChunkRunner(w, inp, distinct_out=True).prepare()
+    r.run()
+    wam.device_error()
+    ref = _oracle_chunk(w, inp64, pad)
+
+    T, F_h, F = w.T, w.F_h, w.F
+    rows_h, rows_f, rows = valid_rows(pad, T, 0, F_h), valid_rows(pad, T, F_h, F), valid_rows(pad, T, 0, F)
+    worst = {}
+
+    def check(got, want, what, stage):
+        e = assert_parity(got, want, "bf16", what)
+        d = np.abs(np.asarray(got) - want)
+        mean_rel = float(d.sum() / np.abs(want).sum())
+        m = worst.setdefault(stage, [0.0, 0.0])
+        m[0], m[1] = max(m[0], e), max(m[1], mean_rel)
+
+    g = lambda t: to64(t)[:, :, heads]
+    for l in range(w.L):
+        check(g(r.hist_o[l])[rows_h], ref["hist_o"][l][rows_h], f"hist {l}", "history")
+        check(g(r.final_o[l])[rows_f], ref["final_o"][l][rows_f], f"final {l}", "final")
+        for s in range(w.n_video_steps):
+            check(g(r.imag_o[s * w.L + l])[rows_f], ref["imag_o"][s][l][rows_f], f"imag {s},{l}", "imagination")
+        np.testing.assert_array_equal(g(r.k_cache[l])[rows], ref["k_cache"][l][rows])
+        np.testing.assert_array_equal(g(r.v_cache[l])[rows], ref["v_cache"][l][rows])
+    for m in range(w.M):
+        check(g(r.fused_k[m])[rows], ref["fused_k"][m][rows], f"fused K {m}", "fused pairs")
+        check(g(r.fused_v[m])[rows], ref["fused_v"][m][rows], f"fused V {m}", "fused pairs")
+    reader = set(C.interaction_layers(w.L, w.S))
+    for i in range(w.n_euler_steps):
+        for l in range(w.L):
+            check(g(r.act_o[i * w.L + l]), ref["act_o"][i][l], f"action {i},{l}",
+                  "fused read" if l in reader else "self-only read")
+    assert_parity(to64(r.x_future), ref["x_future"], "f32", "x_future")
+    assert_parity(to64(r.x_act), ref["x_act"], "f32", "x_act")
+    for stage, (mx, mean) in worst.items():  # margins against the bf16 bounds (1e-2, 2e-3)
+        print(f"bench-config parity {stage}: worst max|err|/max|ref| {mx:.2e}, worst mean rel {mean:.2e}")

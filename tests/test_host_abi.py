@@ -21,7 +21,7 @@ FAKE = 0x7F0000000000  # 16-byte aligned stand-in address; never dereferenced by
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "wam.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(wam_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(wam_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_function():

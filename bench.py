@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--profile-call", default=None, choices=["history", "future", "action"],
+    ap.add_argument("--profile-call", default=None, choices=["history", "future", "action", "action_nvfp4"],
                     help="launch one stage call of the workload --repeat times and exit "
                          "(a small case for ncu captures; prints nothing)")
     ap.add_argument("--repeat", type=int, default=3)
@@ -387,24 +387,29 @@ IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 80.3e6}
 
 
 def time_fused_read(runner, stream, n=20) -> float:
-    """Mean device time (ms) of one fused-cache action read of the prepared chunk.  The call is
-    captured once in a CUDA graph; each sample replays it right after a 256 MB write that
-    flushes the L2 and a 256 MB read of another buffer, which evicts the write's dirty lines
-    (otherwise the timed read also pays for writing them back) and keeps the GPU busy while
-    the replay is submitted, with CUDA events around the replay alone."""
-    fn, args = runner.calls[runner.fused_read_call]
+    """Mean device time (ms) of one fused-cache action read: the chunk's own interaction reads of
+    its first Euler step (one per fused pair, M launches, 8 x 66 MB at 19.2 s: larger than L2),
+    captured back to back in one CUDA graph and replayed after a 256 MB write that flushes the L2
+    and a 256 MB read of another buffer (so no dirty line is left to write back), with CUDA events
+    around the replay; the time divided by the number of reads."""
+    calls = runner.calls
+    first = runner.fused_read_call
+    reads = [i for i in range(first, len(calls))
+             if calls[i][0] is calls[first][0] and calls[i][1][2] is not None][:runner.w.M]
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
     clean = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
     total = torch.zeros((), dtype=torch.float32, device="cuda")
-    st = fn(*args)  # the call once outside capture (one-time per-device set-up)
-    if st:
-        raise RuntimeError(f"fused read call failed: {st}")
+    for i in reads:  # once outside capture (one-time per-device set-up)
+        fn, args = calls[i]
+        if fn(*args):
+            raise RuntimeError("fused read call failed")
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
-        st = fn(*args)
-    if st:
-        raise RuntimeError(f"fused read call failed: {st}")
+        for i in reads:
+            fn, args = calls[i]
+            if fn(*args):
+                raise RuntimeError("fused read call failed")
     ts = []
     for i in range(n + 3):
         flush.fill_(float(i))
@@ -416,7 +421,7 @@ def time_fused_read(runner, stream, n=20) -> float:
         b.record(stream)
         torch.cuda.synchronize()
         if i >= 3:
-            ts.append(a.elapsed_time(b))
+            ts.append(a.elapsed_time(b) / len(reads))
     del g, flush, clean, total
     return statistics.mean(ts)
 
@@ -538,9 +543,11 @@ def run_mine(args, world, rank, local):
                        "frac": fused_gbs / hbm_peak,
                        "kernel": ("action_nvfp4_kernel, one NVFP4 fused-cache read (wam_action_attn_nvfp4)"
                                   if w.kv_format == "nvfp4" else
-                                  "action_split_kernel, one fused-cache read (wam_action_attn)"),
+                                  "action_umma_kernel, one fused-cache read (wam_action_attn)"),
                        "peak_kind": f"{peak_src} copy bandwidth", "bytes_per_launch": fused_bytes,
                        "ms_per_launch": fused_ms,
+                       "method": "one Euler step's interaction reads (one per fused pair) back to back "
+                                 "in a CUDA graph after an L2 flush, time / reads",
                        "action_stage_gbs": work["action_bytes"] / (action_ms * 1e-3) / 1e9}
 
     protocol = {"warmup": args.warmup, "samples": args.steps,
@@ -734,10 +741,16 @@ def profile_call(args):
         q, k, v = g("q", w.F_f * w.T), g("k", w.F_f * w.T), g("v", w.F_f * w.T)
         o = torch.empty((w.B, w.F_f * w.T, w.H, w.D), device="cuda")
         call = lambda: wam.video_prefill_kv(lay, w.F_h, w.F, q, k, v, kc, vc, o, False)
-    else:
+    elif args.profile_call == "action":
         qa, ka, va = g("qa", w.n_act), g("ka", w.n_act), g("va", w.n_act)
         o = torch.empty((w.B, w.n_act, w.H, w.D), device="cuda")
         call = lambda: wam.action_attn(lay, kc, vc, qa, ka, va, o)
+    else:  # the NVFP4 read over the cache encoded once
+        qa, ka, va = g("qa", w.n_act), g("ka", w.n_act), g("va", w.n_act)
+        o = torch.empty((w.B, w.n_act, w.H, w.D), device="cuda")
+        cache = wam.Nvfp4Cache(lay, 2)
+        wam.fused_to_nvfp4(lay, [kc, vc], cache)
+        call = lambda: wam.action_attn_nvfp4(lay, cache, 0, 1, qa, ka, va, o)
     for _ in range(args.repeat):
         call()
     torch.cuda.synchronize()

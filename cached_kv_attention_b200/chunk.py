@@ -203,7 +203,7 @@ class ChunkRunner:
     def _first_fused_read(calls, start):
         return next(i for i in range(start, len(calls))
                     if calls[i][0] is wam.lib.wam_action_attn_nvfp4 or
-                    (calls[i][0] is wam.lib.wam_action_attn and calls[i][1][2] is not None))
+                    (calls[i][0] is wam.lib.wam_action_attn_ex and calls[i][1][2] is not None))
 
     def _history_calls(self, calls, lay, dt, o_dt, s, o_of) -> int:
         """a3: history prefill with the cache store (+ fusion epilogue), all history frames."""
@@ -273,14 +273,16 @@ class ChunkRunner:
                                    ctypes.c_void_p(sg + 8 * m), _vp(q.codes[2 * m + 1]),
                                    _vp(q.scales[2 * m + 1]), ctypes.c_void_p(sg + 8 * m + 4), w.n_act,
                                    qa_, ka_, va_, o_of(self.act_o, i * w.L + l), o_dt,
-                                   _vp(self.workspace), self.workspace.numel(), s)))
+                                   _vp(self.workspace), self.workspace.numel(),
+                                   wam.ACTION_FUSED_READY, s)))
                     continue
                 fk = _vp(self.fused_k[m]) if m is not None else None
                 fv = _vp(self.fused_v[m]) if m is not None else None
-                calls.append((L.wam_action_attn,
+                # the fused pairs are read-only in the action loop (completed by the video stage)
+                calls.append((L.wam_action_attn_ex,
                               (lay, dt, fk, fv, w.n_act, qa_, ka_, va_,
                                o_of(self.act_o, i * w.L + l), o_dt, _vp(self.workspace),
-                               self.workspace.numel(), s)))
+                               self.workspace.numel(), wam.ACTION_FUSED_READY, s)))
             ds = float(self.sig_a[i + 1] - self.sig_a[i])
             calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
         return imag_end, video_end
@@ -353,18 +355,19 @@ class ChunkRunner:
                 m = reader.get(l)
                 fk = _vp(self.fused_k[m]) if m is not None else None
                 fv = _vp(self.fused_v[m]) if m is not None else None
-                calls.append((L.wam_action_attn,
+                # the fused pairs were written by this step's video passes, several calls earlier
+                calls.append((L.wam_action_attn_ex,
                               (lay, dt, fk, fv, w.n_act, _vp(inp["act_q"][i][l]),
                                _vp(inp["act_k"][i][l]), _vp(inp["act_v"][i][l]),
                                o_of(self.act_o, i * w.L + l), o_dt, _vp(self.workspace),
-                               self.workspace.numel(), s)))
+                               self.workspace.numel(), wam.ACTION_FUSED_READY, s)))
             ds = float(sig[i + 1] - sig[i])
             calls.append((L.wam_flow_euler_step, (nf, _vp(self.x_future), _vp(inp["v_future"][i]), ds, s)))
             calls.append((L.wam_flow_euler_step, (na, _vp(self.x_act), _vp(inp["v_act"][i]), ds, s)))
             self.stages += [(f"video{i}", v0, a0), (f"action{i}", a0, len(calls))]
         self.calls = calls
         self.fused_read_call = next(i for i in range(hist_end, len(calls))
-                                    if calls[i][0] is L.wam_action_attn and calls[i][1][2] is not None)
+                                    if calls[i][0] is L.wam_action_attn_ex and calls[i][1][2] is not None)
         return self
 
     def reset_latents(self) -> None:

@@ -1,9 +1,12 @@
 // Asymmetric action attention: 32 action queries read the fused video cache of one
 // interaction layer plus their own K/V ("Fast-WAM 精读" SECTION 07; Long-WAM Summary §4.2).
 // The read is HBM-bound: per key it moves 512 B (K and V, bf16) for 32 x 4 x 128 FLOP.
-// Three kernels (bf16, D = 128, n_act <= 32):
+// Four kernels (bf16, D = 128, n_act <= 32):
 //   action_umma_kernel  T % 128 == 0: tcgen05 tensor cores, one thread-block cluster per
 //                       (episode, head), partials merged in distributed shared memory (below).
+//   action_nvfp4_kernel the same read over an NVFP4 fused pair (wam_action_attn_nvfp4): every
+//                       head cut at the same tile boundaries, one part per CTA, partials merged
+//                       through the workspace (below).
 //   action_tc_kernel    T % 64 == 0 otherwise: mma.sync tiles (M = 32 queries), Q K^T on bf16
 //                       and P V on tf32 (P keeps 10 mantissa bits; the fused cache is already
 //                       rounded to bf16 once).  Persistent and balanced: the call's tiles (per
@@ -75,6 +78,9 @@ struct TileWalk {
     }
     h = g / nb;
     t = g % nb;
+  }
+  __device__ __forceinline__ void init_at(const ActionArgs& a, int b_, int h_, int t_) {
+    b = b_, h = h_, t = t_, nb = tiles_of<kBN>(a, b_);
   }
   __device__ __forceinline__ void next(const ActionArgs& a) {
     if (++t < nb) return;
@@ -591,11 +597,41 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = bars.tmem_base;
+  auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
+    const int t = t0 + i;
+    if (t == 0) {
+      mp = is_v ? &maps.va : &maps.ka, tok = 0;
+    } else {
+      const int vt = t - 1;
+      mp = is_v ? &maps.fv : &maps.fk;
+      tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
+    }
+  };
+  auto load_kv = [&](int i) {  // K and V of the slice's tile i into stage i % kStages
+    const int st = i % kStages;
+    const CUtensorMap* mp;
+    int tok;
+    tile_src(i, false, mp, tok);
+    mbar_arrive_expect_tx(&bars.kfull[st], kTile);
+    tma_load_4d(sK(st), mp, &bars.kfull[st], 0, h, tok, b);
+    tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, h, tok, b);
+    tile_src(i, true, mp, tok);
+    mbar_arrive_expect_tx(&bars.vfull[st], kTile);
+    tma_load_4d(sV(st), mp, &bars.vfull[st], 0, h, tok, b);
+    tma_load_4d(sV(st) + kTile / 2, mp, &bars.vfull[st], 64, h, tok, b);
+  };
   // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
-  // the stream may still be finishing (programmatic dependent launch).
+  // the stream may still be finishing (programmatic dependent launch).  With a.fused_ready the
+  // caller guarantees that kernel does not write the fused pair, so the slice's first fused
+  // tiles are requested now; the action tile and Q wait for it.
+  const int n_pre = n < kStages ? n : kStages;
+  uint32_t pre = 0;  // bit i: tile i requested before the dependency wait
   if (threadIdx.x == 0) {
     prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
     prefetch_tmap(&maps.fk), prefetch_tmap(&maps.fv);
+    if (a.fused_ready)
+      for (int i = 0; i < n_pre; ++i)
+        if (t0 + i != 0) load_kv(i), pre |= 1u << i;
   }
   grid_dependency_wait();
   grid_launch_dependents();
@@ -608,17 +644,9 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       mbar_arrive_expect_tx(&bars.qfull, kQ);
       tma_load_4d(sQ, &maps.q, &bars.qfull, 0, h, 0, b);
       tma_load_4d(sQ + kQ / 2, &maps.q, &bars.qfull, 64, h, 0, b);
-      auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
-        const int t = t0 + i;
-        if (t == 0) {
-          mp = is_v ? &maps.va : &maps.ka, tok = 0;
-        } else {
-          const int vt = t - 1;
-          mp = is_v ? &maps.fv : &maps.fk;
-          tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
-        }
-      };
-      int nk = 0, nv = 0;
+      for (int i = 0; i < n_pre; ++i)  // the first stages: those not requested above
+        if (!((pre >> i) & 1u)) load_kv(i);
+      int nk = n_pre, nv = n_pre;
       for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
         if ((it & 31u) == 31u && *abort) break;
         if (nk < n && (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1))) {
@@ -941,52 +969,43 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   if (threadIdx.x == 0 && bars.abort && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
 }
 
-// ============================================================================================
-// The fused read as a persistent split over every SM: the call's tiles (per (episode, head)
-// the action tile, then the 128-key tiles of the episode's valid frames, in that order, the
-// (episode, head) runs one after another) are cut into P equal runs, one per CTA, P = the SM
-// count (at most the tile count).  A run that covers a whole (episode, head) writes O; the
-// others leave a partial (O, reference max, row sum) in the workspace, and the last CTA to
-// arrive at the (episode, head)'s ticket merges the partials by one shared log-sum-exp and
-// resets the ticket.  Inside a CTA the pipeline is the transposed tcgen05 read above (warps:
-// 0 TMA producer, 1 MMA issuer, 2-5 softmax, one key per thread), extended to runs that cross
-// from one (episode, head) to the next: the Q tile and the O^T accumulator are double-buffered
-// by segment, so the next segment's loads and MMAs start while the previous one is written out.
-namespace sk {
-constexpr int kKeys = 128;
-constexpr int kTile = kKeys * 128 * 2;   // one of K or V: 32 KB
-constexpr int kStages = 3;
-constexpr int kQ = 32 * 128 * 2;         // 8 KB
-constexpr int kP = kKeys * 128;          // P^T: 128 keys x (32 P_hi + 32 P_lo) bf16 = 16 KB
-constexpr int kThreads = 6 * 32;
-constexpr uint32_t kTmemCols = 256;      // S^T at columns 0 and 32; O^T of segment parity p at 64 + 64 p
-constexpr float kLazy = 16.f;            // reference headroom (log2 units): P <= 2^16
-struct Bars {
-  uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
-  uint64_t qfull[2], qempty[2], sfull[2], sfree[2], pfull, pfree, ofull[2], ofree[2], done;
-  uint32_t tmem_base;
-  int abort;
-  int last;  // this CTA is the last to arrive at the current segment's ticket
-  float red[4][32];
-};
-constexpr int kSmemBytes = 1024 + 2 * kQ + kStages * 2 * kTile + kP + int(sizeof(Bars)) + 64;
-static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kSlotFloats == 32 * 128 + 64, "workspace partial: O^T [128][32], m [32], l [32]");
-}  // namespace sk
+// The part of the call a CTA of the 128-key reads owns: episode b, head h, part r of k, i.e. the
+// video tiles [1 + r nv / k, 1 + (r + 1) nv / k) of (b, h), and the action tile for r = 0.  Consecutive CTAs take the same part of consecutive
+// heads, so the CTAs reading at one moment cover the same token range of every head (one fused
+// K or V token row holds all heads, H x 256 bytes).
+__device__ __forceinline__ void aligned_part(const ActionArgs& a, int cta, int& b, int& h, int& r, int& k) {
+  b = 0;
+  for (;;) {
+    k = a.kparts[b];
+    const int n_c = a.H * k;
+    if (cta < n_c || b == a.B - 1) break;
+    cta -= n_c;
+    ++b;
+  }
+  r = cta / a.H;
+  h = cta % a.H;
+}
 
 // End of one segment of a split read, in the 128 softmax threads (thread L = column d of O):
 // o[q] is the segment's unnormalised O^T column, lt[q] its row sums and m[q] its reference maxima
 // (log2 units, the same in every thread).  A segment that covers its whole (episode, head)
-// (tiles t_first = 0 .. t_last = nb - 1) writes O = o / lt.  Otherwise it stores a partial
-// (O^T [128][32], m [32], l [32]) in its workspace slot and takes a ticket; the last of the
-// (episode, head)'s parts to arrive merges every partial by one shared log-sum-exp, writes O and
-// resets the ticket.  `last` is a shared word of the CTA.
-__device__ __forceinline__ void split_finish_segment(const ActionArgs& a, int b, int h, int t_first,
-                                                     int t_last, int nb, int L, int wr, int lane,
+// (parts == 1) writes O = o / lt.  Otherwise it stores a partial (O [32 queries][128], m [32],
+// l [32]) in its workspace slot and takes a ticket; the last of the (episode, head)'s parts to
+// arrive merges every partial, its own included, in slot order (so the result does not depend
+// on the arrival order), writes O and resets the ticket.  The merge brings all partials into
+// shared memory at once with bulk copies (`stage`, room for `stage_parts` of them: the K/V ring,
+// idle by then; `mbar` an mbarrier of the CTA used only here) and merges from there: warp 0 turns
+// the maxima into per-part weights, then each warp combines 8 query rows, 4 columns per lane.
+// More parts than the stage holds are merged from global memory one part at a time.  `last` is a
+// shared word of the CTA.
+__device__ __forceinline__ void split_finish_segment(const ActionArgs& a, int b, int h, int parts,
+                                                     int slot, int L, int wr, int lane,
                                                      float (&o)[32], float (&lt)[32],
-                                                     float (&m)[32], int* last) {
+                                                     float (&m)[32], int* last, uint8_t* stage,
+                                                     int stage_parts, uint64_t* mbar,
+                                                     volatile int* abort) {
   const int bh = b * a.H + h;
-  if (t_first == 0 && t_last == nb - 1) {
+  if (parts == 1) {
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       if (q >= a.n_act) continue;
@@ -997,49 +1016,95 @@ __device__ __forceinline__ void split_finish_segment(const ActionArgs& a, int b,
     }
     return;
   }
-  const int s_bh = first_tile_of<128>(a, b, h);
-  const int c0 = cta_of_start(s_bh, a.G, a.P), c1 = cta_of_end(s_bh + nb, a.G, a.P);
-  const int parts = c1 - c0 + 1;
-  float* slot = a.ws_part + (int64_t(bh) * a.max_parts + (int(blockIdx.x) - c0)) * kSlotFloats;
-  {
-    float4* dst = reinterpret_cast<float4*>(slot + L * 32);
+  const float* part0 = a.ws_part + int64_t(bh) * a.max_parts * kSlotFloats;
+  float* mine = a.ws_part + (int64_t(bh) * a.max_parts + slot) * kSlotFloats;
 #pragma unroll
-    for (int q4 = 0; q4 < 8; ++q4) __stcg(dst + q4, make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]));
-    if (wr == 0) {
-      float mm = -INFINITY, ll = 0.f;
+  for (int q = 0; q < 32; ++q) __stcg(mine + q * 128 + L, o[q]);  // row q: one warp, 128 bytes
+  if (wr == 0) {
+    float mm = -INFINITY, ll = 0.f;
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (q == lane) mm = m[q], ll = lt[q];
-      __stcg(slot + 4096 + lane, mm);
-      __stcg(slot + 4096 + 32 + lane, ll);
-    }
+    for (int q = 0; q < 32; ++q)
+      if (q == lane) mm = m[q], ll = lt[q];
+    __stcg(mine + 4096 + lane, mm);
+    __stcg(mine + 4096 + 32 + lane, ll);
   }
-  __threadfence();
+  // the CTA's stores, ordered before one thread's release of the ticket by the CTA barrier (the
+  // fence is cumulative), so only that thread fences
   um::softmax_sync();
   if (wr == 0 && lane == 0) {
+    __threadfence();
     const int prev = atomicAdd(a.ws_count + bh, 1);
     __threadfence();
     *reinterpret_cast<volatile int*>(last) = prev == parts - 1;
   }
   um::softmax_sync();
-  if (*reinterpret_cast<volatile int*>(last)) {
-    // merge every other part's (O, m, l) into this CTA's own (m becomes the running maximum)
+  if (!*reinterpret_cast<volatile int*>(last)) return;
+
+  if (parts <= stage_parts) {
+    // every partial into shared memory (the other parts' writes were made visible before their
+    // tickets; this CTA's acquire above orders them before the async-proxy reads)
+    constexpr uint32_t kSlotBytes = uint32_t(kSlotFloats) * 4u;
+    if (wr == 0 && lane == 0) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      mbar_arrive_expect_tx(mbar, kSlotBytes * uint32_t(parts));
+      for (int p = 0; p < parts; ++p)
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                smem_u32(stage + p * kSlotBytes)),
+            "l"(part0 + int64_t(p) * kSlotFloats), "r"(kSlotBytes), "r"(smem_u32(mbar))
+            : "memory");
+    }
+    if (!mbar_wait(mbar, 0)) {  // bounded: a wait that gives up reports a timeout, O is not written
+      *abort = 1;
+      return;
+    }
+    const float* sp = reinterpret_cast<const float*>(stage);
+    float* wts = reinterpret_cast<float*>(stage + parts * kSlotBytes);  // [parts][32], then 1 / l [32]
+    if (wr == 0) {
+      const int q = lane;
+      float M = -INFINITY;
+      for (int p = 0; p < parts; ++p) M = fmaxf(M, sp[p * kSlotFloats + 4096 + q]);
+      float den = 0.f;
+      for (int p = 0; p < parts; ++p) {
+        const float w = tc05::fast_exp2(sp[p * kSlotFloats + 4096 + q] - M);
+        wts[p * 32 + q] = w;
+        den = fmaf(w, sp[p * kSlotFloats + 4096 + 32 + q], den);
+      }
+      wts[parts * 32 + q] = den > 0.f ? 1.f / den : 0.f;
+    }
+    um::softmax_sync();
+    for (int q = wr; q < a.n_act; q += 4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p = 0; p < parts; ++p) {
+        const float w = wts[p * 32 + q];
+        const float4 x = *reinterpret_cast<const float4*>(sp + p * kSlotFloats + q * 128 + 4 * lane);
+        acc.x = fmaf(w, x.x, acc.x), acc.y = fmaf(w, x.y, acc.y);
+        acc.z = fmaf(w, x.z, acc.z), acc.w = fmaf(w, x.w, acc.w);
+      }
+      const float inv = wts[parts * 32 + q];
+      const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + 4 * lane;
+      if (a.o_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.o) + off) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      } else {
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + off) =
+            make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+      }
+    }
+  } else {
+    // more parts than the stage holds: thread L merges its column part by part from global memory
+#pragma unroll
+    for (int q = 0; q < 32; ++q) o[q] = 0.f, lt[q] = 0.f, m[q] = -INFINITY;
     for (int p = 0; p < parts; ++p) {
-      if (c0 + p == int(blockIdx.x)) continue;
-      const float4* ps = reinterpret_cast<const float4*>(a.ws_part + (int64_t(bh) * a.max_parts + p) * kSlotFloats);
+      const float* ps = part0 + int64_t(p) * kSlotFloats;
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 x = __ldcg(ps + L * 8 + q4), y = __ldcg(ps + 1024 + q4), z = __ldcg(ps + 1032 + q4);
-        const float po[4] = {x.x, x.y, x.z, x.w}, pm[4] = {y.x, y.y, y.z, y.w}, pz[4] = {z.x, z.y, z.z, z.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int q = 4 * q4 + e;
-          const float mn = fmaxf(m[q], pm[e]);
-          const float fa = exp2f(m[q] - mn), fb = exp2f(pm[e] - mn);
-          o[q] = fmaf(o[q], fa, po[e] * fb);
-          lt[q] = fmaf(lt[q], fa, pz[e] * fb);
-          m[q] = mn;
-        }
+      for (int q = 0; q < 32; ++q) {
+        const float pm = __ldcg(ps + 4096 + q), pz = __ldcg(ps + 4096 + 32 + q), po = __ldcg(ps + q * 128 + L);
+        const float mn = fmaxf(m[q], pm);
+        const float fa = tc05::fast_exp2(m[q] - mn), fb = tc05::fast_exp2(pm - mn);
+        o[q] = fmaf(o[q], fa, po * fb);
+        lt[q] = fmaf(lt[q], fa, pz * fb);
+        m[q] = mn;
       }
     }
 #pragma unroll
@@ -1050,339 +1115,8 @@ __device__ __forceinline__ void split_finish_segment(const ActionArgs& a, int b,
       if (a.o_f32) static_cast<float*>(a.o)[off] = val;
       else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
     }
-    if (wr == 0 && lane == 0) a.ws_count[bh] = 0;  // ready for the next call
   }
-  um::softmax_sync();  // `last` is rewritten by the next segment
-}
-
-__global__ void __launch_bounds__(sk::kThreads, 1)
-action_split_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
-  using namespace sk;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  auto sQ = [&](int s) { return base + (s & 1) * kQ; };
-  auto sK = [&](int st) { return base + 2 * kQ + st * 2 * kTile; };
-  auto sV = [&](int st) { return base + 2 * kQ + st * 2 * kTile + kTile; };
-  uint8_t* sP = base + 2 * kQ + kStages * 2 * kTile;
-  sk::Bars& bars = *reinterpret_cast<sk::Bars*>(sP + kP);
-  volatile int* abort = &bars.abort;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned FULL = 0xffffffffu;
-  const int g0 = int(int64_t(blockIdx.x) * a.G / a.P), g1 = int(int64_t(blockIdx.x + 1) * a.G / a.P);
-  const int n = g1 - g0;  // >= 1: P <= G
-  const int tpf = a.T / kKeys;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.kfull[i], 1);
-      mbar_init(&bars.kempty[i], 1);
-      mbar_init(&bars.vfull[i], 1);
-      mbar_init(&bars.vempty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.qfull[i], 1);
-      mbar_init(&bars.qempty[i], 1);
-      mbar_init(&bars.sfull[i], 1);
-      mbar_init(&bars.sfree[i], 4);
-      mbar_init(&bars.ofull[i], 1);
-      mbar_init(&bars.ofree[i], 4);
-    }
-    mbar_init(&bars.pfull, 4);
-    mbar_init(&bars.pfree, 1);
-    mbar_init(&bars.done, 1);
-    bars.abort = 0;
-    bars.last = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tc05::tmem_alloc(&bars.tmem_base, kTmemCols);
-    tc05::tmem_relinquish();
-  }
-  tc05::fence_before_sync();
-  __syncthreads();
-  tc05::fence_after_sync();
-  const uint32_t tmem = bars.tmem_base;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
-    prefetch_tmap(&maps.fk), prefetch_tmap(&maps.fv);
-  }
-  grid_dependency_wait();
-  grid_launch_dependents();
-
-  // token of the first key of tile (b, t): t = 0 the action keys, t >= 1 the valid frames'
-  auto tile_src = [&](const TileWalk<kKeys>& w, bool is_v, const CUtensorMap*& mp, int& tok) {
-    if (w.t == 0) {
-      mp = is_v ? &maps.va : &maps.ka, tok = 0;
-    } else {
-      const int vt = w.t - 1;
-      mp = is_v ? &maps.fv : &maps.fk;
-      tok = int(a.fl.vlist[w.b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
-    }
-  };
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    // K (with the Q tile of each new segment) and V advance independently through their rings.
-    if (lane == 0) {
-      TileWalk<kKeys> kw, vw;
-      kw.init(a, g0);
-      vw.init(a, g0);
-      int nk = 0, nv = 0, kseg = -1;
-      for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
-        if ((it & 31u) == 31u && *abort) break;
-        if (nk < n) {
-          const bool new_seg = nk == 0 || kw.t == 0;
-          const int s = kseg + 1;
-          const bool can = (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1)) &&
-                           (!new_seg || s < 2 || mbar_test_wait(&bars.qempty[s & 1], ((s >> 1) - 1) & 1));
-          if (can) {
-            if (new_seg) {
-              kseg = s;
-              mbar_arrive_expect_tx(&bars.qfull[s & 1], kQ);
-              tma_load_4d(sQ(s), &maps.q, &bars.qfull[s & 1], 0, kw.h, 0, kw.b);
-              tma_load_4d(sQ(s) + kQ / 2, &maps.q, &bars.qfull[s & 1], 64, kw.h, 0, kw.b);
-            }
-            const int st = nk % kStages;
-            const CUtensorMap* mp;
-            int tok;
-            tile_src(kw, false, mp, tok);
-            mbar_arrive_expect_tx(&bars.kfull[st], kTile);
-            tma_load_4d(sK(st), mp, &bars.kfull[st], 0, kw.h, tok, kw.b);
-            tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, kw.h, tok, kw.b);
-            ++nk;
-            kw.next(a);
-          }
-        }
-        if (nv < n && (nv < kStages || mbar_test_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))) {
-          const int st = nv % kStages;
-          const CUtensorMap* mp;
-          int tok;
-          tile_src(vw, true, mp, tok);
-          mbar_arrive_expect_tx(&bars.vfull[st], kTile);
-          tma_load_4d(sV(st), mp, &bars.vfull[st], 0, vw.h, tok, vw.b);
-          tma_load_4d(sV(st) + kTile / 2, mp, &bars.vfull[st], 64, vw.h, tok, vw.b);
-          ++nv;
-          vw.next(a);
-        }
-      }
-      if (nk < n || nv < n) *abort = 1;
-      // Loads still in flight land before the CTA leaves (only after an abort can any be).
-      for (int i = (nk > kStages ? nk - kStages : 0); i < nk; ++i) mbar_wait(&bars.kfull[i % kStages], (i / kStages) & 1);
-      for (int i = (nv > kStages ? nv - kStages : 0); i < nv; ++i) mbar_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
-      for (int s = (kseg > 1 ? kseg - 1 : 0); s <= kseg; ++s) mbar_wait(&bars.qfull[s & 1], (s >> 1) & 1);
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // S^T of up to two tiles ahead is issued as soon as its K tile (and its segment's Q tile)
-    // has landed and its tensor-memory buffer has been read; P V of the current tile waits for
-    // its P, and the first P V of a segment for that segment's O^T buffer to have been read out.
-    if (lane == 0) {
-      const uint32_t idS = tc05::idesc_bf16_f32(128, 32, false, false);
-      const uint32_t idO = tc05::idesc_bf16_f32(128, 64, true, true);
-      TileWalk<kKeys> sw, pw;
-      sw.init(a, g0);
-      pw.init(a, g0);
-      int ns = 0, sseg = -1, pseg = -1;
-      bool ok = true;
-      for (int i = 0; ok && i < n; ++i) {
-        const bool p_first = i == 0 || pw.t == 0;
-        const bool p_last = i == n - 1 || pw.t == pw.nb - 1;
-        if (p_first) ++pseg;
-        bool v_ready = false, p_ready = false, o_ready = !(p_first && pseg >= 2);
-        for (uint32_t it = 0;; ++it) {
-          if (ns < n && ns <= i + 2) {
-            const bool s_first = ns == 0 || sw.t == 0;
-            const int s = sseg + (s_first ? 1 : 0);
-            if (mbar_test_wait(&bars.kfull[ns % kStages], (ns / kStages) & 1) &&
-                (!s_first || mbar_test_wait(&bars.qfull[s & 1], (s >> 1) & 1)) &&
-                (ns < 2 || mbar_test_wait(&bars.sfree[ns & 1], ((ns >> 1) - 1) & 1))) {
-              const bool s_last = ns == n - 1 || sw.t == sw.nb - 1;
-              sseg = s;
-              const int st = ns % kStages;
-              tc05::fence_after_sync();
-              const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ(s));
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                tc05::mma_ss(tmem + 32 * (ns & 1),
-                             tc05::smem_desc_sw128(k_s + (kk >> 2) * (kTile / 2) + (kk & 3) * 32, 16, 1024),
-                             tc05::smem_desc_sw128(q_s + (kk >> 2) * (kQ / 2) + (kk & 3) * 32, 16, 1024), idS,
-                             kk > 0 ? 1u : 0u);
-              tc05::mma_commit(&bars.sfull[ns & 1]);
-              tc05::mma_commit(&bars.kempty[st]);
-              if (s_last) tc05::mma_commit(&bars.qempty[s & 1]);
-              ++ns;
-              sw.next(a);
-            }
-          }
-          if (ns > i) {
-            v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
-            o_ready = o_ready || mbar_test_wait(&bars.ofree[pseg & 1], ((pseg >> 1) - 1) & 1);
-            p_ready = v_ready && o_ready && mbar_test_wait(&bars.pfull, i & 1);
-            if (p_ready) break;
-          }
-          if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
-          if ((it & 31u) == 31u && *abort) { ok = false; break; }
-        }
-        if (!ok) break;
-        tc05::fence_after_sync();
-        const int st = i % kStages;
-        const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP);
-        const uint32_t o_t = tmem + 64 + 64 * (pseg & 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc05::mma_ss(o_t, tc05::smem_desc_sw128(v_s + kk * 2048, kTile / 2, 1024),
-                       tc05::smem_desc_sw128(p_s + kk * 2048, kTile / 2, 1024), idO,
-                       (!p_first || kk > 0) ? 1u : 0u);
-        tc05::mma_commit(&bars.pfree);
-        tc05::mma_commit(&bars.vempty[st]);
-        if (p_last) tc05::mma_commit(&bars.ofull[pseg & 1]);
-        pw.next(a);
-      }
-      tc05::mma_commit(&bars.done);  // arrives once every MMA issued above has completed
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax, one key per thread
-    // Every wait in front of a warp-collective instruction is voted across the warp, and all
-    // four warps run the same sequence of named barriers whatever happens, so after a timeout
-    // they keep walking their tiles without doing work and no barrier waits on a warp that left.
-    const int quarter = warp & 3;
-    const int L = 32 * quarter + lane;  // key of the tile (S^T lane) and column d of O (O^T lane)
-    const uint32_t lane_off = uint32_t(32 * quarter) << 16;
-    const int wr = warp - 2;
-    const float c = a.scale_log2;
-    bool ok = true;
-    float m[32], l[32];
-    TileWalk<kKeys> tw;
-    tw.init(a, g0);
-    int seg = -1, i_first = 0;
-    for (int i = 0; i < n; ++i, tw.next(a)) {
-      if (i == 0 || tw.t == 0) {
-        ++seg;
-        i_first = i;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) m[q] = -INFINITY, l[q] = 0.f;
-      }
-      const bool last = i == n - 1 || tw.t == tw.nb - 1;
-      ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.sfull[i & 1], (i >> 1) & 1, abort));
-      uint32_t sr[32];
-      if (ok) {
-        tc05::fence_after_sync();
-        tc05::tmem_ld32(tmem + 32 * (i & 1) + lane_off, sr);
-        tc05::tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) sr[q] = 0u;
-      }
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.sfree[i & 1]);
-      const bool kv = tw.t != 0 || L < a.n_act;  // keys past n_act in the action tile are padding
-      const uint32_t o_t = tmem + 64 + 64 * (seg & 1);
-      float ymax = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 32; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));
-      if (um::softmax_any(ok && kv && !(ymax <= kLazy))) {
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = kv ? __uint_as_float(sr[q]) * c : -INFINITY;
-        bars.red[wr][lane] = um::reduce_scatter32<true>(v, lane);
-        um::softmax_sync();
-        float al[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float tm = fmaxf(fmaxf(bars.red[0][q], bars.red[1][q]), fmaxf(bars.red[2][q], bars.red[3][q]));
-          const float mn = tm > m[q] + kLazy ? tm : m[q];
-          al[q] = tc05::fast_exp2(m[q] - mn);
-          l[q] *= al[q];
-          m[q] = mn;
-        }
-        if (i > i_first) {  // O^T holds the P V of the segment's earlier tiles: rescale it
-          ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
-          if (ok) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t o[32];
-              tc05::tmem_ld32(o_t + 32 * half + lane_off, o);
-              tc05::tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
-              tc05::tmem_st32(o_t + 32 * half + lane_off, o);
-            }
-            tc05::tmem_wait_st();
-          }
-        }
-        um::softmax_sync();
-      }
-      uint32_t pk[16], pl[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j]), c, -m[2 * j])) : 0.f;
-        const float p1 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -m[2 * j + 1])) : 0.f;
-        l[2 * j] += p0, l[2 * j + 1] += p1;
-        pk[j] = pack_bf16(p0, p1);
-        pl[j] = pack_bf16(p0 - __uint_as_float(pk[j] << 16), p1 - __uint_as_float(pk[j] & 0xffff0000u));
-      }
-      if (i > 0) ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
-      if (ok) {
-        uint8_t* row = sP + L * 128;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          *reinterpret_cast<uint4*>(row + ((ch ^ (L & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(row + (((ch + 4) ^ (L & 7)) << 4)) =
-              make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
-        }
-      }
-      tc05::fence_proxy_async_smem();
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.pfull);
-      if (!last) continue;
-
-      // ---- segment done: O^T column d = L and the row sums over all 128 keys of each tile
-      float o[32];
-      ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.ofull[seg & 1], (seg >> 1) & 1, abort));
-      if (ok) {
-        uint32_t ohi[32], olo[32];
-        tc05::fence_after_sync();
-        tc05::tmem_ld32(o_t + lane_off, ohi);
-        tc05::tmem_ld32(o_t + 32 + lane_off, olo);
-        tc05::tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = 0.f;
-      }
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.ofree[seg & 1]);
-      {
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = l[q];
-        bars.red[wr][lane] = um::reduce_scatter32<false>(v, lane);
-      }
-      um::softmax_sync();
-      float lt[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
-      um::softmax_sync();  // bars.red is rewritten by the next tile
-      split_finish_segment(a, tw.b, tw.h, tw.t - (i - i_first), tw.t, tw.nb, L, wr, lane, o, lt, m,
-                           &bars.last);
-    }
-  }
-
-  // ---------------------------------------------------------------- teardown
-  __syncwarp();
-  tc05::fence_before_sync();
-  __syncthreads();
-  if (warp == 1) {
-    mbar_wait(&bars.done, 0);  // every MMA has completed (bounded)
-    tc05::fence_after_sync();
-    tc05::tmem_dealloc(tmem, kTmemCols);
-  }
-  if (threadIdx.x == 0 && bars.abort && a.err) atomicExch(a.err, int(WAM_ERR_TIMEOUT));
+  if (wr == 0 && lane == 0) a.ws_count[bh] = 0;  // ready for the next call
 }
 
 // ============================================================================================
@@ -1392,8 +1126,8 @@ action_split_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
 // memory and the operand type:
 //  - the producer copies a video tile's 8 KB of codes and 1 KB of scales with two bulk copies into
 //    a raw ring (3 slots for K, 3 for V); one converter warp for K (warp 6) and one for V
-//    (warp 7), four key rows per thread, decode e2m1 x e4m3 into fp16, exactly (a product has
-//    at most 6 significant bits), in the 128-byte-swizzled layout the MMA descriptors name;
+//    (warp 7) decode e2m1 x e4m3 into fp16, exactly (a product has at most 6 significant bits),
+//    in the 128-byte-swizzled layout the MMA descriptors name;
 //  - the action tile and the Q tile arrive in bf16 by TMA and are converted in place to fp16;
 //  - both MMAs run on fp16 operands (P = P_hi + P_lo in fp16; the reference headroom is 2^15 so
 //    P stays below fp16's largest finite value);
@@ -1419,14 +1153,18 @@ struct Bars {
   uint64_t vland[kStages], vfull[kStages], vempty[kStages];
   uint64_t rkfull[kRaw], rkfree[kRaw], rvfull[kRaw], rvfree[kRaw];
   uint64_t sfull[2], sfree[2], pfull, pfree, ofull[2], ofree[2], done;
+  uint64_t mfull;
   uint32_t tmem_base;
   int abort;
   int last;
+  int part_r, part_k;
   float red[4][32];
 };
 constexpr int kSmemBytes =
     1024 + 2 * kQ + kStages * 2 * kTile + 2 * kRaw * kRawBytes + kP + int(sizeof(Bars)) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory");
+// partials the fp16 K/V stages and the raw rings (contiguous) hold for the merge
+constexpr int kStageParts = (kStages * 2 * kTile + 2 * kRaw * kRawBytes - 128) / (kSlotFloats * 4 + 128);
 
 // Instruction descriptor of .kind::f16 with fp16 A and B and an fp32 accumulator (format 0).
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major, bool a_mn_major) {
@@ -1475,29 +1213,28 @@ __device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-// Key row r of a raw tile (64 bytes of codes, 8 E4M3 scales) decoded into row r of an fp16 tile.
-__device__ __forceinline__ void decode_row(const uint8_t* raw, uint8_t* tile, int r) {
-  const uint4* cr = reinterpret_cast<const uint4*>(raw + r * 64);
+// 16 bytes of codes (32 elements: blocks 2 q and 2 q + 1 of key row r) of a raw tile decoded into
+// the fp16 tile.  A warp decodes 8 rows at a time, lane t taking row 8 i + t / 4 and chunk t % 4,
+// so each load instruction reads 512 contiguous bytes of codes (no bank conflict) and the rows'
+// 8 scale bytes are shared by 4 lanes.
+__device__ __forceinline__ void decode_chunk(const uint8_t* raw, uint8_t* tile, int r, int q) {
+  const uint4 c = *reinterpret_cast<const uint4*>(raw + r * 64 + q * 16);
   const uint2 sc = *reinterpret_cast<const uint2*>(raw + kCodes + r * 8);
-  const uint32_t sw[2] = {sc.x, sc.y};
+  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+  const uint32_t sw = q < 2 ? sc.x : sc.y;  // scale bytes 2 q and 2 q + 1
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {  // 16 bytes of codes = 32 elements = two scale blocks
-    const uint4 c = cr[q];
-    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+  for (int half = 0; half < 2; ++half) {  // one 16-element block, two 8-element chunks
+    const int blk = 2 * q + half;
+    const uint32_t s2 = e4m3_to_f16x2((sw >> (8 * (blk & 3))) & 0xFFu);
+    uint32_t out[8];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {  // one 16-element block, two 8-element chunks
-      const int blk = 2 * q + half;
-      const uint32_t s2 = e4m3_to_f16x2((sw[blk >> 2] >> (8 * (blk & 3))) & 0xFFu);
-      uint32_t out[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t word = cw[2 * half + (e >> 2)];
-        out[e] = mul_f16x2(e2m1x2_to_f16x2((word >> (8 * (e & 3))) & 0xFFu), s2);
-      }
-      const int ch0 = 2 * blk;  // 8-element chunks 2 blk and 2 blk + 1 of the row
-      *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0)) = make_uint4(out[0], out[1], out[2], out[3]);
-      *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0 + 8)) = make_uint4(out[4], out[5], out[6], out[7]);
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t word = cw[2 * half + (e >> 2)];
+      out[e] = mul_f16x2(e2m1x2_to_f16x2((word >> (8 * (e & 3))) & 0xFFu), s2);
     }
+    const int ch0 = 2 * blk;  // 8-element chunks 2 blk and 2 blk + 1 of the row
+    *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0)) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0 + 8)) = make_uint4(out[4], out[5], out[6], out[7]);
   }
 }
 }  // namespace fq
@@ -1517,8 +1254,12 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   volatile int* abort = &bars.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
-  const int g0 = int(int64_t(blockIdx.x) * a.G / a.P), g1 = int(int64_t(blockIdx.x + 1) * a.G / a.P);
-  const int n = g1 - g0;
+  int part_b, part_h, part_r, part_k;
+  aligned_part(a, int(blockIdx.x), part_b, part_h, part_r, part_k);
+  // the video tiles 1 .. nv of (b, h) cut evenly; part 0 also takes the action tile (t = 0)
+  const int part_nv = tiles_of<kKeys>(a, part_b) - 1;
+  const int t0 = part_r == 0 ? 0 : 1 + part_r * part_nv / part_k;
+  const int n = 1 + (part_r + 1) * part_nv / part_k - t0;  // n >= 1: k <= nv
   const int tpf = a.T / kKeys;
   const int64_t N = int64_t(a.F) * a.T;
 
@@ -1551,6 +1292,8 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     mbar_init(&bars.done, 1);
     bars.abort = 0;
     bars.last = 0;
+    bars.part_r = part_r, bars.part_k = part_k;
+    mbar_init(&bars.mfull, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -1561,25 +1304,43 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = bars.tmem_base;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
-  }
-  grid_dependency_wait();
-  grid_launch_dependents();
-
   // head-major row of the first key of video tile t of (b, h)
   auto raw_row = [&](const TileWalk<kKeys>& w) {
     const int vt = w.t - 1;
     const int64_t tok = int64_t(a.fl.vlist[w.b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
     return (int64_t(w.b) * a.H + w.h) * N + tok;
   };
+  // With a.fused_ready (the previous kernel does not write the NVFP4 pair) the first raw tiles
+  // are requested before the dependency wait; bit i of pre: tile i of the part.
+  uint32_t pre = 0;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
+    if (a.fused_ready) {
+      TileWalk<kKeys> w;
+      w.init_at(a, part_b, part_h, t0);
+      for (int i = 0, r = 0; i < n && r < kRaw; ++i, w.next(a)) {
+        if (w.t == 0) continue;
+        const int64_t row = raw_row(w);
+        mbar_arrive_expect_tx(&bars.rkfull[r], kRawBytes);
+        bulk_load(rK(r), a.k_codes + row * 64, kCodes, &bars.rkfull[r]);
+        bulk_load(rK(r) + kCodes, a.k_scales + row * 8, kScales, &bars.rkfull[r]);
+        mbar_arrive_expect_tx(&bars.rvfull[r], kRawBytes);
+        bulk_load(rV(r), a.v_codes + row * 64, kCodes, &bars.rvfull[r]);
+        bulk_load(rV(r) + kCodes, a.v_scales + row * 8, kScales, &bars.rvfull[r]);
+        pre |= 1u << i;
+        ++r;
+      }
+    }
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       TileWalk<kKeys> kw, vw;
-      kw.init(a, g0);
-      vw.init(a, g0);
+      kw.init_at(a, part_b, part_h, t0);
+      vw.init_at(a, part_b, part_h, t0);
       int nk = 0, nv = 0, kseg = -1, rk = 0, rv = 0;
       int kact[kStages] = {0, 0}, vact[kStages] = {0, 0};
       for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
@@ -1605,10 +1366,12 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
               ++kact[st];
             } else {
               const int sl = rk % kRaw;
-              const int64_t row = raw_row(kw);
-              mbar_arrive_expect_tx(&bars.rkfull[sl], kRawBytes);
-              bulk_load(rK(sl), a.k_codes + row * 64, kCodes, &bars.rkfull[sl]);
-              bulk_load(rK(sl) + kCodes, a.k_scales + row * 8, kScales, &bars.rkfull[sl]);
+              if (!(nk < 32 && ((pre >> nk) & 1u))) {  // not requested before the wait
+                const int64_t row = raw_row(kw);
+                mbar_arrive_expect_tx(&bars.rkfull[sl], kRawBytes);
+                bulk_load(rK(sl), a.k_codes + row * 64, kCodes, &bars.rkfull[sl]);
+                bulk_load(rK(sl) + kCodes, a.k_scales + row * 8, kScales, &bars.rkfull[sl]);
+              }
               ++rk;
             }
             ++nk;
@@ -1628,10 +1391,12 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
               ++vact[st];
             } else {
               const int sl = rv % kRaw;
-              const int64_t row = raw_row(vw);
-              mbar_arrive_expect_tx(&bars.rvfull[sl], kRawBytes);
-              bulk_load(rV(sl), a.v_codes + row * 64, kCodes, &bars.rvfull[sl]);
-              bulk_load(rV(sl) + kCodes, a.v_scales + row * 8, kScales, &bars.rvfull[sl]);
+              if (!(nv < 32 && ((pre >> nv) & 1u))) {
+                const int64_t row = raw_row(vw);
+                mbar_arrive_expect_tx(&bars.rvfull[sl], kRawBytes);
+                bulk_load(rV(sl), a.v_codes + row * 64, kCodes, &bars.rvfull[sl]);
+                bulk_load(rV(sl) + kCodes, a.v_scales + row * 8, kScales, &bars.rvfull[sl]);
+              }
               ++rv;
             }
             ++nv;
@@ -1651,12 +1416,12 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     }
   } else if (warp >= 6) {
     // ---------------------------------------------------------------- converters
-    // warp 6: Q and K tiles; warp 7: V tiles.  Lane t handles key rows t, t + 32, t + 64 and
-    // t + 96 of a raw tile; in-place bf16 tiles are split by 16-byte chunks.
+    // warp 6: Q and K tiles; warp 7: V tiles.  A raw tile is decoded 8 rows per step
+    // (decode_chunk); in-place bf16 tiles are split by 16-byte chunks.
     const bool is_k = warp == 6;
     const int t = lane;
     TileWalk<kKeys> cw;
-    cw.init(a, g0);
+    cw.init_at(a, part_b, part_h, t0);
     int seg = -1, r = 0;
     int nact[kStages] = {0, 0};
     bool ok = true;
@@ -1684,8 +1449,8 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
         ok = __all_sync(FULL, ok && um::wait_or_abort(&full[sl], (r / kRaw) & 1, abort));
         if (ok) {
           const uint8_t* raw = is_k ? rK(sl) : rV(sl);
-#pragma unroll 1
-          for (int rr = 0; rr < 4; ++rr) decode_row(raw, tile, t + 32 * rr);
+#pragma unroll 2
+          for (int it = 0; it < 16; ++it) decode_chunk(raw, tile, 8 * it + (t >> 2), t & 3);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(is_k ? &bars.rkfree[sl] : &bars.rvfree[sl]);
@@ -1701,8 +1466,8 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
       const uint32_t idS = idesc_f16_f32(128, 32, false, false);
       const uint32_t idO = idesc_f16_f32(128, 64, true, true);
       TileWalk<kKeys> sw, pw;
-      sw.init(a, g0);
-      pw.init(a, g0);
+      sw.init_at(a, part_b, part_h, t0);
+      pw.init_at(a, part_b, part_h, t0);
       int ns = 0, sseg = -1, pseg = -1;
       bool ok = true, vid_started = false;
       for (int i = 0; ok && i < n; ++i) {
@@ -1774,7 +1539,7 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     bool ok = true;
     float m[32], l[32];
     TileWalk<kKeys> tw;
-    tw.init(a, g0);
+    tw.init_at(a, part_b, part_h, t0);
     int seg = -1, i_first = 0;
     bool has_act = false, has_vid = false;  // accumulators written in this segment so far
     for (int i = 0; i < n; ++i, tw.next(a)) {
@@ -1911,8 +1676,9 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
 #pragma unroll
       for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
       um::softmax_sync();
-      split_finish_segment(a, tw.b, tw.h, tw.t - (i - i_first), tw.t, tw.nb, L, wr, lane, o, lt, m,
-                           &bars.last);
+      split_finish_segment(a, tw.b, tw.h, *reinterpret_cast<volatile int*>(&bars.part_k),
+                           *reinterpret_cast<volatile int*>(&bars.part_r), L, wr, lane, o, lt, m, &bars.last,
+                           sK(0), kStageParts, &bars.mfull, abort);
     }
   }
 
@@ -2074,6 +1840,40 @@ int action_tc_max_parts(const ActionArgs& a, int P, int G) {
   return mx;
 }
 
+int action_aligned_plan(ActionArgs& a, int sms) {
+  // part size S video tiles: the smallest that fits every part of every head in one wave of
+  // `sms` CTAs (or one part per head when even that does not fit); kparts[b] = ceil(nv_b / S)
+  int G = 0, V = 0, max_nv = 1;
+  for (int b = 0; b < a.B; ++b) {
+    const int nv = a.with_video ? int(a.fl.nvalid[b]) * (a.T / 128) : 0;
+    G += a.H * (1 + nv);
+    V += a.H * nv;
+    max_nv = nv > max_nv ? nv : max_nv;
+  }
+  int S = sms > 0 ? (V + sms - 1) / sms : max_nv;
+  if (S < 1) S = 1;
+  for (;; ++S) {
+    int64_t total = 0;
+    for (int b = 0; b < a.B; ++b) {
+      const int nv = a.with_video ? int(a.fl.nvalid[b]) * (a.T / 128) : 0;
+      total += int64_t(a.H) * (nv > 0 ? (nv + S - 1) / S : 1);
+    }
+    if (total <= sms || S >= max_nv) break;
+  }
+  int P = 0, mx = 1;
+  for (int b = 0; b < a.B; ++b) {
+    const int nv = a.with_video ? int(a.fl.nvalid[b]) * (a.T / 128) : 0;
+    const int k = nv > 0 ? (nv + S - 1) / S : 1;
+    a.kparts[b] = uint16_t(k);
+    P += a.H * k;
+    mx = k > mx ? k : mx;
+  }
+  a.G = G;
+  a.P = P;
+  a.max_parts = mx;
+  return P;
+}
+
 size_t action_tc_workspace_bytes(int BH, int max_parts) {
   if (max_parts <= 1) return 0;
   return kTicketBytes + size_t(BH) * max_parts * kSlotFloats * sizeof(float);
@@ -2156,10 +1956,11 @@ cudaError_t launch_action_tc(const ActionArgs& a, cudaStream_t s) {
     e = cudaFuncSetAttribute(action_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, um::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (umma) {
-    e = cudaFuncSetAttribute(action_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sk::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(action_split_kernel, dim3(unsigned(a.P)), dim3(sk::kThreads), sk::kSmemBytes, s,
-                      0, a, maps);
+    ActionArgs ac = a;
+    ac.ksplit = umma_split(a.B * a.H, dev);
+    if (ac.ksplit < 1) return cudaErrorUnknown;
+    return launch_pdl(action_umma_kernel, dim3(unsigned(a.B * a.H * ac.ksplit)), dim3(um::kThreads),
+                      um::kSmemBytes, s, unsigned(ac.ksplit), ac, maps);
   }
   // 64-key tiles (T % 128 != 0): the mma.sync kernel
   action_tc_kernel<64><<<a.P, kThreads, kSmemBytes, s>>>(a, maps);

@@ -477,9 +477,13 @@ static wam_status action_plan(wam::ActionArgs& a, size_t* bytes) {
   if (sms <= 0) return fail(WAM_ERR_CUDA, "wam_action_attn: no CUDA device");
   if (int64_t(a.B) * a.H * int64_t(sizeof(int)) > int64_t(wam::kTicketBytes))
     return fail(WAM_ERR_UNSUPPORTED, "wam_action_attn: B * H exceeds %d", int(wam::kTicketBytes / sizeof(int)));
-  a.G = wam::action_tc_total_tiles(a);
-  a.P = a.G < sms ? a.G : sms;
-  a.max_parts = wam::action_tc_max_parts(a, a.P, a.G);
+  if (a.T % 128 == 0) {
+    wam::action_aligned_plan(a, sms);  // the 128-key tensor-core reads
+  } else {
+    a.G = wam::action_tc_total_tiles(a);  // the 64-key mma.sync read: a flat split
+    a.P = a.G < sms ? a.G : sms;
+    a.max_parts = wam::action_tc_max_parts(a, a.P, a.G);
+  }
   *bytes = wam::action_tc_workspace_bytes(a.B * a.H, a.max_parts);
   return WAM_OK;
 }
@@ -506,6 +510,16 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const v
                            const void* fused_v, int32_t n_act, const void* qa, const void* ka,
                            const void* va, void* o, wam_dtype o_dt, void* workspace,
                            size_t ws_bytes, wam_stream_t stream) {
+  return wam_action_attn_ex(layout, dt, fused_k, fused_v, n_act, qa, ka, va, o, o_dt, workspace,
+                            ws_bytes, 0u, stream);
+}
+
+wam_status wam_action_attn_ex(const wam_video_layout* layout, wam_dtype dt, const void* fused_k,
+                              const void* fused_v, int32_t n_act, const void* qa, const void* ka,
+                              const void* va, void* o, wam_dtype o_dt, void* workspace,
+                              size_t ws_bytes, uint32_t flags, wam_stream_t stream) {
+  if (flags & ~uint32_t(WAM_ACTION_FUSED_READY))
+    return fail(WAM_ERR_INVALID_ARGUMENT, "unknown flags 0x%x", unsigned(flags));
   Geo g;
   WAM_CHECK(check_layout(layout, g));
   WAM_CHECK(check_dtype(dt, "dt"));
@@ -530,6 +544,7 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt, const v
   a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.n_act = n_act;
   a.o_f32 = o_dt == WAM_F32;
   a.with_video = fused_k != nullptr;
+  a.fused_ready = (flags & WAM_ACTION_FUSED_READY) ? 1 : 0;
   a.scale_log2 = float(wam::kLog2e / std::sqrt(double(g.D)));
   a.err = device_error_word();
   fill_vlists(g, a.fl);
@@ -557,7 +572,9 @@ wam_status wam_action_attn_nvfp4(const wam_video_layout* layout, const void* k_c
                                  const void* v_scales, const float* v_sg, int32_t n_act,
                                  const void* qa, const void* ka, const void* va, void* o,
                                  wam_dtype o_dt, void* workspace, size_t ws_bytes,
-                                 wam_stream_t stream) {
+                                 uint32_t flags, wam_stream_t stream) {
+  if (flags & ~uint32_t(WAM_ACTION_FUSED_READY))
+    return fail(WAM_ERR_INVALID_ARGUMENT, "unknown flags 0x%x", unsigned(flags));
   Geo g;
   WAM_CHECK(check_layout(layout, g));
   WAM_CHECK(check_dtype(o_dt, "o_dt"));
@@ -586,6 +603,7 @@ wam_status wam_action_attn_nvfp4(const wam_video_layout* layout, const void* k_c
   a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.n_act = n_act;
   a.o_f32 = o_dt == WAM_F32;
   a.with_video = 1;
+  a.fused_ready = (flags & WAM_ACTION_FUSED_READY) ? 1 : 0;
   a.scale_log2 = float(wam::kLog2e / std::sqrt(double(g.D)));
   a.err = device_error_word();
   fill_vlists(g, a.fl);

@@ -69,9 +69,13 @@ struct ActionArgs {
   int32_t P;          // CTAs of the persistent grid
   int32_t G;          // tiles of the whole call (all episodes and heads)
   int32_t max_parts;  // workspace slots per (episode, head)
+  // 128-key reads: every head of episode b is cut into kparts[b] parts with the same tile
+  // boundaries; CTA c of episode b's block of H * kparts[b] CTAs reads part c / H of head c % H
+  uint16_t kparts[WAM_MAX_EPISODE_FRAMES];
   float* ws_part;     // partial (O, m, l) slots [B*H][max_parts][32*128 + 64]
   int* ws_count;      // arrival tickets [B*H]; zero between calls
   int32_t ksplit;     // CTAs (one thread-block cluster) per (episode, head) of the cluster read
+  int32_t fused_ready;  // the fused pair is not written by the previous kernel on the stream
   float scale_log2;
   int* err;
   // NVFP4 fused pair (wam_action_attn_nvfp4; null otherwise): head-major codes [B, H, N, 64],

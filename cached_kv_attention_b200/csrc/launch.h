@@ -26,6 +26,9 @@ cudaError_t launch_action_nvfp4(const ActionArgs& a, cudaStream_t s);  // T % 12
 int action_tc_total_tiles(const ActionArgs& a);
 int action_tc_max_parts(const ActionArgs& a, int P, int G);
 size_t action_tc_workspace_bytes(int BH, int max_parts);
+// The aligned split of the 128-key reads (T % 128 == 0): sets kparts, G, P (the CTA count) and
+// max_parts; returns P.
+int action_aligned_plan(ActionArgs& a, int sms);
 // The action-read workspace starts with a fixed ticket region, so tickets never land on
 // partial data of an earlier call with another layout; partial slots follow it.
 constexpr size_t kTicketBytes = 65536;  // one int per (episode, head): B * H <= 16384

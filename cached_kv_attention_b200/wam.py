@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "wam_fuse_interval_kv": [lay, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                  ctypes.POINTER(f32), i32, i32, vp, vp, vp],
         "wam_action_attn": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp],
+        "wam_action_attn_ex": [lay, i32, vp, vp, i32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t,
+                               ctypes.c_uint32, vp],
         "wam_action_attn_workspace_size": [lay, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)],
         "wam_flow_euler_step": [i64, vp, vp, f32, vp],
         "wam_copy_frames": [lay, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp],
@@ -74,7 +76,7 @@ def _load() -> ctypes.CDLL:
         "wam_fused_to_nvfp4": [lay, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                vp, vp, ctypes.c_size_t, vp],
         "wam_action_attn_nvfp4": [lay, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, i32, vp,
-                                  ctypes.c_size_t, vp],
+                                  ctypes.c_size_t, ctypes.c_uint32, vp],
         "wam_video_prefill_kv_fuse_noalloc": [lay, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp,
                                               i32, f32, i32, i32, vp, vp, vp],
     }
@@ -99,7 +101,8 @@ def exported_names() -> list:
             "wam_debug_video_mask", "wam_device_error", "wam_last_error", "wam_version",
             "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size",
             "wam_copy_frames", "wam_debug_prefill_order", "wam_debug_wait_timeout",
-            "wam_nvfp4_workspace_size", "wam_fused_to_nvfp4", "wam_action_attn_nvfp4"]
+            "wam_nvfp4_workspace_size", "wam_fused_to_nvfp4", "wam_action_attn_nvfp4",
+            "wam_action_attn_ex"]
 
 
 def check(status: int) -> None:
@@ -232,16 +235,21 @@ def action_workspace(nbytes: int, device=None) -> Optional[torch.Tensor]:
     return ws
 
 
+ACTION_FUSED_READY = 1
+
+
 def action_attn(layout: VideoLayout, fused_k, fused_v, qa, ka, va, o, workspace=None,
-                stream=None) -> None:
+                stream=None, flags: int = 0) -> None:
+    """flags: ACTION_FUSED_READY when the fused pair is not written by the call issued right
+    before this one on the stream (see wam_action_attn_ex)."""
     n_act = qa.shape[1]
     if workspace is None:
         need = action_attn_workspace_size(layout, qa.dtype, n_act, fused_k is not None)
         workspace = action_workspace(need, qa.device.index)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    check(lib.wam_action_attn(layout.ref, _dtype(qa), _ptr(fused_k), _ptr(fused_v), n_act,
-                              _ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _ptr(workspace),
-                              ws_bytes, _stream(stream)))
+    check(lib.wam_action_attn_ex(layout.ref, _dtype(qa), _ptr(fused_k), _ptr(fused_v), n_act,
+                                 _ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _ptr(workspace),
+                                 ws_bytes, int(flags), _stream(stream)))
 
 
 def flow_euler_step(x, v, dsigma: float, stream=None) -> None:
@@ -316,7 +324,7 @@ def fused_to_nvfp4(layout: VideoLayout, fused, cache: Nvfp4Cache, stream=None) -
 
 
 def action_attn_nvfp4(layout: VideoLayout, cache: Nvfp4Cache, k_index: int, v_index: int, qa, ka,
-                      va, o, workspace=None, stream=None) -> None:
+                      va, o, workspace=None, stream=None, flags: int = 0) -> None:
     """The action read over the NVFP4 fused pair held in ``cache`` at tensors k_index / v_index."""
     n_act = qa.shape[1]
     if workspace is None:
@@ -328,7 +336,7 @@ def action_attn_nvfp4(layout: VideoLayout, cache: Nvfp4Cache, k_index: int, v_in
                                     sg + 4 * k_index, _ptr(cache.codes[v_index]),
                                     _ptr(cache.scales[v_index]), sg + 4 * v_index, n_act, _ptr(qa),
                                     _ptr(ka), _ptr(va), _ptr(o), _dtype(o), _ptr(workspace), ws_bytes,
-                                    _stream(stream)))
+                                    int(flags), _stream(stream)))
 
 
 def debug_wait_timeout(polls: int = 10000, stream=None) -> None:

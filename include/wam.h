@@ -169,6 +169,24 @@ wam_status wam_action_attn(const wam_video_layout* layout, wam_dtype dt,
                            wam_stream_t stream);
 
 /*
+ * wam_action_attn with flags (0: the same call).
+ *   WAM_ACTION_FUSED_READY  the caller guarantees that the fused pair is not written by the call
+ *                           issued on `stream` right before this one.  In the action loop the
+ *                           fused cache is read-only (the video stage completed it), and the
+ *                           read may then start loading its fused tiles while that call is still
+ *                           running (programmatic dependent launch); the action Q/K/V are read
+ *                           only after it has completed.  Used by the tensor-core read of 128-key
+ *                           tiles; the other paths ignore it.
+ * Unknown flag bits return WAM_ERR_INVALID_ARGUMENT.
+ */
+#define WAM_ACTION_FUSED_READY 1u
+wam_status wam_action_attn_ex(const wam_video_layout* layout, wam_dtype dt,
+                              const void* fused_k, const void* fused_v,
+                              int32_t n_act, const void* qa, const void* ka, const void* va,
+                              void* o, wam_dtype o_dt, void* workspace, size_t ws_bytes,
+                              uint32_t flags, wam_stream_t stream);
+
+/*
  * Bytes of workspace wam_action_attn needs for this layout on the current device
  * (with_video != 0: a layer that reads a fused pair).  Depends on the device's SM count.
  */
@@ -268,6 +286,8 @@ wam_status wam_fused_to_nvfp4(const wam_video_layout* layout, int32_t n, const v
  *   qa, ka, va   device bf16 [B, n_act, H, 128], 1 <= n_act <= 32; o device [B, n_act, H, 128]
  *                (o_dt WAM_F32 or WAM_BF16)
  *   workspace    as for wam_action_attn (wam_action_attn_workspace_size with dt = WAM_BF16)
+ *   flags        0 or WAM_ACTION_FUSED_READY (as for wam_action_attn_ex: the codes and scales
+ *                are not written by the call issued on `stream` right before this one)
  * T % 128 == 0.  The tiles are decoded exactly into fp16 and the matrix products run on fp16
  * operands with fp32 accumulation (the action Q/K/V are rounded to fp16 once: they must lie
  * within fp16's range, |x| < 65504); P is carried as two fp16 terms.
@@ -277,7 +297,7 @@ wam_status wam_action_attn_nvfp4(const wam_video_layout* layout, const void* k_c
                                  const void* v_scales, const float* v_sg, int32_t n_act,
                                  const void* qa, const void* ka, const void* va, void* o,
                                  wam_dtype o_dt, void* workspace, size_t ws_bytes,
-                                 wam_stream_t stream);
+                                 uint32_t flags, wam_stream_t stream);
 
 /* ---- host helpers (no GPU work) ---------------------------------------------------------- */
 

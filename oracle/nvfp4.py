@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and 
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.  The
 product path never imports, links or calls it, and it imports nothing from the product path.
 
-Source: "Long-WAM: 机器人操作模型的长历史..." (bloombook.cn), §三 (the LongLive-2.0 stack the
+Source: "Long-WAM: 机器人操作模型的长历史..." (bloombook.cn), §四 (the LongLive-2.0 stack the
 real-time loop builds on quantizes its KV cache block-wise to NVFP4, about 3.6x smaller), and
 "Long-WAM: Scaling the Context of World-Action Models | Summary", §4.2 (Long-WAM itself keeps
 its KV storage in BF16).  The pages name the format but not its parameters; this module takes

@@ -63,12 +63,15 @@ def test_nvfp4_encoder_ties_saturation_and_zeros():
     ties = [6.0, 2.5, 0.25, 0.75, 1.25, 1.75, 3.5, 5.0, -2.5, -0.25, -5.0, 0.1, -0.1, 4.5, 2.75, 0.0]
     x[0, 1, 0, :16] = torch.tensor(ties)
     x[0, 2, 1, :16] = torch.tensor([v * 4 for v in ties])     # scale 4: the same ties
-    x[0, 3, 1, 16:32] = 3000.0                                 # above the scale range: saturates
+    # amax 6.1875 rounds its block scale down to 1 (6.1875 / 6 = 1.03): 6.1875 saturates to 6
+    x[0, 3, 1, 16:32] = torch.tensor([6.1875] + [1.0] * 15)
     z = torch.zeros((B, F * T, H, D), dtype=torch.bfloat16)  # all zero: s_g = 0, every code 0
     cache = _check(lay, np.zeros((B, F), np.uint8), [x.cuda(), z.cuda()])
     assert cache.s_g[0].item() == 1.0 and cache.s_g[1].item() == 0.0
-    vals = Q.e2m1_decode(_unpack(cache.codes[0], cache.scales[0])[0][0, 1, 0, :16])
-    assert list(vals) == [6.0, 2.0, 0.0, 1.0, 1.0, 2.0, 4.0, 4.0, -2.0, 0.0, -4.0, 0.0, 0.0, 4.0, 3.0, 0.0]
+    codes, scales = _unpack(cache.codes[0], cache.scales[0])
+    assert list(Q.e2m1_decode(codes[0, 1, 0, :16])) == \
+        [6.0, 2.0, 0.0, 1.0, 1.0, 2.0, 4.0, 4.0, -2.0, 0.0, -4.0, 0.0, 0.0, 4.0, 3.0, 0.0]
+    assert Q.e4m3_decode(scales[0, 3, 1, 1]) == 1.0 and Q.e2m1_decode(codes[0, 3, 1, 16]) == 6.0
 
 
 def test_nvfp4_encoder_on_a_fused_pair_of_the_bench_layout():
@@ -99,7 +102,17 @@ READ_CASES = [
     (2, 3, 128, 5, [[1, 0, 0, 1, 0], [0, 0, 0, 0, 0]], 32, 1.0),   # logit std ~1: reference moves
     (1, 4, 256, 4, [[1, 0, 0, 0]], 1, 2.0),                         # peaky, one action token
     (3, 24, 128, 6, [[1, 1, 1, 0, 0, 0], [0] * 6, [1, 0, 0, 0, 0, 0]], 32, 1 / np.sqrt(128)),
+    (1, 24, 768, 4, [[1, 0, 0, 0]], 32, 1 / np.sqrt(128)),          # 768-token frames, 19 tiles
+    (1, 8, 128, 12, [[0] * 12], 32, 1 / np.sqrt(128)),              # long runs: the rings wrap
 ]
+
+
+def _report_non_finite(o, what):
+    bad = ~np.isfinite(o)
+    if bad.any():
+        idx = np.nonzero(bad)
+        print(f"{what}: {int(bad.sum())} non-finite outputs; episodes {np.unique(idx[0])}, "
+              f"queries {np.unique(idx[1])}, heads {np.unique(idx[2])}")
 
 
 @pytest.mark.parametrize("B,H,T,F,pad,n_act,std", READ_CASES)
@@ -119,6 +132,7 @@ def test_nvfp4_read_matches_oracle(B, H, T, F, pad, n_act, std):
     qk = Q.quantize_cache(to64(fk).astype(np.float32), pad, T)
     qv = Q.quantize_cache(to64(fv).astype(np.float32), pad, T)
     ref = Q.action_attention_nvfp4(to64(qa), to64(ka), to64(va), qk, qv, pad, T)
+    _report_non_finite(to64(o), "nvfp4 read")
     assert_parity(to64(o), ref, "bf16", "nvfp4 read")
 
 
@@ -146,6 +160,7 @@ def test_nvfp4_read_at_the_bench_layout_sampled_heads():
     qv = (full_v[0][:, :, heads], full_v[1][:, :, heads], full_v[2])
     ref = Q.action_attention_nvfp4(to64(qa[:, :, heads]), to64(ka[:, :, heads]), to64(va[:, :, heads]),
                                    qk, qv, pad, w.T)
+    _report_non_finite(to64(o), "nvfp4 read, bench layout")
     assert_parity(to64(o)[:, :, heads], ref, "bf16", "nvfp4 read, bench layout")
 
 

@@ -3,7 +3,7 @@
 Each pin checks the oracle against something other than itself: the formats' bit-field
 definitions, rounding written a second way (scale into the binade and round half to even),
 values that must survive a round trip exactly, the degenerate cases, and the storage ratio
-the pages quote ("Long-WAM: 机器人操作模型的长历史...", §三: NVFP4 KV cache about 3.6x smaller)."""
+the pages quote ("Long-WAM: 机器人操作模型的长历史...", §四: NVFP4 KV cache about 3.6x smaller)."""
 
 import numpy as np
 import pytest

@@ -1196,11 +1196,15 @@ __device__ __forceinline__ void bf16_to_f16_chunk(uint8_t* p) {
 __device__ __forceinline__ void bf16_tile_to_f16(uint8_t* tile, int bytes, int t, int nt) {
   for (int c = t; c < bytes / 16; c += nt) bf16_to_f16_chunk(tile + 16 * c);
 }
-// Two E2M1 codes of one byte (element 2i in the low nibble) -> an fp16 pair (element 2i low).
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t r;
-  asm("{ .reg .b8 c; cvt.u8.u32 c, %1; cvt.rn.f16x2.e2m1x2 %0, c; }" : "=r"(r) : "r"(byte));
-  return r;
+// Eight E2M1 codes of one word (element 2i in the low nibble of byte i) -> four fp16 pairs
+// (pair i = elements 2i, 2i + 1, the first in the low half): one unpack, four conversions.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t word, uint32_t (&out)[4]) {
+  asm("{ .reg .b8 b0, b1, b2, b3;\n"
+      " mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(word));
 }
 // An E4M3 code -> its value as an fp16 pair (both halves).
 __device__ __forceinline__ uint32_t e4m3_to_f16x2(uint32_t code) {
@@ -1227,11 +1231,10 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* raw, uint8_t* tile, 
     const int blk = 2 * q + half;
     const uint32_t s2 = e4m3_to_f16x2((sw >> (8 * (blk & 3))) & 0xFFu);
     uint32_t out[8];
+    e2m1x8_to_f16x2(cw[2 * half], *reinterpret_cast<uint32_t(*)[4]>(&out[0]));
+    e2m1x8_to_f16x2(cw[2 * half + 1], *reinterpret_cast<uint32_t(*)[4]>(&out[4]));
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t word = cw[2 * half + (e >> 2)];
-      out[e] = mul_f16x2(e2m1x2_to_f16x2((word >> (8 * (e & 3))) & 0xFFu), s2);
-    }
+    for (int e = 0; e < 8; ++e) out[e] = mul_f16x2(out[e], s2);
     const int ch0 = 2 * blk;  // 8-element chunks 2 blk and 2 blk + 1 of the row
     *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0)) = make_uint4(out[0], out[1], out[2], out[3]);
     *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0 + 8)) = make_uint4(out[4], out[5], out[6], out[7]);

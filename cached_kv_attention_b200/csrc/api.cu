@@ -636,6 +636,25 @@ wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin,
                      "wam_debug_video_mask");
 }
 
+wam_status wam_debug_action_plan(const wam_video_layout* layout, int32_t n_sms, int32_t* kparts,
+                                 int32_t* n_ctas, int32_t* max_parts) {
+  Geo g;
+  WAM_CHECK(check_layout(layout, g));
+  if (!kparts || !n_ctas || !max_parts)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "an output pointer is NULL");
+  if (n_sms < 1) return fail(WAM_ERR_INVALID_ARGUMENT, "n_sms must be >= 1");
+  if (g.T % 128 != 0)
+    return fail(WAM_ERR_INVALID_ARGUMENT, "T = %d is not a multiple of 128", g.T);
+  static thread_local wam::ActionArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = g.B, a.H = g.H, a.T = g.T, a.F = g.F, a.with_video = 1;
+  fill_vlists(g, a.fl);
+  *n_ctas = wam::action_aligned_plan(a, n_sms);
+  *max_parts = a.max_parts;
+  for (int b = 0; b < g.B; ++b) kparts[b] = a.kparts[b];
+  return ok();
+}
+
 wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
                                    int32_t n_sms, int32_t* episode, int32_t* frame,
                                    int32_t* n_key_frames, int32_t* n_items) {

@@ -19,6 +19,7 @@ __all__ = [
     "video_prefill_kv_fuse_noalloc", "NOALLOC_FUSE_ACC_ELEMS", "action_attn_workspace_size",
     "action_workspace", "debug_prefill_order", "debug_wait_timeout",
     "nvfp4_workspace_size", "fused_to_nvfp4", "Nvfp4Cache", "action_attn_nvfp4",
+    "debug_action_plan", "ACTION_FUSED_READY",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwam.so")
@@ -72,6 +73,8 @@ def _load() -> ctypes.CDLL:
                                     ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "wam_device_error": [i32],
         "wam_debug_wait_timeout": [i32, vp],
+        "wam_debug_action_plan": [lay, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                  ctypes.POINTER(i32)],
         "wam_nvfp4_workspace_size": [i32, ctypes.POINTER(ctypes.c_size_t)],
         "wam_fused_to_nvfp4": [lay, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                vp, vp, ctypes.c_size_t, vp],
@@ -102,7 +105,7 @@ def exported_names() -> list:
             "wam_video_prefill_kv_fuse_noalloc", "wam_action_attn_workspace_size",
             "wam_copy_frames", "wam_debug_prefill_order", "wam_debug_wait_timeout",
             "wam_nvfp4_workspace_size", "wam_fused_to_nvfp4", "wam_action_attn_nvfp4",
-            "wam_action_attn_ex"]
+            "wam_action_attn_ex", "wam_debug_action_plan"]
 
 
 def check(status: int) -> None:
@@ -343,6 +346,16 @@ def debug_wait_timeout(polls: int = 10000, stream=None) -> None:
     """Launch a wait that gives up after ``polls`` polls and records WAM_ERR_TIMEOUT in the
     device error word (read it with ``device_error``)."""
     check(lib.wam_debug_wait_timeout(int(polls), _stream(stream)))
+
+
+def debug_action_plan(layout: VideoLayout, n_sms: int):
+    """The NVFP4 read's work split on a device of n_sms SMs (host only): (kparts [B] int32,
+    CTAs launched, largest part count)."""
+    k = np.zeros(layout.B, dtype=np.int32)
+    n, mx = ctypes.c_int32(0), ctypes.c_int32(0)
+    check(lib.wam_debug_action_plan(layout.ref, int(n_sms), k.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                    ctypes.byref(n), ctypes.byref(mx)))
+    return k, n.value, mx.value
 
 
 def device_error(clear: bool = True) -> None:

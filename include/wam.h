@@ -348,6 +348,18 @@ wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_beg
 wam_status wam_debug_wait_timeout(int32_t polls, wam_stream_t stream);
 
 /*
+ * The work split of the NVFP4 read (T % 128 == 0) on a device with n_sms SMs; host only, no GPU
+ * needed.  Every head of episode b is cut into kparts[b] parts at the same tile boundaries:
+ * part r of k reads the video tiles [1 + r nv / k, 1 + (r + 1) nv / k) of the (episode, head)
+ * (nv = 128-key tiles of the episode's valid frames) and part 0 also the action tile.  The
+ * smallest part size is chosen for which all B * H * k CTAs fit in n_sms (one part per head if
+ * none does).
+ *   kparts host int32 [B]; *n_ctas the CTAs launched; *max_parts the largest kparts[b].
+ */
+wam_status wam_debug_action_plan(const wam_video_layout* layout, int32_t n_sms, int32_t* kparts,
+                                 int32_t* n_ctas, int32_t* max_parts);
+
+/*
  * Synchronise the current device and report its error word: WAM_OK, or WAM_ERR_TIMEOUT when
  * a kernel's bounded wait on an mbarrier gave up (the kernel then skipped its remaining work
  * and returned without faulting).  clear != 0 resets the word.  Host-blocking.

@@ -467,13 +467,18 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
 // Work split: one thread-block cluster of k <= 8 CTAs per (episode, head); CTA r of the
 // cluster streams the r-th of k contiguous slices of the (episode, head)'s tiles (the action
 // tile first, then the valid frames' tiles).  The k partials (O, m, l) meet in distributed
-// shared memory: after a cluster barrier CTA r merges query rows [r n_act / k, (r+1) n_act / k)
-// by reading its peers' partials, so no partial leaves the chip.
+// shared memory and never leave the chip: CTA r owns query rows [r n_act / k, (r+1) n_act / k).
+// Once its MMAs are done its K/V stage buffers are free, and it tells its peers so (a release
+// arrive on each peer's barrier); every CTA then writes its partial rows straight into their
+// owners' stage buffers (shared::cluster stores, released by one arrive per owner) and merges
+// its own rows from local memory.  One one-way hop follows the slowest slice, and no CTA waits
+// on another before leaving.
 // Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-5 softmax (TMEM lane quarters 2, 3, 0, 1).
 namespace um {
 constexpr int kKeys = 128;
 constexpr int kTile = kKeys * 128 * 2;   // one of K or V: 32 KB
-constexpr int kStages = 3;
+constexpr int kKStages = 3;            // K ring
+constexpr int kVStages = 2;            // V ring (its tiles are needed one S^T later than K's)
 constexpr int kQ = 32 * 128 * 2;         // 8 KB
 constexpr int kP = kKeys * 128;          // P^T: 128 keys x (32 P_hi + 32 P_lo) bf16 = 16 KB
 constexpr int kThreads = 6 * 32;
@@ -481,14 +486,26 @@ constexpr uint32_t kTmemCols = 128;      // S^T buffers at columns 0 and 32, O^T
 constexpr float kLazy = 16.f;            // reference headroom (log2 units): P <= 2^16
 constexpr int kMaxSplit = 8;             // portable cluster size
 struct Bars {
-  uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
+  uint64_t kfull[kKStages], kempty[kKStages], vfull[kVStages], vempty[kVStages];
   uint64_t qfull, sfull[2], sfree[2], pfull, pfree, ofull, done;
   uint32_t tmem_base;
   int abort;
   float red[4][32];
+  // the merge over the cluster: completes once every peer's partial rows for this CTA have landed
+  uint64_t rx_full;
   float part_m[32], part_l[32];  // this CTA's partial: reference max and row sum per query
+  // where row q of this CTA's partial goes: the owner's rank, and the byte offsets of its O row
+  // and of its (m, l) pair in the owner's receive region
+  int row_owner[32], row_off[32], ml_off[32];
 };
-constexpr int kSmemBytes = 1024 + kQ + kStages * 2 * kTile + kP + int(sizeof(Bars)) + 64;
+// Receive region of the merge: k slots (one per rank of the cluster) of this CTA's query rows,
+// [slot][row][128 floats] then the (m, l) pairs [slot][row]; k x ceil(32 / k) x 520 bytes at most.
+constexpr int kRx = 19 * 1024;
+constexpr int rx_bytes(int k) { return k * ((32 + k - 1) / k) * 520; }
+static_assert(rx_bytes(2) <= kRx && rx_bytes(3) <= kRx && rx_bytes(4) <= kRx && rx_bytes(5) <= kRx &&
+                  rx_bytes(6) <= kRx && rx_bytes(7) <= kRx && rx_bytes(8) <= kRx,
+              "receive region");
+constexpr int kSmemBytes = 1024 + kQ + (kKStages + kVStages) * kTile + kP + kRx + int(sizeof(Bars)) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(32 * 128 * 4 == kP, "the partial O [32][128] fp32 reuses the P^T buffer");
 
@@ -512,23 +529,42 @@ __device__ __forceinline__ bool softmax_any(bool v) {
       : "memory");
   return r != 0;
 }
-// A float in CTA `peer`'s shared memory at the offset of `local` in this CTA's.
-__device__ __forceinline__ float ld_peer(const float* local, uint32_t peer) {
+// The address, in the cluster's shared window, of the byte at the offset of `local` in CTA
+// `peer`'s shared memory.
+__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t peer) {
   uint32_t pa;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(pa) : "r"(smem_u32(local)), "r"(peer));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(pa) : "memory");
-  return v;
+  return pa;
 }
-__device__ __forceinline__ float4 ld_peer4(const float* local, uint32_t peer) {
-  uint32_t pa;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(pa) : "r"(smem_u32(local)), "r"(peer));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(pa)
+// Asynchronous stores into a peer's shared memory (cluster window addresses), each counted in
+// bytes on the barrier at `bar` in that peer.
+__device__ __forceinline__ void st_async4(uint32_t pa, float4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(pa),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
                : "memory");
-  return v;
+}
+__device__ __forceinline__ void st_async2(uint32_t pa, float x, float y, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(pa), "f"(x),
+               "f"(y), "r"(bar)
+               : "memory");
+}
+// A bounded wait on a local barrier that peers arrive on, acquiring their writes at cluster scope.
+// It does not give up early when this CTA has aborted: peers may still write into this CTA's
+// shared memory until they have arrived, and every peer runs the exchange whatever happened to
+// it, so only the spin limit ends the wait (and then reports a timeout).
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  *abort = 1;
+  return false;
 }
 // After the call lane q holds the max (or sum) over the warp's lanes of v[q]; v is clobbered.
 template <bool kMax>
@@ -554,10 +590,11 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  auto sK = [&](int st) { return base + kQ + st * 2 * kTile; };
-  auto sV = [&](int st) { return base + kQ + st * 2 * kTile + kTile; };
-  uint8_t* sP = base + kQ + kStages * 2 * kTile;
-  um::Bars& bars = *reinterpret_cast<um::Bars*>(sP + kP);
+  auto sK = [&](int st) { return base + kQ + st * kTile; };
+  auto sV = [&](int st) { return base + kQ + (kKStages + st) * kTile; };
+  uint8_t* sP = base + kQ + (kKStages + kVStages) * kTile;
+  uint8_t* rx = sP + kP;  // receive region of the cluster merge (k > 1)
+  um::Bars& bars = *reinterpret_cast<um::Bars*>(rx + kRx);
   volatile int* abort = &bars.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
@@ -571,9 +608,11 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   const int t0 = rank * nb / k, t1 = (rank + 1) * nb / k, n = t1 - t0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&bars.kfull[i], 1);
       mbar_init(&bars.kempty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&bars.vfull[i], 1);
       mbar_init(&bars.vempty[i], 1);
     }
@@ -587,6 +626,22 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
     mbar_init(&bars.ofull, 1);
     mbar_init(&bars.done, 1);
     bars.abort = 0;
+    if (k > 1) {
+      // armed now with every byte the k - 1 peers will send (their rows of this CTA's range),
+      // before the cluster barrier below lets any of them send
+      const int rows = (rank + 1) * a.n_act / k - rank * a.n_act / k;
+      mbar_init(&bars.rx_full, 1);
+      mbar_arrive_expect_tx(&bars.rx_full, uint32_t((k - 1) * rows * 520));
+      // row q of this CTA's partial goes to slot `rank` of its owner's receive region
+      for (int r = 0; r < k; ++r) {
+        const int r0 = r * a.n_act / k, r1 = (r + 1) * a.n_act / k, rows = r1 - r0;
+        for (int q = r0; q < r1; ++q) {
+          bars.row_owner[q] = r;
+          bars.row_off[q] = (rank * rows + (q - r0)) * 512;
+          bars.ml_off[q] = k * rows * 512 + (rank * rows + (q - r0)) * 8;
+        }
+      }
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -596,6 +651,10 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   tc05::fence_before_sync();
   __syncthreads();
   tc05::fence_after_sync();
+  // every CTA of the cluster has initialised (and armed) its barriers once this phase completes;
+  // each thread waits on it before its first access to a peer (the softmax warps) or before
+  // leaving
+  if (k > 1) asm volatile("barrier.cluster.arrive.release;" ::: "memory");
   const uint32_t tmem = bars.tmem_base;
   auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
     const int t = t0 + i;
@@ -607,24 +666,23 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
     }
   };
-  auto load_kv = [&](int i) {  // K and V of the slice's tile i into stage i % kStages
-    const int st = i % kStages;
+  auto load_kv = [&](int i) {  // K and V of the slice's tile i (i < both ring sizes)
     const CUtensorMap* mp;
     int tok;
     tile_src(i, false, mp, tok);
-    mbar_arrive_expect_tx(&bars.kfull[st], kTile);
-    tma_load_4d(sK(st), mp, &bars.kfull[st], 0, h, tok, b);
-    tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, h, tok, b);
+    mbar_arrive_expect_tx(&bars.kfull[i], kTile);
+    tma_load_4d(sK(i), mp, &bars.kfull[i], 0, h, tok, b);
+    tma_load_4d(sK(i) + kTile / 2, mp, &bars.kfull[i], 64, h, tok, b);
     tile_src(i, true, mp, tok);
-    mbar_arrive_expect_tx(&bars.vfull[st], kTile);
-    tma_load_4d(sV(st), mp, &bars.vfull[st], 0, h, tok, b);
-    tma_load_4d(sV(st) + kTile / 2, mp, &bars.vfull[st], 64, h, tok, b);
+    mbar_arrive_expect_tx(&bars.vfull[i], kTile);
+    tma_load_4d(sV(i), mp, &bars.vfull[i], 0, h, tok, b);
+    tma_load_4d(sV(i) + kTile / 2, mp, &bars.vfull[i], 64, h, tok, b);
   };
   // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
   // the stream may still be finishing (programmatic dependent launch).  With a.fused_ready the
   // caller guarantees that kernel does not write the fused pair, so the slice's first fused
   // tiles are requested now; the action tile and Q wait for it.
-  const int n_pre = n < kStages ? n : kStages;
+  const int n_pre = n < kVStages ? n : kVStages;  // kVStages <= kKStages
   uint32_t pre = 0;  // bit i: tile i requested before the dependency wait
   if (threadIdx.x == 0) {
     prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
@@ -638,8 +696,9 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // K and V stream through separate 3-stage rings: a K stage is refilled as soon as its S^T
-    // MMA has completed, a V stage once its P V has.  The two sequences advance independently.
+    // K and V stream through separate rings (3 and 2 stages): a K stage is refilled as soon as
+    // its S^T MMA has completed, a V stage once its P V has.  The two sequences advance
+    // independently.
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(&bars.qfull, kQ);
       tma_load_4d(sQ, &maps.q, &bars.qfull, 0, h, 0, b);
@@ -649,8 +708,9 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       int nk = n_pre, nv = n_pre;
       for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
         if ((it & 31u) == 31u && *abort) break;
-        if (nk < n && (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1))) {
-          const int st = nk % kStages;
+        const int nk0 = nk, nv0 = nv;
+        if (nk < n && (nk < kKStages || mbar_test_wait(&bars.kempty[nk % kKStages], ((nk / kKStages) - 1) & 1))) {
+          const int st = nk % kKStages;
           const CUtensorMap* mp;
           int tok;
           tile_src(nk, false, mp, tok);
@@ -659,8 +719,8 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
           tma_load_4d(sK(st) + kTile / 2, mp, &bars.kfull[st], 64, h, tok, b);
           ++nk;
         }
-        if (nv < n && (nv < kStages || mbar_test_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))) {
-          const int st = nv % kStages;
+        if (nv < n && (nv < kVStages || mbar_test_wait(&bars.vempty[nv % kVStages], ((nv / kVStages) - 1) & 1))) {
+          const int st = nv % kVStages;
           const CUtensorMap* mp;
           int tok;
           tile_src(nv, true, mp, tok);
@@ -669,11 +729,12 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
           tma_load_4d(sV(st) + kTile / 2, mp, &bars.vfull[st], 64, h, tok, b);
           ++nv;
         }
+        if (nk == nk0 && nv == nv0) poll_pause();
       }
       if (nk < n || nv < n) *abort = 1;
       // Loads still in flight land before the CTA leaves (only after an abort can any be).
-      for (int i = (nk > kStages ? nk - kStages : 0); i < nk; ++i) mbar_wait(&bars.kfull[i % kStages], (i / kStages) & 1);
-      for (int i = (nv > kStages ? nv - kStages : 0); i < nv; ++i) mbar_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
+      for (int i = (nk > kKStages ? nk - kKStages : 0); i < nk; ++i) mbar_wait(&bars.kfull[i % kKStages], (i / kKStages) & 1);
+      for (int i = (nv > kVStages ? nv - kVStages : 0); i < nv; ++i) mbar_wait(&bars.vfull[i % kVStages], (i / kVStages) & 1);
       mbar_wait(&bars.qfull, 0);
     }
   } else if (warp == 1) {
@@ -685,12 +746,12 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       const uint32_t idS = tc05::idesc_bf16_f32(128, 32, false, false);
       const uint32_t idO = tc05::idesc_bf16_f32(128, 64, true, true);
       auto s_ready = [&](int j) {
-        return mbar_test_wait(&bars.kfull[j % kStages], (j / kStages) & 1) &&
+        return mbar_test_wait(&bars.kfull[j % kKStages], (j / kKStages) & 1) &&
                (j > 0 || mbar_test_wait(&bars.qfull, 0)) &&
                (j < 2 || mbar_test_wait(&bars.sfree[j & 1], ((j >> 1) - 1) & 1));
       };
       auto issue_S = [&](int j) {
-        const int st = j % kStages;
+        const int st = j % kKStages;
         tc05::fence_after_sync();
         const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ);
 #pragma unroll
@@ -707,18 +768,20 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       for (int i = 0; ok && i < n; ++i) {
         bool p_ready = false, v_ready = false;
         for (uint32_t it = 0;; ++it) {
+          const int ns0 = ns;
           if (ns < n && ns <= i + 2 && s_ready(ns)) issue_S(ns++);
           if (ns > i) {
-            v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
+            v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kVStages], (i / kVStages) & 1);
             p_ready = v_ready && mbar_test_wait(&bars.pfull, i & 1);
             if (p_ready) break;
           }
+          if (ns == ns0) poll_pause();
           if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
           if ((it & 31u) == 31u && *abort) { ok = false; break; }
         }
         if (!ok) break;
         tc05::fence_after_sync();
-        const int st = i % kStages;
+        const int st = i % kVStages;
         const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -827,7 +890,18 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.pfull);
     }
-    // ---- slice done: O^T column d = L of this thread and the row sums over all 128 keys
+    // ---- slice done: the row sums over all 128 keys (while the last P V runs), then O^T
+    // column d = L of this thread
+    {
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = l[q];
+      bars.red[wr][lane] = reduce_scatter32<false>(v, lane);
+    }
+    softmax_sync();
+    float lt[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
     float o[32];
 #pragma unroll
     for (int q = 0; q < 32; ++q) o[q] = 0.f;
@@ -843,16 +917,6 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
         for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
       }
     }
-    {
-      float v[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = l[q];
-      bars.red[wr][lane] = reduce_scatter32<false>(v, lane);
-    }
-    softmax_sync();
-    float lt[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
     if (k == 1) {
       // the whole (b, h) in this CTA: O = O^T / l
 #pragma unroll
@@ -864,8 +928,11 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
         else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
       }
     } else {
-      // the partial into this CTA's shared memory (the P^T buffer is free: every P V is done)
-      float* part = reinterpret_cast<float*>(sP);  // [32 queries][128]
+      // ---- the merge over the cluster.  Row q of this CTA's partial goes to slot `rank` of the
+      // receive region of the row's owner, 16 bytes per st.async counted on the owner's rx_full
+      // (armed at the start with every byte it will receive); this CTA's own rows are copied
+      // locally.  The P^T buffer (every P V is done) stages the partial as [32 queries][128].
+      float* part = reinterpret_cast<float*>(sP);
 #pragma unroll
       for (int q = 0; q < 32; ++q) part[q * 128 + L] = o[q];
       if (wr == 0) {
@@ -876,86 +943,69 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
         bars.part_m[lane] = mm;
         bars.part_l[lane] = ll;
       }
-    }
-  }
-
-  if (k > 1) {
-    // ---------------------------------------------------------------- merge over the cluster
-    __syncwarp();
-    // Every CTA's partial is in its shared memory after this barrier.  Only the softmax warps
-    // wrote it, so only they arrive with release semantics: a release arrive of the TMA and MMA
-    // warps measured ~2 us on B200 and held up the whole cluster.
-    if (warp >= 2)
-      asm volatile("barrier.cluster.arrive.release;" ::: "memory");
-    else
-      asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-    {
-      // One query row per half-warp (all 6 warps; at most 2 rows each, a rank has <= 16), 8
-      // columns per lane: every peer's (m, l) and its 32 bytes of the partial row are loaded
-      // before any is used (one round trip per row).  The CTA arrives on the closing cluster
-      // barrier once its peer reads are done and only then stores O.  That arrive is relaxed:
-      // it orders nothing, it only says that this thread's peer loads, whose values it has
-      // already consumed, can no longer touch a peer's shared memory.
-      const int hw = threadIdx.x >> 4, c0 = 8 * (threadIdx.x & 15);
-      const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k;
-      const float* part = reinterpret_cast<const float*>(sP);
-      float val[2][8];
+      softmax_sync();
+      asm volatile("barrier.cluster.wait.acquire;" ::: "memory");  // every owner has armed rx_full
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int q = r0 + hw + rr * (um::kThreads / 16);
-        if (q >= r1) continue;
+      for (int it = 0; it < 8; ++it) {  // chunk c: 16 bytes of row c / 32 (n_act <= 32 rows)
+        const int c = L + 128 * it, q = c >> 5, ch = c & 31;
+        if (q >= a.n_act) continue;
+        const int r = bars.row_owner[q];
+        const float4 v = *reinterpret_cast<const float4*>(part + q * 128 + 4 * ch);
+        uint8_t* dst = rx + bars.row_off[q] + 16 * ch;
+        if (r == rank) *reinterpret_cast<float4*>(dst) = v;
+        else st_async4(peer_addr(dst, uint32_t(r)), v, peer_addr(&bars.rx_full, uint32_t(r)));
+      }
+      if (L < a.n_act) {
+        const int r = bars.row_owner[L];
+        uint8_t* dst = rx + bars.ml_off[L];
+        if (r == rank) *reinterpret_cast<float2*>(dst) = make_float2(bars.part_m[L], bars.part_l[L]);
+        else st_async2(peer_addr(dst, uint32_t(r)), bars.part_m[L], bars.part_l[L], peer_addr(&bars.rx_full, uint32_t(r)));
+      }
+      wait_cluster(&bars.rx_full, 0, abort);  // every peer's rows for this CTA have landed
+      softmax_sync();                         // and this CTA's own copies
+      // merge rows [r0, r1): warp wr takes rows wr, wr + 4, ...; lane the columns 4 lane .. + 3
+      const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k, rows = r1 - r0;
+      const float* rxo = reinterpret_cast<const float*>(rx);
+      const float* rml = reinterpret_cast<const float*>(rx + k * rows * 512);
+      for (int j = wr; j < rows; j += 4) {
+        // every slot's (m, l) and 16 bytes of its row first: one round of shared loads
         float pm[kMaxSplit], pl_[kMaxSplit];
-        float4 pa[kMaxSplit], pb[kMaxSplit];
+        float4 px[kMaxSplit];
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p) {
           if (p >= k) continue;
-          pm[p] = ld_peer(&bars.part_m[q], uint32_t(p));
-          pl_[p] = ld_peer(&bars.part_l[q], uint32_t(p));
-          pa[p] = ld_peer4(part + q * 128 + c0, uint32_t(p));
-          pb[p] = ld_peer4(part + q * 128 + c0 + 4, uint32_t(p));
+          pm[p] = rml[2 * (p * rows + j)], pl_[p] = rml[2 * (p * rows + j) + 1];
+          px[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + 4 * lane);
         }
         float M = -INFINITY;
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p)
           if (p < k) M = fmaxf(M, pm[p]);
         const float Mu = M == -INFINITY ? 0.f : M;
-        float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
+        float num[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p) {
           if (p >= k) continue;
           const float wgt = exp2f(pm[p] - Mu);
           den = fmaf(wgt, pl_[p], den);
-          num[0] = fmaf(wgt, pa[p].x, num[0]), num[1] = fmaf(wgt, pa[p].y, num[1]);
-          num[2] = fmaf(wgt, pa[p].z, num[2]), num[3] = fmaf(wgt, pa[p].w, num[3]);
-          num[4] = fmaf(wgt, pb[p].x, num[4]), num[5] = fmaf(wgt, pb[p].y, num[5]);
-          num[6] = fmaf(wgt, pb[p].z, num[6]), num[7] = fmaf(wgt, pb[p].w, num[7]);
+          num[0] = fmaf(wgt, px[p].x, num[0]), num[1] = fmaf(wgt, px[p].y, num[1]);
+          num[2] = fmaf(wgt, px[p].z, num[2]), num[3] = fmaf(wgt, px[p].w, num[3]);
         }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        float val[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) val[rr][e] = den > 0.f ? num[e] / den : 0.f;
+        for (int e = 0; e < 4; ++e) val[e] = num[e] * inv;
+        const int64_t off = ((int64_t(b) * a.n_act + r0 + j) * a.H + h) * 128 + 4 * lane;
+        if (a.o_f32)
+          *reinterpret_cast<float4*>(static_cast<float*>(a.o) + off) = make_float4(val[0], val[1], val[2], val[3]);
+        else
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + off) =
+              make_uint2(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]));
       }
-      __syncwarp();
-      asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");  // peer reads done
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int q = r0 + hw + rr * (um::kThreads / 16);
-        if (q >= r1) continue;
-        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + c0;
-        if (a.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
-          dst[0] = make_float4(val[rr][0], val[rr][1], val[rr][2], val[rr][3]);
-          dst[1] = make_float4(val[rr][4], val[rr][5], val[rr][6], val[rr][7]);
-        } else {
-          uint4 u;
-          u.x = pack_bf16(val[rr][0], val[rr][1]), u.y = pack_bf16(val[rr][2], val[rr][3]);
-          u.z = pack_bf16(val[rr][4], val[rr][5]), u.w = pack_bf16(val[rr][6], val[rr][7]);
-          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off) = u;
-        }
-      }
-      // no CTA leaves while a peer may still read its shared memory
-      asm volatile("barrier.cluster.wait;" ::: "memory");
     }
   }
+  // the producer and MMA warps close their phase of the cluster barrier before leaving
+  if (k > 1 && warp < 2) asm volatile("barrier.cluster.wait;" ::: "memory");
 
   // ---------------------------------------------------------------- teardown
   __syncwarp();
@@ -1138,13 +1188,20 @@ namespace fq {
 constexpr int kKeys = 128;
 constexpr int kTile = kKeys * 128 * 2;   // one fp16 K or V tile: 32 KB
 constexpr int kStages = 2;               // fp16 K and V tiles
-constexpr int kRaw = 3;                  // raw slots for K and for V
+constexpr int kRaw = 2;                  // raw slots for K and for V
 constexpr int kCodes = kKeys * 64;       // codes of one tile: 8 KB
 constexpr int kScales = kKeys * 8;       // E4M3 scales of one tile: 1 KB
 constexpr int kRawBytes = kCodes + kScales;
 constexpr int kQ = 32 * 128 * 2;
 constexpr int kP = kKeys * 128;
-constexpr int kThreads = 8 * 32;
+// Warpgroups: 0 = producer (warp 0), MMA issuer (warp 1), two idle warps; 1 = softmax; 2 = K (and
+// Q) converters; 3 = V converters.  The softmax warpgroup holds 32 running maxima and sums per
+// thread, so the registers are split unevenly (setmaxnreg); the shares add up to the block's
+// launch allocation of 128 per thread.
+constexpr int kThreads = 16 * 32;
+constexpr int kConvWarps = 4;
+constexpr uint32_t kRegsCtl = 80, kRegsSoftmax = 256, kRegsConv = 88, kRegsLaunch = 128;
+static_assert(kRegsCtl + kRegsSoftmax + 2 * kRegsConv == 4 * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;      // S^T 0, 32; O^T video 64 + 64 p; O^T action 192 + 64 p
 constexpr float kLazy = 15.f;            // P <= 2^15 < 65504
 struct Bars {
@@ -1152,7 +1209,7 @@ struct Bars {
   uint64_t kland[kStages], kfull[kStages], kempty[kStages];
   uint64_t vland[kStages], vfull[kStages], vempty[kStages];
   uint64_t rkfull[kRaw], rkfree[kRaw], rvfull[kRaw], rvfree[kRaw];
-  uint64_t sfull[2], sfree[2], pfull, pfree, ofull[2], ofree[2], done;
+  uint64_t sfull[2], sfree[2], pfull[2], pfree[2], ofull[2], ofree[2], done;
   uint64_t mfull;
   uint32_t tmem_base;
   int abort;
@@ -1161,7 +1218,7 @@ struct Bars {
   float red[4][32];
 };
 constexpr int kSmemBytes =
-    1024 + 2 * kQ + kStages * 2 * kTile + 2 * kRaw * kRawBytes + kP + int(sizeof(Bars)) + 64;
+    1024 + 2 * kQ + kStages * 2 * kTile + 2 * kRaw * kRawBytes + 2 * kP + int(sizeof(Bars)) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory");
 // partials the fp16 K/V stages and the raw rings (contiguous) hold for the merge
 constexpr int kStageParts = (kStages * 2 * kTile + 2 * kRaw * kRawBytes - 128) / (kSlotFloats * 4 + 128);
@@ -1217,19 +1274,38 @@ __device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-// 16 bytes of codes (32 elements: blocks 2 q and 2 q + 1 of key row r) of a raw tile decoded into
-// the fp16 tile.  A warp decodes 8 rows at a time, lane t taking row 8 i + t / 4 and chunk t % 4,
-// so each load instruction reads 512 contiguous bytes of codes (no bank conflict) and the rows'
-// 8 scale bytes are shared by 4 lanes.
-__device__ __forceinline__ void decode_chunk(const uint8_t* raw, uint8_t* tile, int r, int q) {
-  const uint4 c = *reinterpret_cast<const uint4*>(raw + r * 64 + q * 16);
-  const uint2 sc = *reinterpret_cast<const uint2*>(raw + kCodes + r * 8);
-  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-  const uint32_t sw = q < 2 ? sc.x : sc.y;  // scale bytes 2 q and 2 q + 1
+// 16 bytes of codes (32 elements: blocks 2 q and 2 q + 1 of key row r) of a raw tile and the 4
+// scale bytes of those blocks.  A warp instruction covers 8 rows x 4 chunks; 16-byte accesses
+// are served by quarter-warps of 8 lanes, so the lanes of each quarter take rows and chunks that
+// fall in 8 different 16-byte bank groups both for the loads (row r, chunk q of 64-byte code
+// rows: group 4 (r & 1) + q) and for the stores into the swizzled fp16 tile (chunks 0 and 4 of
+// a 64-column half XOR r & 7): quarter p takes rows 4 (p / 2) .. +3, pairs of rows with chunks
+// {0, 1} and {2, 3}, swapped for odd p.
+__device__ __forceinline__ int chunk_row(int lane) {
+  const int p = lane >> 3, k = lane & 7;
+  return 4 * (p >> 1) + 2 * (k >> 2) + (k & 1);
+}
+__device__ __forceinline__ int chunk_q(int lane) {
+  const int p = lane >> 3, k = lane & 7;
+  return (((k >> 1) & 1) | ((k >> 2) << 1)) ^ ((p & 1) << 1);
+}
+struct RawChunk {
+  uint4 c;
+  uint32_t sw;
+};
+__device__ __forceinline__ RawChunk load_chunk(const uint8_t* raw, int r, int q) {
+  RawChunk x;
+  x.c = *reinterpret_cast<const uint4*>(raw + r * 64 + q * 16);
+  x.sw = *reinterpret_cast<const uint32_t*>(raw + kCodes + r * 8 + (q >> 1) * 4);
+  return x;
+}
+// The chunk decoded (code value times its block's scale, in fp16) into the swizzled fp16 tile.
+__device__ __forceinline__ void store_chunk(const RawChunk& x, uint8_t* tile, int r, int q) {
+  const uint32_t cw[4] = {x.c.x, x.c.y, x.c.z, x.c.w};
 #pragma unroll
   for (int half = 0; half < 2; ++half) {  // one 16-element block, two 8-element chunks
     const int blk = 2 * q + half;
-    const uint32_t s2 = e4m3_to_f16x2((sw >> (8 * (blk & 3))) & 0xFFu);
+    const uint32_t s2 = e4m3_to_f16x2((x.sw >> (8 * (blk & 3))) & 0xFFu);
     uint32_t out[8];
     e2m1x8_to_f16x2(cw[2 * half], *reinterpret_cast<uint32_t(*)[4]>(&out[0]));
     e2m1x8_to_f16x2(cw[2 * half + 1], *reinterpret_cast<uint32_t(*)[4]>(&out[4]));
@@ -1239,6 +1315,24 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* raw, uint8_t* tile, 
     *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0)) = make_uint4(out[0], out[1], out[2], out[3]);
     *reinterpret_cast<uint4*>(tile + swz128<128>(r, 8 * ch0 + 8)) = make_uint4(out[4], out[5], out[6], out[7]);
   }
+}
+// The row groups g, g + 4, g + 8, g + 12 (of 16 groups of 8 rows) of a raw tile decoded by warp g of
+// the four converter warps: all loads first, so that the warp has four chunks in flight.
+__device__ __forceinline__ void decode_rows(const uint8_t* raw, uint8_t* tile, int g, int lane) {
+  const int rr = chunk_row(lane), q = chunk_q(lane);
+  RawChunk x[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x[j] = load_chunk(raw, 8 * (g + 4 * j) + rr, q);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) store_chunk(x[j], tile, 8 * (g + 4 * j) + rr, q);
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 }  // namespace fq
 
@@ -1252,8 +1346,10 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   auto sV = [&](int st) { return base + 2 * kQ + st * 2 * kTile + kTile; };
   auto rK = [&](int sl) { return base + 2 * kQ + kStages * 2 * kTile + sl * kRawBytes; };
   auto rV = [&](int sl) { return base + 2 * kQ + kStages * 2 * kTile + (kRaw + sl) * kRawBytes; };
-  uint8_t* sP = base + 2 * kQ + kStages * 2 * kTile + 2 * kRaw * kRawBytes;
-  fq::Bars& bars = *reinterpret_cast<fq::Bars*>(sP + kP);
+  // P^T of tile i in buffer i % 2, so that the softmax writes tile i while the MMA reads tile i - 1
+  uint8_t* sP0 = base + 2 * kQ + kStages * 2 * kTile + 2 * kRaw * kRawBytes;
+  auto sP = [&](int i) { return sP0 + (i & 1) * kP; };
+  fq::Bars& bars = *reinterpret_cast<fq::Bars*>(sP0 + 2 * kP);
   volatile int* abort = &bars.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
@@ -1269,7 +1365,7 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.qland[i], 1);
-      mbar_init(&bars.qfull[i], 1);
+      mbar_init(&bars.qfull[i], kConvWarps);
       mbar_init(&bars.qempty[i], 1);
       mbar_init(&bars.sfull[i], 1);
       mbar_init(&bars.sfree[i], 4);
@@ -1278,20 +1374,22 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&bars.kland[i], 1);
-      mbar_init(&bars.kfull[i], 1);
+      mbar_init(&bars.kfull[i], kConvWarps);
       mbar_init(&bars.kempty[i], 1);
       mbar_init(&bars.vland[i], 1);
-      mbar_init(&bars.vfull[i], 1);
+      mbar_init(&bars.vfull[i], kConvWarps);
       mbar_init(&bars.vempty[i], 1);
     }
     for (int i = 0; i < kRaw; ++i) {
       mbar_init(&bars.rkfull[i], 1);
-      mbar_init(&bars.rkfree[i], 1);
+      mbar_init(&bars.rkfree[i], kConvWarps);
       mbar_init(&bars.rvfull[i], 1);
-      mbar_init(&bars.rvfree[i], 1);
+      mbar_init(&bars.rvfree[i], kConvWarps);
     }
-    mbar_init(&bars.pfull, 4);
-    mbar_init(&bars.pfree, 1);
+    mbar_init(&bars.pfull[0], 4);
+    mbar_init(&bars.pfull[1], 4);
+    mbar_init(&bars.pfree[0], 1);
+    mbar_init(&bars.pfree[1], 1);
     mbar_init(&bars.done, 1);
     bars.abort = 0;
     bars.last = 0;
@@ -1337,207 +1435,169 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   }
   grid_dependency_wait();
   grid_launch_dependents();
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      TileWalk<kKeys> kw, vw;
-      kw.init_at(a, part_b, part_h, t0);
-      vw.init_at(a, part_b, part_h, t0);
-      int nk = 0, nv = 0, kseg = -1, rk = 0, rv = 0;
-      int kact[kStages] = {0, 0}, vact[kStages] = {0, 0};
-      for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
-        if ((it & 31u) == 31u && *abort) break;
-        if (nk < n) {
-          const bool new_seg = nk == 0 || kw.t == 0, act = kw.t == 0;
-          const int s = kseg + 1;
-          bool can = !new_seg || s < 2 || mbar_test_wait(&bars.qempty[s & 1], ((s >> 1) - 1) & 1);
-          if (act) can = can && (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1));
-          else can = can && (rk < kRaw || mbar_test_wait(&bars.rkfree[rk % kRaw], ((rk / kRaw) - 1) & 1));
-          if (can) {
-            if (new_seg) {
-              kseg = s;
-              mbar_arrive_expect_tx(&bars.qland[s & 1], kQ);
-              tma_load_4d(sQ(s), &maps.q, &bars.qland[s & 1], 0, kw.h, 0, kw.b);
-              tma_load_4d(sQ(s) + kQ / 2, &maps.q, &bars.qland[s & 1], 64, kw.h, 0, kw.b);
-            }
-            if (act) {
-              const int st = nk % kStages;
-              mbar_arrive_expect_tx(&bars.kland[st], kTile);
-              tma_load_4d(sK(st), &maps.ka, &bars.kland[st], 0, kw.h, 0, kw.b);
-              tma_load_4d(sK(st) + kTile / 2, &maps.ka, &bars.kland[st], 64, kw.h, 0, kw.b);
-              ++kact[st];
-            } else {
-              const int sl = rk % kRaw;
-              if (!(nk < 32 && ((pre >> nk) & 1u))) {  // not requested before the wait
-                const int64_t row = raw_row(kw);
-                mbar_arrive_expect_tx(&bars.rkfull[sl], kRawBytes);
-                bulk_load(rK(sl), a.k_codes + row * 64, kCodes, &bars.rkfull[sl]);
-                bulk_load(rK(sl) + kCodes, a.k_scales + row * 8, kScales, &bars.rkfull[sl]);
+  // One register share per warpgroup, taken by all four of its warps at the top of its branch.
+  if (warp < 4) {
+    regs_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ---------------------------------------------------------------- producer
+      if (lane == 0) {
+        TileWalk<kKeys> kw, vw;
+        kw.init_at(a, part_b, part_h, t0);
+        vw.init_at(a, part_b, part_h, t0);
+        int nk = 0, nv = 0, kseg = -1, rk = 0, rv = 0;
+        int kact[kStages] = {0, 0}, vact[kStages] = {0, 0};
+        for (uint32_t it = 0; (nk < n || nv < n) && it < kWaitSpinLimit; ++it) {
+          if ((it & 31u) == 31u && *abort) break;
+          const int nk0 = nk, nv0 = nv;
+          if (nk < n) {
+            const bool new_seg = nk == 0 || kw.t == 0, act = kw.t == 0;
+            const int s = kseg + 1;
+            bool can = !new_seg || s < 2 || mbar_test_wait(&bars.qempty[s & 1], ((s >> 1) - 1) & 1);
+            if (act) can = can && (nk < kStages || mbar_test_wait(&bars.kempty[nk % kStages], ((nk / kStages) - 1) & 1));
+            else can = can && (rk < kRaw || mbar_test_wait(&bars.rkfree[rk % kRaw], ((rk / kRaw) - 1) & 1));
+            if (can) {
+              if (new_seg) {
+                kseg = s;
+                mbar_arrive_expect_tx(&bars.qland[s & 1], kQ);
+                tma_load_4d(sQ(s), &maps.q, &bars.qland[s & 1], 0, kw.h, 0, kw.b);
+                tma_load_4d(sQ(s) + kQ / 2, &maps.q, &bars.qland[s & 1], 64, kw.h, 0, kw.b);
               }
-              ++rk;
-            }
-            ++nk;
-            kw.next(a);
-          }
-        }
-        if (nv < n) {
-          const bool act = vw.t == 0;
-          const bool can = act ? (nv < kStages || mbar_test_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))
-                               : (rv < kRaw || mbar_test_wait(&bars.rvfree[rv % kRaw], ((rv / kRaw) - 1) & 1));
-          if (can) {
-            if (act) {
-              const int st = nv % kStages;
-              mbar_arrive_expect_tx(&bars.vland[st], kTile);
-              tma_load_4d(sV(st), &maps.va, &bars.vland[st], 0, vw.h, 0, vw.b);
-              tma_load_4d(sV(st) + kTile / 2, &maps.va, &bars.vland[st], 64, vw.h, 0, vw.b);
-              ++vact[st];
-            } else {
-              const int sl = rv % kRaw;
-              if (!(nv < 32 && ((pre >> nv) & 1u))) {
-                const int64_t row = raw_row(vw);
-                mbar_arrive_expect_tx(&bars.rvfull[sl], kRawBytes);
-                bulk_load(rV(sl), a.v_codes + row * 64, kCodes, &bars.rvfull[sl]);
-                bulk_load(rV(sl) + kCodes, a.v_scales + row * 8, kScales, &bars.rvfull[sl]);
+              if (act) {
+                const int st = nk % kStages;
+                mbar_arrive_expect_tx(&bars.kland[st], kTile);
+                tma_load_4d(sK(st), &maps.ka, &bars.kland[st], 0, kw.h, 0, kw.b);
+                tma_load_4d(sK(st) + kTile / 2, &maps.ka, &bars.kland[st], 64, kw.h, 0, kw.b);
+                ++kact[st];
+              } else {
+                const int sl = rk % kRaw;
+                if (!(nk < 32 && ((pre >> nk) & 1u))) {  // not requested before the wait
+                  const int64_t row = raw_row(kw);
+                  mbar_arrive_expect_tx(&bars.rkfull[sl], kRawBytes);
+                  bulk_load(rK(sl), a.k_codes + row * 64, kCodes, &bars.rkfull[sl]);
+                  bulk_load(rK(sl) + kCodes, a.k_scales + row * 8, kScales, &bars.rkfull[sl]);
+                }
+                ++rk;
               }
-              ++rv;
-            }
-            ++nv;
-            vw.next(a);
-          }
-        }
-      }
-      if (nk < n || nv < n) *abort = 1;
-      // Copies still in flight land before the CTA leaves (only after an abort can any be).
-      for (int i = (rk > kRaw ? rk - kRaw : 0); i < rk; ++i) mbar_wait(&bars.rkfull[i % kRaw], (i / kRaw) & 1);
-      for (int i = (rv > kRaw ? rv - kRaw : 0); i < rv; ++i) mbar_wait(&bars.rvfull[i % kRaw], (i / kRaw) & 1);
-      for (int st = 0; st < kStages; ++st) {
-        if (kact[st]) mbar_wait(&bars.kland[st], (kact[st] - 1) & 1);
-        if (vact[st]) mbar_wait(&bars.vland[st], (vact[st] - 1) & 1);
-      }
-      for (int s = (kseg > 1 ? kseg - 1 : 0); s <= kseg; ++s) mbar_wait(&bars.qland[s & 1], (s >> 1) & 1);
-    }
-  } else if (warp >= 6) {
-    // ---------------------------------------------------------------- converters
-    // warp 6: Q and K tiles; warp 7: V tiles.  A raw tile is decoded 8 rows per step
-    // (decode_chunk); in-place bf16 tiles are split by 16-byte chunks.
-    const bool is_k = warp == 6;
-    const int t = lane;
-    TileWalk<kKeys> cw;
-    cw.init_at(a, part_b, part_h, t0);
-    int seg = -1, r = 0;
-    int nact[kStages] = {0, 0};
-    bool ok = true;
-    for (int i = 0; i < n; ++i, cw.next(a)) {
-      if (is_k && (i == 0 || cw.t == 0)) {
-        ++seg;
-        ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.qland[seg & 1], (seg >> 1) & 1, abort));
-        if (ok) bf16_tile_to_f16(sQ(seg), kQ, t, 32);
-        tc05::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.qfull[seg & 1]);
-      }
-      const int st = i % kStages;
-      uint8_t* tile = is_k ? sK(st) : sV(st);
-      uint64_t* empty = is_k ? bars.kempty : bars.vempty;
-      if (i >= kStages) ok = __all_sync(FULL, ok && um::wait_or_abort(&empty[st], ((i / kStages) - 1) & 1, abort));
-      if (cw.t == 0) {
-        uint64_t* land = is_k ? bars.kland : bars.vland;
-        ok = __all_sync(FULL, ok && um::wait_or_abort(&land[st], nact[st] & 1, abort));
-        ++nact[st];
-        if (ok) bf16_tile_to_f16(tile, kTile, t, 32);
-      } else {
-        const int sl = r % kRaw;
-        uint64_t* full = is_k ? bars.rkfull : bars.rvfull;
-        ok = __all_sync(FULL, ok && um::wait_or_abort(&full[sl], (r / kRaw) & 1, abort));
-        if (ok) {
-          const uint8_t* raw = is_k ? rK(sl) : rV(sl);
-#pragma unroll 2
-          for (int it = 0; it < 16; ++it) decode_chunk(raw, tile, 8 * it + (t >> 2), t & 3);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(is_k ? &bars.rkfree[sl] : &bars.rvfree[sl]);
-        ++r;
-      }
-      tc05::fence_proxy_async_smem();  // generic writes to the tile before the MMA reads it
-      __syncwarp();
-      if (lane == 0) mbar_arrive(is_k ? &bars.kfull[st] : &bars.vfull[st]);
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idS = idesc_f16_f32(128, 32, false, false);
-      const uint32_t idO = idesc_f16_f32(128, 64, true, true);
-      TileWalk<kKeys> sw, pw;
-      sw.init_at(a, part_b, part_h, t0);
-      pw.init_at(a, part_b, part_h, t0);
-      int ns = 0, sseg = -1, pseg = -1;
-      bool ok = true, vid_started = false;
-      for (int i = 0; ok && i < n; ++i) {
-        const bool p_first = i == 0 || pw.t == 0;
-        const bool p_last = i == n - 1 || pw.t == pw.nb - 1;
-        if (p_first) ++pseg, vid_started = false;
-        bool v_ready = false, p_ready = false, o_ready = !(p_first && pseg >= 2);
-        for (uint32_t it = 0;; ++it) {
-          if (ns < n && ns <= i + 2) {
-            const bool s_first = ns == 0 || sw.t == 0;
-            const int s = sseg + (s_first ? 1 : 0);
-            if (mbar_test_wait(&bars.kfull[ns % kStages], (ns / kStages) & 1) &&
-                (!s_first || mbar_test_wait(&bars.qfull[s & 1], (s >> 1) & 1)) &&
-                (ns < 2 || mbar_test_wait(&bars.sfree[ns & 1], ((ns >> 1) - 1) & 1))) {
-              const bool s_last = ns == n - 1 || sw.t == sw.nb - 1;
-              sseg = s;
-              const int st = ns % kStages;
-              tc05::fence_after_sync();
-              const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ(s));
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                tc05::mma_ss(tmem + 32 * (ns & 1),
-                             tc05::smem_desc_sw128(k_s + (kk >> 2) * (kTile / 2) + (kk & 3) * 32, 16, 1024),
-                             tc05::smem_desc_sw128(q_s + (kk >> 2) * (kQ / 2) + (kk & 3) * 32, 16, 1024), idS,
-                             kk > 0 ? 1u : 0u);
-              tc05::mma_commit(&bars.sfull[ns & 1]);
-              tc05::mma_commit(&bars.kempty[st]);
-              if (s_last) tc05::mma_commit(&bars.qempty[s & 1]);
-              ++ns;
-              sw.next(a);
+              ++nk;
+              kw.next(a);
             }
           }
-          if (ns > i) {
-            v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
-            o_ready = o_ready || mbar_test_wait(&bars.ofree[pseg & 1], ((pseg >> 1) - 1) & 1);
-            p_ready = v_ready && o_ready && mbar_test_wait(&bars.pfull, i & 1);
-            if (p_ready) break;
+          if (nv < n) {
+            const bool act = vw.t == 0;
+            const bool can = act ? (nv < kStages || mbar_test_wait(&bars.vempty[nv % kStages], ((nv / kStages) - 1) & 1))
+                                 : (rv < kRaw || mbar_test_wait(&bars.rvfree[rv % kRaw], ((rv / kRaw) - 1) & 1));
+            if (can) {
+              if (act) {
+                const int st = nv % kStages;
+                mbar_arrive_expect_tx(&bars.vland[st], kTile);
+                tma_load_4d(sV(st), &maps.va, &bars.vland[st], 0, vw.h, 0, vw.b);
+                tma_load_4d(sV(st) + kTile / 2, &maps.va, &bars.vland[st], 64, vw.h, 0, vw.b);
+                ++vact[st];
+              } else {
+                const int sl = rv % kRaw;
+                if (!(nv < 32 && ((pre >> nv) & 1u))) {
+                  const int64_t row = raw_row(vw);
+                  mbar_arrive_expect_tx(&bars.rvfull[sl], kRawBytes);
+                  bulk_load(rV(sl), a.v_codes + row * 64, kCodes, &bars.rvfull[sl]);
+                  bulk_load(rV(sl) + kCodes, a.v_scales + row * 8, kScales, &bars.rvfull[sl]);
+                }
+                ++rv;
+              }
+              ++nv;
+              vw.next(a);
+            }
           }
-          if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
-          if ((it & 31u) == 31u && *abort) { ok = false; break; }
+          if (nk == nk0 && nv == nv0) poll_pause();
         }
-        if (!ok) break;
-        tc05::fence_after_sync();
-        const int st = i % kStages;
-        const bool act = pw.t == 0;
-        const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP);
-        const uint32_t o_t = tmem + (act ? 192 : 64) + 64 * (pseg & 1);
-        const bool acc = !act && vid_started;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc05::mma_ss(o_t, tc05::smem_desc_sw128(v_s + kk * 2048, kTile / 2, 1024),
-                       tc05::smem_desc_sw128(p_s + kk * 2048, kTile / 2, 1024), idO,
-                       (acc || kk > 0) ? 1u : 0u);
-        if (!act) vid_started = true;
-        tc05::mma_commit(&bars.pfree);
-        tc05::mma_commit(&bars.vempty[st]);
-        if (p_last) tc05::mma_commit(&bars.ofull[pseg & 1]);
-        pw.next(a);
+        if (nk < n || nv < n) *abort = 1;
+        // Copies still in flight land before the CTA leaves (only after an abort can any be).
+        for (int i = (rk > kRaw ? rk - kRaw : 0); i < rk; ++i) mbar_wait(&bars.rkfull[i % kRaw], (i / kRaw) & 1);
+        for (int i = (rv > kRaw ? rv - kRaw : 0); i < rv; ++i) mbar_wait(&bars.rvfull[i % kRaw], (i / kRaw) & 1);
+        for (int st = 0; st < kStages; ++st) {
+          if (kact[st]) mbar_wait(&bars.kland[st], (kact[st] - 1) & 1);
+          if (vact[st]) mbar_wait(&bars.vland[st], (vact[st] - 1) & 1);
+        }
+        for (int s = (kseg > 1 ? kseg - 1 : 0); s <= kseg; ++s) mbar_wait(&bars.qland[s & 1], (s >> 1) & 1);
       }
-      tc05::mma_commit(&bars.done);
+    } else if (warp == 1) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t idS = idesc_f16_f32(128, 32, false, false);
+        const uint32_t idO = idesc_f16_f32(128, 64, true, true);
+        TileWalk<kKeys> sw, pw;
+        sw.init_at(a, part_b, part_h, t0);
+        pw.init_at(a, part_b, part_h, t0);
+        int ns = 0, sseg = -1, pseg = -1;
+        bool ok = true, vid_started = false;
+        for (int i = 0; ok && i < n; ++i) {
+          const bool p_first = i == 0 || pw.t == 0;
+          const bool p_last = i == n - 1 || pw.t == pw.nb - 1;
+          if (p_first) ++pseg, vid_started = false;
+          bool v_ready = false, p_ready = false, o_ready = !(p_first && pseg >= 2);
+          for (uint32_t it = 0;; ++it) {
+            const int ns0 = ns;
+            if (ns < n && ns <= i + 2) {
+              const bool s_first = ns == 0 || sw.t == 0;
+              const int s = sseg + (s_first ? 1 : 0);
+              if (mbar_test_wait(&bars.kfull[ns % kStages], (ns / kStages) & 1) &&
+                  (!s_first || mbar_test_wait(&bars.qfull[s & 1], (s >> 1) & 1)) &&
+                  (ns < 2 || mbar_test_wait(&bars.sfree[ns & 1], ((ns >> 1) - 1) & 1))) {
+                const bool s_last = ns == n - 1 || sw.t == sw.nb - 1;
+                sseg = s;
+                const int st = ns % kStages;
+                tc05::fence_after_sync();
+                const uint32_t k_s = smem_u32(sK(st)), q_s = smem_u32(sQ(s));
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                  tc05::mma_ss(tmem + 32 * (ns & 1),
+                               tc05::smem_desc_sw128(k_s + (kk >> 2) * (kTile / 2) + (kk & 3) * 32, 16, 1024),
+                               tc05::smem_desc_sw128(q_s + (kk >> 2) * (kQ / 2) + (kk & 3) * 32, 16, 1024), idS,
+                               kk > 0 ? 1u : 0u);
+                tc05::mma_commit(&bars.sfull[ns & 1]);
+                tc05::mma_commit(&bars.kempty[st]);
+                if (s_last) tc05::mma_commit(&bars.qempty[s & 1]);
+                ++ns;
+                sw.next(a);
+              }
+            }
+            if (ns > i) {
+              v_ready = v_ready || mbar_test_wait(&bars.vfull[i % kStages], (i / kStages) & 1);
+              o_ready = o_ready || mbar_test_wait(&bars.ofree[pseg & 1], ((pseg >> 1) - 1) & 1);
+              p_ready = v_ready && o_ready && mbar_test_wait(&bars.pfull[i & 1], (i >> 1) & 1);
+              if (p_ready) break;
+            }
+            if (ns == ns0) poll_pause();
+            if (it >= kWaitSpinLimit) { *abort = 1; ok = false; break; }
+            if ((it & 31u) == 31u && *abort) { ok = false; break; }
+          }
+          if (!ok) break;
+          tc05::fence_after_sync();
+          const int st = i % kStages;
+          const bool act = pw.t == 0;
+          const uint32_t v_s = smem_u32(sV(st)), p_s = smem_u32(sP(i));
+          const uint32_t o_t = tmem + (act ? 192 : 64) + 64 * (pseg & 1);
+          const bool acc = !act && vid_started;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc05::mma_ss(o_t, tc05::smem_desc_sw128(v_s + kk * 2048, kTile / 2, 1024),
+                         tc05::smem_desc_sw128(p_s + kk * 2048, kTile / 2, 1024), idO,
+                         (acc || kk > 0) ? 1u : 0u);
+          if (!act) vid_started = true;
+          tc05::mma_commit(&bars.pfree[i & 1]);
+          tc05::mma_commit(&bars.vempty[st]);
+          if (p_last) tc05::mma_commit(&bars.ofull[pseg & 1]);
+          pw.next(a);
+        }
+        tc05::mma_commit(&bars.done);
+      }
     }
-  } else if (warp >= 2) {
+  } else if (warp < 8) {
+    regs_inc<kRegsSoftmax>();
     // ---------------------------------------------------------------- softmax, one key per thread
     const int quarter = warp & 3;
     const int L = 32 * quarter + lane;
     const uint32_t lane_off = uint32_t(32 * quarter) << 16;
-    const int wr = warp - 2;
+    const int wr = warp - 4;
     const float c_act = a.scale_log2, c_vid = a.scale_log2 * *a.k_sg, sg_v = *a.v_sg;
     bool ok = true;
     float m[32], l[32];
@@ -1545,6 +1605,14 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     tw.init_at(a, part_b, part_h, t0);
     int seg = -1, i_first = 0;
     bool has_act = false, has_vid = false;  // accumulators written in this segment so far
+    // A P^T row holds P (fp16) in query columns 0-31 and zeros in 32-63: the fp16 P is kept
+    // whole (no low part), so O^T columns 32-63 stay zero and are never read.
+#pragma unroll
+    for (int buf = 0; buf < 2; ++buf) {
+#pragma unroll
+      for (int ch = 4; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(sP(buf) + L * 128 + ((ch ^ (L & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int i = 0; i < n; ++i, tw.next(a)) {
       if (i == 0 || tw.t == 0) {
         ++seg;
@@ -1590,84 +1658,51 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
           m[q] = mn;
         }
         if (i > i_first) {  // rescale the accumulators the segment's earlier tiles wrote
-          ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
+          ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree[(i - 1) & 1], ((i - 1) >> 1) & 1, abort));
           if (ok) {
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
               if (which == 0 ? !has_vid : !has_act) continue;
               const uint32_t ob = which == 0 ? o_vid : o_act;
+              uint32_t o[32];
+              tc05::tmem_ld32(ob + lane_off, o);
+              tc05::tmem_wait_ld();
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                uint32_t o[32];
-                tc05::tmem_ld32(ob + 32 * half + lane_off, o);
-                tc05::tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
-                tc05::tmem_st32(ob + 32 * half + lane_off, o);
-              }
+              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
+              tc05::tmem_st32(ob + lane_off, o);
             }
             tc05::tmem_wait_st();
           }
         }
         um::softmax_sync();
       }
-      // P = P_hi + P_lo, both fp16 (query columns 0-31 and 32-63 of the P^T row)
-      uint32_t pk[16], pl[16];
+      // P in fp16 (query columns 0-31 of the P^T row); its rounding (a relative 2^-12) is far
+      // inside the read's bf16 tolerance
+      uint32_t pk[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float p0 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j]), c, -m[2 * j])) : 0.f;
         const float p1 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -m[2 * j + 1])) : 0.f;
         l[2 * j] += p0, l[2 * j + 1] += p1;
         pk[j] = pack_f16(p0, p1);
-        const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[j]));
-        pl[j] = pack_f16(p0 - hi.x, p1 - hi.y);
       }
-      if (i > 0) ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
+      if (i > 1) ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.pfree[i & 1], ((i >> 1) - 1) & 1, abort));
       if (ok) {
-        uint8_t* row = sP + L * 128;
+        uint8_t* row = sP(i) + L * 128;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 4; ++ch)
           *reinterpret_cast<uint4*>(row + ((ch ^ (L & 7)) << 4)) =
               make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(row + (((ch + 4) ^ (L & 7)) << 4)) =
-              make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
-        }
       }
       tc05::fence_proxy_async_smem();
       tc05::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.pfull);
+      if (lane == 0) mbar_arrive(&bars.pfull[i & 1]);
       if (act) has_act = true;
       else has_vid = true;
       if (!last) continue;
 
-      // ---- segment done: O = s_g(V) O_video + O_action
-      float o[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) o[q] = 0.f;
-      ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.ofull[seg & 1], (seg >> 1) & 1, abort));
-      if (ok) {
-        tc05::fence_after_sync();
-        if (has_vid) {
-          uint32_t ohi[32], olo[32];
-          tc05::tmem_ld32(o_vid + lane_off, ohi);
-          tc05::tmem_ld32(o_vid + 32 + lane_off, olo);
-          tc05::tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = sg_v * (__uint_as_float(ohi[q]) + __uint_as_float(olo[q]));
-        }
-        if (has_act) {
-          uint32_t ohi[32], olo[32];
-          tc05::tmem_ld32(o_act + lane_off, ohi);
-          tc05::tmem_ld32(o_act + 32 + lane_off, olo);
-          tc05::tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] += __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
-        }
-      }
-      tc05::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.ofree[seg & 1]);
+      // ---- segment done: the row sums (while the last P V runs), then O = s_g(V) O_video + O_action
       {
         float v[32];
 #pragma unroll
@@ -1679,9 +1714,78 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
 #pragma unroll
       for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
       um::softmax_sync();
+      float o[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) o[q] = 0.f;
+      ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.ofull[seg & 1], (seg >> 1) & 1, abort));
+      if (ok) {
+        tc05::fence_after_sync();
+        if (has_vid) {
+          uint32_t ov[32];
+          tc05::tmem_ld32(o_vid + lane_off, ov);
+          tc05::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = sg_v * __uint_as_float(ov[q]);
+        }
+        if (has_act) {
+          uint32_t oa[32];
+          tc05::tmem_ld32(o_act + lane_off, oa);
+          tc05::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] += __uint_as_float(oa[q]);
+        }
+      }
+      tc05::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.ofree[seg & 1]);
       split_finish_segment(a, tw.b, tw.h, *reinterpret_cast<volatile int*>(&bars.part_k),
                            *reinterpret_cast<volatile int*>(&bars.part_r), L, wr, lane, o, lt, m, &bars.last,
                            sK(0), kStageParts, &bars.mfull, abort);
+    }
+  } else {
+    regs_dec<kRegsConv>();
+    // ---------------------------------------------------------------- converters
+    // warps 8-11: Q and K tiles; warps 12-15: V tiles.  Warp g of a group decodes row groups g,
+    // g + 4, g + 8, g + 12 of a raw tile (decode_rows); in-place bf16 tiles are split by 16-byte
+    // chunks over the group's 128 threads.  Every warp of the group arrives on the tile's barriers.
+    const bool is_k = warp < 12;
+    const int g = warp & 3;
+    const int t = 32 * g + lane;
+    TileWalk<kKeys> cw;
+    cw.init_at(a, part_b, part_h, t0);
+    int seg = -1, r = 0;
+    int nact[kStages] = {0, 0};
+    bool ok = true;
+    for (int i = 0; i < n; ++i, cw.next(a)) {
+      if (is_k && (i == 0 || cw.t == 0)) {
+        ++seg;
+        ok = __all_sync(FULL, ok && um::wait_or_abort(&bars.qland[seg & 1], (seg >> 1) & 1, abort));
+        if (ok) bf16_tile_to_f16(sQ(seg), kQ, t, 32 * kConvWarps);
+        tc05::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.qfull[seg & 1]);
+      }
+      const int st = i % kStages;
+      uint8_t* tile = is_k ? sK(st) : sV(st);
+      uint64_t* empty = is_k ? bars.kempty : bars.vempty;
+      if (i >= kStages) ok = __all_sync(FULL, ok && um::wait_or_abort(&empty[st], ((i / kStages) - 1) & 1, abort));
+      if (cw.t == 0) {
+        uint64_t* land = is_k ? bars.kland : bars.vland;
+        ok = __all_sync(FULL, ok && um::wait_or_abort(&land[st], nact[st] & 1, abort));
+        ++nact[st];
+        if (ok) bf16_tile_to_f16(tile, kTile, t, 32 * kConvWarps);
+      } else {
+        const int sl = r % kRaw;
+        uint64_t* full = is_k ? bars.rkfull : bars.rvfull;
+        ok = __all_sync(FULL, ok && um::wait_or_abort(&full[sl], (r / kRaw) & 1, abort));
+        if (ok) decode_rows(is_k ? rK(sl) : rV(sl), tile, g, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(is_k ? &bars.rkfree[sl] : &bars.rvfree[sl]);
+        ++r;
+      }
+      tc05::fence_proxy_async_smem();  // generic writes to the tile before the MMA reads it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(is_k ? &bars.kfull[st] : &bars.vfull[st]);
     }
   }
 
@@ -1927,6 +2031,12 @@ cudaError_t launch_action_nvfp4(const ActionArgs& a, cudaStream_t s) {
   maps.fk = maps.ka, maps.fv = maps.va;  // unused: the video tiles come by bulk copies
   cudaError_t e = cudaFuncSetAttribute(action_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fq::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // the warpgroups' register shares add up to exactly the launch allocation: a build that
+  // launched with fewer registers per thread would leave the softmax warps' increase unmet
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, action_nvfp4_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != int(fq::kRegsLaunch)) return cudaErrorInvalidDeviceFunction;
   return launch_pdl(action_nvfp4_kernel, dim3(unsigned(a.P)), dim3(fq::kThreads), fq::kSmemBytes, s, 0, a,
                     maps);
 }

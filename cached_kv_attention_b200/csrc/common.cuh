@@ -137,6 +137,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 }
 
 constexpr uint32_t kWaitSpinLimit = 1u << 24;  // try_wait rounds before a wait gives up
+// A warp that polls several barriers with test_wait and found none of them ready pauses for a
+// moment (at most twice this many nanoseconds), so that the warps sharing its scheduler keep
+// their issue slots.
+constexpr unsigned kPollPauseNs = 32;
+__device__ __forceinline__ void poll_pause() { __nanosleep(kPollPauseNs); }
 
 // ---------------------------------------------------------------------------------------
 // PTX wrappers: shared-memory addresses, mbarriers, TMA, ldmatrix, mma.sync

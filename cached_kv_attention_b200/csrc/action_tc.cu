@@ -134,7 +134,7 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
   constexpr int kWK = kBN / 4;               // keys per warp per tile
   constexpr int kNT = kWK / 8;               // 8-key groups per warp per tile
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   uint8_t* sq[2] = {base, base + kQBytes};
   uint8_t* sk[kStages];
   uint8_t* sv[kStages];
@@ -587,8 +587,14 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 __global__ void __launch_bounds__(um::kThreads, 1)
 action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
   using namespace um;
+  // the tensor maps' descriptors first: fetching one takes about a microsecond, hidden behind
+  // the set-up below (parameter space: the previous kernel on the stream cannot write it)
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
+    prefetch_tmap(&maps.fk), prefetch_tmap(&maps.fv);
+  }
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   uint8_t* sQ = base;
   auto sK = [&](int st) { return base + kQ + st * kTile; };
   auto sV = [&](int st) { return base + kQ + (kKStages + st) * kTile; };
@@ -632,15 +638,6 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       const int rows = (rank + 1) * a.n_act / k - rank * a.n_act / k;
       mbar_init(&bars.rx_full, 1);
       mbar_arrive_expect_tx(&bars.rx_full, uint32_t((k - 1) * rows * 520));
-      // row q of this CTA's partial goes to slot `rank` of its owner's receive region
-      for (int r = 0; r < k; ++r) {
-        const int r0 = r * a.n_act / k, r1 = (r + 1) * a.n_act / k, rows = r1 - r0;
-        for (int q = r0; q < r1; ++q) {
-          bars.row_owner[q] = r;
-          bars.row_off[q] = (rank * rows + (q - r0)) * 512;
-          bars.ml_off[q] = k * rows * 512 + (rank * rows + (q - r0)) * 8;
-        }
-      }
     }
     fence_barrier_init();
   }
@@ -685,8 +682,6 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   const int n_pre = n < kVStages ? n : kVStages;  // kVStages <= kKStages
   uint32_t pre = 0;  // bit i: tile i requested before the dependency wait
   if (threadIdx.x == 0) {
-    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
-    prefetch_tmap(&maps.fk), prefetch_tmap(&maps.fv);
     if (a.fused_ready)
       for (int i = 0; i < n_pre; ++i)
         if (t0 + i != 0) load_kv(i), pre |= 1u << i;
@@ -804,6 +799,16 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
     const uint32_t lane_off = uint32_t(32 * quarter) << 16;
     const int wr = warp - 2;            // this warp's row of bars.red
     const float c = a.scale_log2;
+    if (k > 1 && wr == 0 && lane < a.n_act) {
+      // row q = lane of this CTA's partial goes to slot `rank` of its owner's receive region
+      // (read at the merge, after several softmax barriers)
+      int r = 0;
+      while ((r + 1) * a.n_act / k <= lane) ++r;
+      const int r0 = r * a.n_act / k, rows = (r + 1) * a.n_act / k - r0;
+      bars.row_owner[lane] = r;
+      bars.row_off[lane] = (rank * rows + (lane - r0)) * 512;
+      bars.ml_off[lane] = k * rows * 512 + (rank * rows + (lane - r0)) * 8;
+    }
     bool ok = true;
     float m[32], l[32];
 #pragma unroll
@@ -1339,8 +1344,9 @@ __device__ __forceinline__ void regs_inc() {
 __global__ void __launch_bounds__(fq::kThreads, 1)
 action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ ActionMaps maps) {
   using namespace fq;
+  if (threadIdx.x == 0) prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   auto sQ = [&](int s) { return base + (s & 1) * kQ; };
   auto sK = [&](int st) { return base + 2 * kQ + st * 2 * kTile; };
   auto sV = [&](int st) { return base + 2 * kQ + st * 2 * kTile + kTile; };
@@ -1415,7 +1421,6 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   // are requested before the dependency wait; bit i of pre: tile i of the part.
   uint32_t pre = 0;
   if (threadIdx.x == 0) {
-    prefetch_tmap(&maps.q), prefetch_tmap(&maps.ka), prefetch_tmap(&maps.va);
     if (a.fused_ready) {
       TileWalk<kKeys> w;
       w.init_at(a, part_b, part_h, t0);

@@ -149,6 +149,12 @@ __device__ __forceinline__ void poll_pause() { __nanosleep(kPollPauseNs); }
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// The first 1024-byte-aligned byte of dynamic shared memory, found by pointer arithmetic on the
+// shared array itself: the compiler then keeps every access through the result in the shared
+// state space, where a round trip through an integer would leave a generic pointer.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

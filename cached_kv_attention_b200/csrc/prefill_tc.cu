@@ -262,8 +262,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
+  // the tensor maps' descriptors first, hidden behind the set-up below (parameter space: the
+  // previous kernel on the stream cannot write it)
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&maps.q), prefetch_tmap(&maps.kn), prefetch_tmap(&maps.vn);
+    prefetch_tmap(&maps.kc), prefetch_tmap(&maps.vc);
+  }
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   // Tiles by arithmetic, not through pointer arrays (a runtime index would put those in local memory).
   auto sQ = [&](int w) { return base + w * kTile; };
   auto sK = [&](int i) { return base + (2 + i) * kTile; };
@@ -320,10 +326,6 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const uint32_t tmem = bars.tmem_base;
   // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
   // the stream may still be finishing (programmatic dependent launch).
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&maps.q), prefetch_tmap(&maps.kn), prefetch_tmap(&maps.vn);
-    prefetch_tmap(&maps.kc), prefetch_tmap(&maps.vc);
-  }
   grid_dependency_wait();
   grid_launch_dependents();
 

@@ -968,44 +968,53 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       }
       wait_cluster(&bars.rx_full, 0, abort);  // every peer's rows for this CTA have landed
       softmax_sync();                         // and this CTA's own copies
-      // merge rows [r0, r1): warp wr takes rows wr, wr + 4, ...; lane the columns 4 lane .. + 3
+      // merge rows [r0, r1): half-warp hw = 2 wr + lane / 16 takes rows hw, hw + 8, ... (one round
+      // for rows <= 8), its lane the columns 8 (lane % 16) .. + 7
       const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k, rows = r1 - r0;
       const float* rxo = reinterpret_cast<const float*>(rx);
       const float* rml = reinterpret_cast<const float*>(rx + k * rows * 512);
-      for (int j = wr; j < rows; j += 4) {
-        // every slot's (m, l) and 16 bytes of its row first: one round of shared loads
+      const int hw = 2 * wr + (lane >> 4), c0 = 8 * (lane & 15);
+      for (int j = hw; j < rows; j += 8) {
+        // every slot's (m, l) and its 32 bytes of the row first: one round of shared loads
         float pm[kMaxSplit], pl_[kMaxSplit];
-        float4 px[kMaxSplit];
+        float4 pa[kMaxSplit], pb[kMaxSplit];
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p) {
           if (p >= k) continue;
           pm[p] = rml[2 * (p * rows + j)], pl_[p] = rml[2 * (p * rows + j) + 1];
-          px[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + 4 * lane);
+          pa[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0);
+          pb[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0 + 4);
         }
         float M = -INFINITY;
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p)
           if (p < k) M = fmaxf(M, pm[p]);
         const float Mu = M == -INFINITY ? 0.f : M;
-        float num[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
+        float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
 #pragma unroll
         for (int p = 0; p < kMaxSplit; ++p) {
           if (p >= k) continue;
           const float wgt = exp2f(pm[p] - Mu);
           den = fmaf(wgt, pl_[p], den);
-          num[0] = fmaf(wgt, px[p].x, num[0]), num[1] = fmaf(wgt, px[p].y, num[1]);
-          num[2] = fmaf(wgt, px[p].z, num[2]), num[3] = fmaf(wgt, px[p].w, num[3]);
+          num[0] = fmaf(wgt, pa[p].x, num[0]), num[1] = fmaf(wgt, pa[p].y, num[1]);
+          num[2] = fmaf(wgt, pa[p].z, num[2]), num[3] = fmaf(wgt, pa[p].w, num[3]);
+          num[4] = fmaf(wgt, pb[p].x, num[4]), num[5] = fmaf(wgt, pb[p].y, num[5]);
+          num[6] = fmaf(wgt, pb[p].z, num[6]), num[7] = fmaf(wgt, pb[p].w, num[7]);
         }
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        float val[4];
+        float val[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) val[e] = num[e] * inv;
-        const int64_t off = ((int64_t(b) * a.n_act + r0 + j) * a.H + h) * 128 + 4 * lane;
-        if (a.o_f32)
-          *reinterpret_cast<float4*>(static_cast<float*>(a.o) + off) = make_float4(val[0], val[1], val[2], val[3]);
-        else
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + off) =
-              make_uint2(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]));
+        for (int e = 0; e < 8; ++e) val[e] = num[e] * inv;
+        const int64_t off = ((int64_t(b) * a.n_act + r0 + j) * a.H + h) * 128 + c0;
+        if (a.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
+          dst[0] = make_float4(val[0], val[1], val[2], val[3]);
+          dst[1] = make_float4(val[4], val[5], val[6], val[7]);
+        } else {
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off) =
+              make_uint4(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]), pack_bf16(val[4], val[5]),
+                         pack_bf16(val[6], val[7]));
+        }
       }
     }
   }

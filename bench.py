@@ -383,7 +383,11 @@ def run_reference(args, world, rank):
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one imagination-pass prefill
 # launch, from one ncu capture of the same kernel (`bench.py --profile-call future`); the
 # stride variants launch the identical imagination pass, other workloads report None.
-IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 80.3e6}
+IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 79.75e6}
+# The same for one fused-cache action read (`bench.py --profile-call action`, and
+# `--workload nvfp4_ctx19.2s_bf16 --profile-call action_nvfp4` for the NVFP4 read); the stride
+# variants issue the identical bf16 read.
+ACTION_TRAFFIC_BYTES = {"ctx19.2s_bf16": 67.42e6, "nvfp4_ctx19.2s_bf16": 19.27e6}
 
 
 def time_fused_read(runner, stream, n=20) -> float:
@@ -539,12 +543,15 @@ def run_mine(args, world, rank, local):
                 "video_stage_tflops": work["prefill_flops"] / (video_ms * 1e-3) / 1e12}
     fused_bytes = work["fused_read_bytes"] + w.n_act * w.H * w.D * (3 * 2 + 4) * w.B
     fused_gbs = fused_bytes / (fused_ms * 1e-3) / 1e9
+    traffic_key = "ctx19.2s_bf16" if w.name.startswith("stride") and w.name.endswith("_ctx19.2s_bf16") else w.name
+    action_traffic = ACTION_TRAFFIC_BYTES.get(traffic_key)
     roofline_action = {"bound": "hbm", "achieved": fused_gbs, "peak": hbm_peak, "unit": "GB/s",
                        "frac": fused_gbs / hbm_peak,
                        "kernel": ("action_nvfp4_kernel, one NVFP4 fused-cache read (wam_action_attn_nvfp4)"
                                   if w.kv_format == "nvfp4" else
                                   "action_umma_kernel, one fused-cache read (wam_action_attn)"),
                        "peak_kind": f"{peak_src} copy bandwidth", "bytes_per_launch": fused_bytes,
+                       "traffic": action_traffic,
                        "ms_per_launch": fused_ms,
                        "method": "one Euler step's interaction reads (one per fused pair) back to back "
                                  "in a CUDA graph after an L2 flush, time / reads",

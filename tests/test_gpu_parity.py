@@ -260,6 +260,35 @@ def test_action_attention(B, H, D, T, F, n_act, pad, dtype, std, video):
     assert_parity(to64(o), ref, dtype, "action O")
 
 
+# One case per cluster size of the 128-key read: the runtime co-schedules 15 clusters of 8 CTAs,
+# 22 of 6, 26 of 5, 33 of 4, 45 of 3, 74 of 2 on a 148-SM B200 at this footprint, so these B x H
+# give 8, 6, 5, 4, 3, 2 and 1 CTAs per (episode, head).  n_act below the cluster size leaves
+# owners with no rows of the merge, and the first case (one valid 512-token frame: 5 tiles with
+# the action tile, over 8 CTAs) leaves three slices with no tile at all.
+MERGE_CASES = [
+    # B, H, F, n_act, pad
+    (1, 4, 2, 1, [[1, 0]]),
+    (2, 8, 3, 5, [[0, 0, 0], [1, 0, 0]]),
+    (1, 24, 3, 32, [[0, 1, 0]]),
+    (1, 30, 3, 7, [[0, 0, 0]]),
+    (2, 20, 3, 32, [[1, 0, 0], [0, 0, 0]]),
+    (3, 20, 2, 3, [[0, 0], [0, 1], [0, 0]]),
+    (4, 25, 2, 32, [[0, 0]] * 4),
+]
+
+
+@pytest.mark.parametrize("B,H,F,n_act,pad", MERGE_CASES)
+def test_action_cluster_merge_every_split(B, H, F, n_act, pad):
+    T = 512
+    lay = wam.VideoLayout(B, H, 128, T, F, pad)
+    fk, fv = (dev_normal((B, F * T, H, 128), 65, x, dtype=torch.bfloat16) for x in ("fk", "fv"))
+    qa, ka, va = (dev_normal((B, n_act, H, 128), 65, x, dtype=torch.bfloat16) for x in ("qa", "ka", "va"))
+    o = torch.full((B, n_act, H, 128), SENTINEL, device="cuda")
+    wam.action_attn(lay, fk, fv, qa, ka, va, o)
+    ref = O.action_attention(to64(qa), to64(ka), to64(va), to64(fk), to64(fv), np.array(pad), T)
+    assert_parity(to64(o), ref, "bf16", f"action O, B x H = {B * H}")
+
+
 @pytest.mark.parametrize("n_act", [32, 5])
 def test_action_large_logit_jumps(n_act):
     # Later key frames score far above earlier ones, so each query's running reference has to

@@ -829,6 +829,20 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.sfree[i & 1]);
       const bool kv = t != 0 || L < a.n_act;  // keys past n_act in the action tile are padding
+      if (i == 0) {
+        // Every query's first reference: its score against key 0 (a valid key of every tile),
+        // so that the exact tile maxima below are taken only for a score more than 2^16 above it
+        // (with -inf they always were, a reduction across the 128 threads on every CTA's first
+        // tile).  Any finite reference gives the same result; only its headroom matters.
+        if (L == 0) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) bars.red[0][q] = __uint_as_float(sr[q]) * c;
+        }
+        softmax_sync();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) m[q] = bars.red[0][q];
+        softmax_sync();  // bars.red is rewritten below
+      }
       float ymax = -INFINITY;
 #pragma unroll
       for (int q = 0; q < 32; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));
@@ -1653,6 +1667,18 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
       if (lane == 0) mbar_arrive(&bars.sfree[i & 1]);
       const bool kv = !act || L < a.n_act;
       const uint32_t o_vid = tmem + 64 + 64 * (seg & 1), o_act = tmem + 192 + 64 * (seg & 1);
+      if (i == i_first) {
+        // the segment's first reference: each query's score against key 0 (valid in every tile),
+        // as in the bf16 read
+        if (L == 0) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) bars.red[0][q] = __uint_as_float(sr[q]) * c;
+        }
+        um::softmax_sync();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) m[q] = bars.red[0][q];
+        um::softmax_sync();
+      }
       float ymax = -INFINITY;
 #pragma unroll
       for (int q = 0; q < 32; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));

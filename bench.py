@@ -358,15 +358,19 @@ def run_reference(args, world, rank):
     # the video stages were sampled on 1/stride of their query rows: time them at full rows
     full = oracle_sample_seconds(w, pad, n_heads, n_layers, seed=3000, row_stride=1)
     part = oracle_sample_seconds(w, pad, n_heads, n_layers, seed=3000, row_stride=stride)
-    chunk_s = sum(times) / len(times) * (full / part) * scale
-    value = 1.0 / chunk_s
+    step_s = sum(times) / len(times)
+    # one timed step does this fraction of a chunk's work (its rows on 1 / stride of the video
+    # queries, timed against one full-row step, and 1 / scale of the heads x layers)
+    chunks_per_step = 1.0 / ((full / part) * scale)
+    value = chunks_per_step / step_s
     sample = (f"each step: all stages of one chunk for {n_heads}/{w.H} heads x {n_layers}/{w.L} "
               f"layers on every {stride}th video query row, scaled to all rows by one full-row "
               f"step (x{full / part:.2f}) and x{scale:.0f} to a whole chunk")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": chunk_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": step_s * 1e3, "chunks_per_step": chunks_per_step,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "T": w.T,
                    "F_h": w.F_h, "F_f": w.F_f, "pad_frames": int(pad.sum()), "n_act": w.n_act,

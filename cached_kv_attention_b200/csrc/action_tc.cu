@@ -612,8 +612,41 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   const int tpf = a.T / kKeys;
   const int nb = tiles_of<kKeys>(a, b);
   const int t0 = rank * nb / k, t1 = (rank + 1) * nb / k, n = t1 - t0;
+  auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
+    const int t = t0 + i;
+    if (t == 0) {
+      mp = is_v ? &maps.va : &maps.ka, tok = 0;
+    } else {
+      const int vt = t - 1;
+      mp = is_v ? &maps.fv : &maps.fk;
+      tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
+    }
+  };
+  auto load_kv = [&](int i) {  // K and V of the slice's tile i (i < both ring sizes)
+    const CUtensorMap* mp;
+    int tok;
+    tile_src(i, false, mp, tok);
+    mbar_arrive_expect_tx(&bars.kfull[i], kTile);
+    tma_load_4d(sK(i), mp, &bars.kfull[i], 0, h, tok, b);
+    tma_load_4d(sK(i) + kTile / 2, mp, &bars.kfull[i], 64, h, tok, b);
+    tile_src(i, true, mp, tok);
+    mbar_arrive_expect_tx(&bars.vfull[i], kTile);
+    tma_load_4d(sV(i), mp, &bars.vfull[i], 0, h, tok, b);
+    tma_load_4d(sV(i) + kTile / 2, mp, &bars.vfull[i], 64, h, tok, b);
+  };
+  const int n_pre = n < kVStages ? n : kVStages;  // kVStages <= kKStages
+  uint32_t pre = 0;  // bit i: tile i requested before the dependency wait (thread 0)
 
   if (threadIdx.x == 0) {
+    // the frame table's entries for the first tiles, fetched while the barriers are set up
+    int warm = 0;
+    for (int i = 0; i < n_pre; ++i) {
+      const CUtensorMap* mp;
+      int tok;
+      tile_src(i, false, mp, tok);
+      warm += tok;
+    }
+    asm volatile("" ::"r"(warm));
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(&bars.kfull[i], 1);
       mbar_init(&bars.kempty[i], 1);
@@ -640,6 +673,14 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       mbar_arrive_expect_tx(&bars.rx_full, uint32_t((k - 1) * rows * 520));
     }
     fence_barrier_init();
+    // Up to here only this CTA's shared memory was touched: the previous kernel on the stream
+    // may still be finishing (programmatic dependent launch).  With a.fused_ready the caller
+    // guarantees that kernel does not write the fused pair, so the slice's first fused tiles
+    // are requested now, by the thread that set up their barriers (the fence above makes them
+    // visible to the copies); the action tile and Q wait for the dependency.
+    if (a.fused_ready)
+      for (int i = 0; i < n_pre; ++i)
+        if (t0 + i != 0) load_kv(i), pre |= 1u << i;
   }
   if (warp == 1) {
     tc05::tmem_alloc(&bars.tmem_base, kTmemCols);
@@ -648,44 +689,12 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
   tc05::fence_before_sync();
   __syncthreads();
   tc05::fence_after_sync();
-  // every CTA of the cluster has initialised (and armed) its barriers once this phase completes;
-  // each thread waits on it before its first access to a peer (the softmax warps) or before
-  // leaving
-  if (k > 1) asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  // every CTA of the cluster has initialised (and armed) its barriers once this phase completes
+  // (the barrier-init fence above orders the initialisation; the receive barrier's byte count
+  // may be armed after a peer's first bytes land); each thread waits on it before its first
+  // access to a peer (the softmax warps) or before leaving
+  if (k > 1) asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
   const uint32_t tmem = bars.tmem_base;
-  auto tile_src = [&](int i, bool is_v, const CUtensorMap*& mp, int& tok) {
-    const int t = t0 + i;
-    if (t == 0) {
-      mp = is_v ? &maps.va : &maps.ka, tok = 0;
-    } else {
-      const int vt = t - 1;
-      mp = is_v ? &maps.fv : &maps.fk;
-      tok = int(a.fl.vlist[b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
-    }
-  };
-  auto load_kv = [&](int i) {  // K and V of the slice's tile i (i < both ring sizes)
-    const CUtensorMap* mp;
-    int tok;
-    tile_src(i, false, mp, tok);
-    mbar_arrive_expect_tx(&bars.kfull[i], kTile);
-    tma_load_4d(sK(i), mp, &bars.kfull[i], 0, h, tok, b);
-    tma_load_4d(sK(i) + kTile / 2, mp, &bars.kfull[i], 64, h, tok, b);
-    tile_src(i, true, mp, tok);
-    mbar_arrive_expect_tx(&bars.vfull[i], kTile);
-    tma_load_4d(sV(i), mp, &bars.vfull[i], 0, h, tok, b);
-    tma_load_4d(sV(i) + kTile / 2, mp, &bars.vfull[i], 64, h, tok, b);
-  };
-  // Up to here only this CTA's shared and tensor memory was touched: the previous kernel on
-  // the stream may still be finishing (programmatic dependent launch).  With a.fused_ready the
-  // caller guarantees that kernel does not write the fused pair, so the slice's first fused
-  // tiles are requested now; the action tile and Q wait for it.
-  const int n_pre = n < kVStages ? n : kVStages;  // kVStages <= kKStages
-  uint32_t pre = 0;  // bit i: tile i requested before the dependency wait
-  if (threadIdx.x == 0) {
-    if (a.fused_ready)
-      for (int i = 0; i < n_pre; ++i)
-        if (t0 + i != 0) load_kv(i), pre |= 1u << i;
-  }
   grid_dependency_wait();
   grid_launch_dependents();
 

@@ -973,7 +973,7 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       }
       softmax_sync();
       asm volatile("barrier.cluster.wait.acquire;" ::: "memory");  // every owner has armed rx_full
-#pragma unroll
+#pragma unroll 1
       for (int it = 0; it < 8; ++it) {  // chunk c: 16 bytes of row c / 32 (n_act <= 32 rows)
         const int c = L + 128 * it, q = c >> 5, ch = c & 31;
         if (q >= a.n_act) continue;
@@ -997,34 +997,27 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       const float* rxo = reinterpret_cast<const float*>(rx);
       const float* rml = reinterpret_cast<const float*>(rx + k * rows * 512);
       const int hw = 2 * wr + (lane >> 4), c0 = 8 * (lane & 15);
+      // (the merge and the sends above run once per CTA, from a cold instruction cache: their
+      // loops stay rolled)
       for (int j = hw; j < rows; j += 8) {
-        // every slot's (m, l) and its 32 bytes of the row first: one round of shared loads
-        float pm[kMaxSplit], pl_[kMaxSplit];
-        float4 pa[kMaxSplit], pb[kMaxSplit];
-#pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p) {
-          if (p >= k) continue;
-          pm[p] = rml[2 * (p * rows + j)], pl_[p] = rml[2 * (p * rows + j) + 1];
-          pa[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0);
-          pb[p] = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0 + 4);
-        }
         float M = -INFINITY;
-#pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p)
-          if (p < k) M = fmaxf(M, pm[p]);
+#pragma unroll 1
+        for (int p = 0; p < k; ++p) M = fmaxf(M, rml[2 * (p * rows + j)]);
         const float Mu = M == -INFINITY ? 0.f : M;
         float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
-#pragma unroll
-        for (int p = 0; p < kMaxSplit; ++p) {
-          if (p >= k) continue;
-          const float wgt = exp2f(pm[p] - Mu);
-          den = fmaf(wgt, pl_[p], den);
-          num[0] = fmaf(wgt, pa[p].x, num[0]), num[1] = fmaf(wgt, pa[p].y, num[1]);
-          num[2] = fmaf(wgt, pa[p].z, num[2]), num[3] = fmaf(wgt, pa[p].w, num[3]);
-          num[4] = fmaf(wgt, pb[p].x, num[4]), num[5] = fmaf(wgt, pb[p].y, num[5]);
-          num[6] = fmaf(wgt, pb[p].z, num[6]), num[7] = fmaf(wgt, pb[p].w, num[7]);
+#pragma unroll 1
+        for (int p = 0; p < k; ++p) {
+          const float2 ml = *reinterpret_cast<const float2*>(rml + 2 * (p * rows + j));
+          const float4 pa = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0);
+          const float4 pb = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0 + 4);
+          const float wgt = tc05::fast_exp2(ml.x - Mu);
+          den = fmaf(wgt, ml.y, den);
+          num[0] = fmaf(wgt, pa.x, num[0]), num[1] = fmaf(wgt, pa.y, num[1]);
+          num[2] = fmaf(wgt, pa.z, num[2]), num[3] = fmaf(wgt, pa.w, num[3]);
+          num[4] = fmaf(wgt, pb.x, num[4]), num[5] = fmaf(wgt, pb.y, num[5]);
+          num[6] = fmaf(wgt, pb.z, num[6]), num[7] = fmaf(wgt, pb.w, num[7]);
         }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
+        const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
         float val[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) val[e] = num[e] * inv;

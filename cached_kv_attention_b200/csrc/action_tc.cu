@@ -481,7 +481,7 @@ constexpr int kKStages = 3;            // K ring
 constexpr int kVStages = 2;            // V ring (its tiles are needed one S^T later than K's)
 constexpr int kQ = 32 * 128 * 2;         // 8 KB
 constexpr int kP = kKeys * 128;          // P^T: 128 keys x (32 P_hi + 32 P_lo) bf16 = 16 KB
-constexpr int kThreads = 6 * 32;
+constexpr int kThreads = 10 * 32;       // producer, MMA issuer, 8 softmax warps
 constexpr uint32_t kTmemCols = 128;      // S^T buffers at columns 0 and 32, O^T at 64
 constexpr float kLazy = 16.f;            // reference headroom (log2 units): P <= 2^16
 constexpr int kMaxSplit = 8;             // portable cluster size
@@ -490,7 +490,7 @@ struct Bars {
   uint64_t qfull, sfull[2], sfree[2], pfull, pfree, ofull, done;
   uint32_t tmem_base;
   int abort;
-  float red[4][32];
+  float red[8][16];  // per softmax warp: one value per query of its group
   // the merge over the cluster: completes once every peer's partial rows for this CTA have landed
   uint64_t rx_full;
   float part_m[32], part_l[32];  // this CTA's partial: reference max and row sum per query
@@ -519,6 +519,18 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }
 // Named barrier 1 over the 128 softmax threads, and the same barrier with an OR-reduction.
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The same over the 256 threads of two softmax warpgroups.
+__device__ __forceinline__ void softmax8_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool softmax8_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n barrier.red.or.pred p, 1, 256, q;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ bool softmax_any(bool v) {
   uint32_t r;
   asm volatile(
@@ -571,6 +583,28 @@ template <bool kMax>
 __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) {
+    const bool hi = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = hi ? v[i] : v[i + off];
+      const float keep = hi ? v[i + off] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+// The same for 16 values: after the call lanes q and q + 16 hold the max (or sum) over the
+// warp's lanes of v[q]; v is clobbered.
+template <bool kMax>
+__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float got = __shfl_xor_sync(0xffffffffu, v[i], 16);
+    v[i] = kMax ? fmaxf(v[i], got) : v[i] + got;
+  }
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) {
     const bool hi = (lane & off) != 0;
 #pragma unroll
     for (int i = 0; i < off; ++i) {
@@ -658,9 +692,9 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
     mbar_init(&bars.qfull, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.sfull[i], 1);
-      mbar_init(&bars.sfree[i], 4);
+      mbar_init(&bars.sfree[i], 8);  // one arrival per softmax warp
     }
-    mbar_init(&bars.pfull, 4);
+    mbar_init(&bars.pfull, 8);
     mbar_init(&bars.pfree, 1);
     mbar_init(&bars.ofull, 1);
     mbar_init(&bars.done, 1);
@@ -800,13 +834,18 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
     }
   } else {
     // ---------------------------------------------------------------- softmax, one key per thread
-    // Every wait in front of a warp-collective instruction is voted across the warp, and all
-    // four warps run the same sequence of named barriers whatever happens, so after a timeout
-    // they keep walking their tiles without doing work and no barrier waits on a warp that left.
+    // Two warpgroups: warp w takes keys 32 (w % 4) .. + 31 of each tile (its TMEM lane quarter)
+    // and the 16 queries 16 qh .. + 15 of its group qh, so a tile's exponentials and P stores
+    // are spread over 8 warps, two per SM sub-partition.  Every wait in front of a warp-collective
+    // instruction is voted across the warp, and all eight warps run the same sequence of named
+    // barriers whatever happens, so after a timeout they keep walking their tiles without doing
+    // work and no barrier waits on a warp that left.
     const int quarter = warp & 3;
     const int L = 32 * quarter + lane;  // key of the tile (S^T lane) and column d of O (O^T lane)
     const uint32_t lane_off = uint32_t(32 * quarter) << 16;
-    const int wr = warp - 2;            // this warp's row of bars.red
+    const int wr = warp - 2;            // this warp's row of bars.red (0-7)
+    const int qh = wr >> 2, q0 = 16 * qh;
+    const int st_i = int(threadIdx.x) - 64;  // this thread among the 256 softmax threads
     const float c = a.scale_log2;
     if (k > 1 && wr == 0 && lane < a.n_act) {
       // row q = lane of this CTA's partial goes to slot `rank` of its owner's receive region
@@ -819,20 +858,20 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       bars.ml_off[lane] = k * rows * 512 + (rank * rows + (lane - r0)) * 8;
     }
     bool ok = true;
-    float m[32], l[32];
+    float m[16], l[16];  // query q0 + q: reference max and this thread's share of the row sum
 #pragma unroll
-    for (int q = 0; q < 32; ++q) m[q] = -INFINITY, l[q] = 0.f;
+    for (int q = 0; q < 16; ++q) m[q] = -INFINITY, l[q] = 0.f;
     for (int i = 0; i < n; ++i) {
       const int t = t0 + i;
       ok = __all_sync(FULL, ok && wait_or_abort(&bars.sfull[i & 1], (i >> 1) & 1, abort));
-      uint32_t sr[32];
+      uint32_t sr[16];
       if (ok) {
         tc05::fence_after_sync();
-        tc05::tmem_ld32(tmem + 32 * (i & 1) + lane_off, sr);
+        tc05::tmem_ld16(tmem + 32 * (i & 1) + q0 + lane_off, sr);
         tc05::tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sr[q] = 0u;
+        for (int q = 0; q < 16; ++q) sr[q] = 0u;
       }
       tc05::fence_before_sync();
       __syncwarp();
@@ -841,76 +880,81 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       if (i == 0) {
         // Every query's first reference: its score against key 0 (a valid key of every tile),
         // so that the exact tile maxima below are taken only for a score more than 2^16 above it
-        // (with -inf they always were, a reduction across the 128 threads on every CTA's first
+        // (with -inf they always were, a reduction across the 128 keys on every CTA's first
         // tile).  Any finite reference gives the same result; only its headroom matters.
         if (L == 0) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) bars.red[0][q] = __uint_as_float(sr[q]) * c;
+          for (int q = 0; q < 16; ++q) bars.red[qh][q] = __uint_as_float(sr[q]) * c;
         }
-        softmax_sync();
+        softmax8_sync();
 #pragma unroll
-        for (int q = 0; q < 32; ++q) m[q] = bars.red[0][q];
-        softmax_sync();  // bars.red is rewritten below
+        for (int q = 0; q < 16; ++q) m[q] = bars.red[qh][q];
+        softmax8_sync();  // bars.red is rewritten below
       }
       float ymax = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));
-      if (softmax_any(ok && kv && !(ymax <= kLazy))) {
-        // Some query's reference must move: the tile's max per query over its valid keys.
-        float v[32];
+      for (int q = 0; q < 16; ++q) ymax = fmaxf(ymax, fmaf(__uint_as_float(sr[q]), c, -m[q]));
+      if (softmax8_any(ok && kv && !(ymax <= kLazy))) {
+        // Some query's reference must move: the tile's max per query over its valid keys (the
+        // four warps of the group, one lane quarter each).
+        float v[16];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = kv ? __uint_as_float(sr[q]) * c : -INFINITY;
-        bars.red[wr][lane] = reduce_scatter32<true>(v, lane);
-        softmax_sync();
-        float al[32];
+        for (int q = 0; q < 16; ++q) v[q] = kv ? __uint_as_float(sr[q]) * c : -INFINITY;
+        const float red = reduce_scatter16<true>(v, lane);
+        if (lane < 16) bars.red[wr][lane] = red;
+        softmax8_sync();
+        float al[16];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float tm = fmaxf(fmaxf(bars.red[0][q], bars.red[1][q]), fmaxf(bars.red[2][q], bars.red[3][q]));
+        for (int q = 0; q < 16; ++q) {
+          const float tm = fmaxf(fmaxf(bars.red[4 * qh][q], bars.red[4 * qh + 1][q]),
+                                 fmaxf(bars.red[4 * qh + 2][q], bars.red[4 * qh + 3][q]));
           const float mn = tm > m[q] + kLazy ? tm : m[q];
           al[q] = tc05::fast_exp2(m[q] - mn);  // 0 when m was -inf, 1 when it stays
           l[q] *= al[q];
           m[q] = mn;
         }
-        if (i > 0) {  // O^T holds the P V of the earlier tiles: rescale it
+        if (i > 0) {  // O^T holds the P V of the earlier tiles: rescale its columns of this group
           ok = __all_sync(FULL, ok && wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
           if (ok) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {  // the P_hi and P_lo column blocks
-              uint32_t o[32];
-              tc05::tmem_ld32(tmem + 64 + 32 * half + lane_off, o);
+              uint32_t o[16];
+              tc05::tmem_ld16(tmem + 64 + 32 * half + q0 + lane_off, o);
               tc05::tmem_wait_ld();
 #pragma unroll
-              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
-              tc05::tmem_st32(tmem + 64 + 32 * half + lane_off, o);
+              for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * al[q]);
+              tc05::tmem_st16(tmem + 64 + 32 * half + q0 + lane_off, o);
             }
             tc05::tmem_wait_st();
           }
         }
-        softmax_sync();  // bars.red is rewritten by the next tile
+        softmax8_sync();  // bars.red is rewritten by the next tile
       }
       // P = P_hi + P_lo, both bf16: query columns 0-31 of the P^T row hold P_hi and columns
       // 32-63 P_lo, so the one N = 64 MMA accumulates both and O^T's two column halves add up
       // to P V with P carried to ~16 significant bits (the cache itself is bf16 already).
-      uint32_t pk[16], pl[16];
+      uint32_t pk[8], pl[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const float p0 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j]), c, -m[2 * j])) : 0.f;
         const float p1 = kv ? tc05::fast_exp2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -m[2 * j + 1])) : 0.f;
         l[2 * j] += p0, l[2 * j + 1] += p1;
-        pk[j] = pack_bf16(p0, p1);  // query 2j in the low half
+        pk[j] = pack_bf16(p0, p1);  // query q0 + 2j in the low half
         pl[j] = pack_bf16(p0 - __uint_as_float(pk[j] << 16), p1 - __uint_as_float(pk[j] & 0xffff0000u));
       }
-      // P^T row L (the 128-byte-swizzled layout the MMA descriptor names) once P V of the
-      // previous tile has read the buffer.
+      // this group's 32 bytes of P_hi and of P_lo in P^T row L (the 128-byte-swizzled layout the
+      // MMA descriptor names: 16-byte chunk ch at (ch ^ (L % 8)) x 16), once P V of the previous
+      // tile has read the buffer
       if (i > 0) ok = __all_sync(FULL, ok && wait_or_abort(&bars.pfree, (i - 1) & 1, abort));
       if (ok) {
         uint8_t* row = sP + L * 128;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ch = 2 * qh + cc;
           *reinterpret_cast<uint4*>(row + ((ch ^ (L & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
           *reinterpret_cast<uint4*>(row + (((ch + 4) ^ (L & 7)) << 4)) =
-              make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+              make_uint4(pl[4 * cc], pl[4 * cc + 1], pl[4 * cc + 2], pl[4 * cc + 3]);
         }
       }
       tc05::fence_proxy_async_smem();  // P^T (generic stores) and O^T (tcgen05.st) before the MMA
@@ -919,38 +963,40 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       if (lane == 0) mbar_arrive(&bars.pfull);
     }
     // ---- slice done: the row sums over all 128 keys (while the last P V runs), then O^T
-    // column d = L of this thread
+    // column d = L of this thread, for the group's 16 queries
     {
-      float v[32];
+      float v[16];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = l[q];
-      bars.red[wr][lane] = reduce_scatter32<false>(v, lane);
+      for (int q = 0; q < 16; ++q) v[q] = l[q];
+      const float red = reduce_scatter16<false>(v, lane);
+      if (lane < 16) bars.red[wr][lane] = red;
     }
-    softmax_sync();
-    float lt[32];
+    softmax8_sync();
+    float lt[16];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) lt[q] = (bars.red[0][q] + bars.red[1][q]) + (bars.red[2][q] + bars.red[3][q]);
-    float o[32];
+    for (int q = 0; q < 16; ++q)
+      lt[q] = (bars.red[4 * qh][q] + bars.red[4 * qh + 1][q]) + (bars.red[4 * qh + 2][q] + bars.red[4 * qh + 3][q]);
+    float o[16];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) o[q] = 0.f;
+    for (int q = 0; q < 16; ++q) o[q] = 0.f;
     if (n > 0) {
       ok = __all_sync(FULL, ok && wait_or_abort(&bars.ofull, 0, abort));
       if (ok) {
-        uint32_t ohi[32], olo[32];
+        uint32_t ohi[16], olo[16];
         tc05::fence_after_sync();
-        tc05::tmem_ld32(tmem + 64 + lane_off, ohi);
-        tc05::tmem_ld32(tmem + 96 + lane_off, olo);
+        tc05::tmem_ld16(tmem + 64 + q0 + lane_off, ohi);
+        tc05::tmem_ld16(tmem + 96 + q0 + lane_off, olo);
         tc05::tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
+        for (int q = 0; q < 16; ++q) o[q] = __uint_as_float(ohi[q]) + __uint_as_float(olo[q]);
       }
     }
     if (k == 1) {
       // the whole (b, h) in this CTA: O = O^T / l
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        if (q >= a.n_act) continue;
-        const int64_t off = ((int64_t(b) * a.n_act + q) * a.H + h) * 128 + L;
+      for (int q = 0; q < 16; ++q) {
+        if (q0 + q >= a.n_act) continue;
+        const int64_t off = ((int64_t(b) * a.n_act + q0 + q) * a.H + h) * 128 + L;
         const float val = o[q] / lt[q];
         if (a.o_f32) static_cast<float*>(a.o)[off] = val;
         else static_cast<__nv_bfloat16*>(a.o)[off] = __float2bfloat16_rn(val);
@@ -962,20 +1008,20 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       // locally.  The P^T buffer (every P V is done) stages the partial as [32 queries][128].
       float* part = reinterpret_cast<float*>(sP);
 #pragma unroll
-      for (int q = 0; q < 32; ++q) part[q * 128 + L] = o[q];
-      if (wr == 0) {
+      for (int q = 0; q < 16; ++q) part[(q0 + q) * 128 + L] = o[q];
+      if (quarter == 0 && lane < 16) {  // one warp of each group: its queries' (m, l)
         float mm = -INFINITY, ll = 0.f;
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
+        for (int q = 0; q < 16; ++q)
           if (q == lane) mm = m[q], ll = lt[q];
-        bars.part_m[lane] = mm;
-        bars.part_l[lane] = ll;
+        bars.part_m[q0 + lane] = mm;
+        bars.part_l[q0 + lane] = ll;
       }
-      softmax_sync();
+      softmax8_sync();
       asm volatile("barrier.cluster.wait.acquire;" ::: "memory");  // every owner has armed rx_full
 #pragma unroll 1
-      for (int it = 0; it < 8; ++it) {  // chunk c: 16 bytes of row c / 32 (n_act <= 32 rows)
-        const int c = L + 128 * it, q = c >> 5, ch = c & 31;
+      for (int it = 0; it < 4; ++it) {  // chunk c: 16 bytes of row c / 32 (n_act <= 32 rows)
+        const int cidx = st_i + 256 * it, q = cidx >> 5, ch = cidx & 31;
         if (q >= a.n_act) continue;
         const int r = bars.row_owner[q];
         const float4 v = *reinterpret_cast<const float4*>(part + q * 128 + 4 * ch);
@@ -983,23 +1029,23 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
         if (r == rank) *reinterpret_cast<float4*>(dst) = v;
         else st_async4(peer_addr(dst, uint32_t(r)), v, peer_addr(&bars.rx_full, uint32_t(r)));
       }
-      if (L < a.n_act) {
-        const int r = bars.row_owner[L];
-        uint8_t* dst = rx + bars.ml_off[L];
-        if (r == rank) *reinterpret_cast<float2*>(dst) = make_float2(bars.part_m[L], bars.part_l[L]);
-        else st_async2(peer_addr(dst, uint32_t(r)), bars.part_m[L], bars.part_l[L], peer_addr(&bars.rx_full, uint32_t(r)));
+      if (st_i < a.n_act) {
+        const int r = bars.row_owner[st_i];
+        uint8_t* dst = rx + bars.ml_off[st_i];
+        if (r == rank) *reinterpret_cast<float2*>(dst) = make_float2(bars.part_m[st_i], bars.part_l[st_i]);
+        else st_async2(peer_addr(dst, uint32_t(r)), bars.part_m[st_i], bars.part_l[st_i], peer_addr(&bars.rx_full, uint32_t(r)));
       }
       wait_cluster(&bars.rx_full, 0, abort);  // every peer's rows for this CTA have landed
-      softmax_sync();                         // and this CTA's own copies
-      // merge rows [r0, r1): half-warp hw = 2 wr + lane / 16 takes rows hw, hw + 8, ... (one round
-      // for rows <= 8), its lane the columns 8 (lane % 16) .. + 7
+      softmax8_sync();                        // and this CTA's own copies
+      // merge rows [r0, r1): half-warp hw = 2 wr + lane / 16 takes rows hw, hw + 16, ... (one
+      // round for rows <= 16), its lane the columns 8 (lane % 16) .. + 7
       const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k, rows = r1 - r0;
       const float* rxo = reinterpret_cast<const float*>(rx);
       const float* rml = reinterpret_cast<const float*>(rx + k * rows * 512);
       const int hw = 2 * wr + (lane >> 4), c0 = 8 * (lane & 15);
       // (the merge and the sends above run once per CTA, from a cold instruction cache: their
       // loops stay rolled)
-      for (int j = hw; j < rows; j += 8) {
+      for (int j = hw; j < rows; j += 16) {
         float M = -INFINITY;
 #pragma unroll 1
         for (int p = 0; p < k; ++p) M = fmaxf(M, rml[2 * (p * rows + j)]);

@@ -240,25 +240,6 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-      "%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
@@ -495,14 +476,14 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
               }
               for (int qp2 = 0; qp2 < q; ++qp2) {  // P chunks of this tile already written
                 uint32_t pw[16];
-                tmem_ld16(tS + 16 * qp2, pw);
+                tc05::tmem_ld16(tS + 16 * qp2, pw);
                 tc05::tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                   const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pw[i]);
                   pw[i] = pack_p(__low2float(v) * alpha, __high2float(v) * alpha);
                 }
-                tmem_st16(tS + 16 * qp2, pw);
+                tc05::tmem_st16(tS + 16 * qp2, pw);
               }
               tc05::tmem_wait_st();
               m_ref = m_new;
@@ -516,7 +497,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
               }
             }
             l += csum;
-            tmem_st16(tS + 16 * q, pk);
+            tc05::tmem_st16(tS + 16 * q, pk);
           }
         }
         tc05::tmem_wait_st();

@@ -1438,6 +1438,13 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
   const int n = 1 + (part_r + 1) * part_nv / part_k - t0;  // n >= 1: k <= nv
   const int tpf = a.T / kKeys;
   const int64_t N = int64_t(a.F) * a.T;
+  // head-major row of the first key of video tile t of (b, h)
+  auto raw_row = [&](const TileWalk<kKeys>& w) {
+    const int vt = w.t - 1;
+    const int64_t tok = int64_t(a.fl.vlist[w.b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
+    return (int64_t(w.b) * a.H + w.h) * N + tok;
+  };
+  uint32_t pre = 0;  // bit i: raw tile i of the part requested before the dependency wait
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -1473,25 +1480,9 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     bars.part_r = part_r, bars.part_k = part_k;
     mbar_init(&bars.mfull, 1);
     fence_barrier_init();
-  }
-  if (warp == 1) {
-    tc05::tmem_alloc(&bars.tmem_base, kTmemCols);
-    tc05::tmem_relinquish();
-  }
-  tc05::fence_before_sync();
-  __syncthreads();
-  tc05::fence_after_sync();
-  const uint32_t tmem = bars.tmem_base;
-  // head-major row of the first key of video tile t of (b, h)
-  auto raw_row = [&](const TileWalk<kKeys>& w) {
-    const int vt = w.t - 1;
-    const int64_t tok = int64_t(a.fl.vlist[w.b * a.F + vt / tpf]) * a.T + (vt % tpf) * kKeys;
-    return (int64_t(w.b) * a.H + w.h) * N + tok;
-  };
-  // With a.fused_ready (the previous kernel does not write the NVFP4 pair) the first raw tiles
-  // are requested before the dependency wait; bit i of pre: tile i of the part.
-  uint32_t pre = 0;
-  if (threadIdx.x == 0) {
+    // Up to here only this CTA's shared memory was touched.  With a.fused_ready (the previous
+    // kernel does not write the NVFP4 pair) the part's first raw tiles are requested now, by
+    // the thread that set up their barriers, before the block-wide sync and the dependency wait.
     if (a.fused_ready) {
       TileWalk<kKeys> w;
       w.init_at(a, part_b, part_h, t0);
@@ -1509,6 +1500,14 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
       }
     }
   }
+  if (warp == 1) {
+    tc05::tmem_alloc(&bars.tmem_base, kTmemCols);
+    tc05::tmem_relinquish();
+  }
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  const uint32_t tmem = bars.tmem_base;
   grid_dependency_wait();
   grid_launch_dependents();
   // One register share per warpgroup, taken by all four of its warps at the top of its branch.

@@ -1598,7 +1598,8 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
         const uint32_t idS = idesc_f16_f32(128, 32, false, false);
-        const uint32_t idO = idesc_f16_f32(128, 64, true, true);
+        // N = 32: P is one fp16 part, in query columns 0-31 of each P^T row
+        const uint32_t idO = idesc_f16_f32(128, 32, true, true);
         TileWalk<kKeys> sw, pw;
         sw.init_at(a, part_b, part_h, t0);
         pw.init_at(a, part_b, part_h, t0);
@@ -1680,14 +1681,8 @@ action_nvfp4_kernel(const __grid_constant__ ActionArgs a, const __grid_constant_
     tw.init_at(a, part_b, part_h, t0);
     int seg = -1, i_first = 0;
     bool has_act = false, has_vid = false;  // accumulators written in this segment so far
-    // A P^T row holds P (fp16) in query columns 0-31 and zeros in 32-63: the fp16 P is kept
-    // whole (no low part), so O^T columns 32-63 stay zero and are never read.
-#pragma unroll
-    for (int buf = 0; buf < 2; ++buf) {
-#pragma unroll
-      for (int ch = 4; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(sP(buf) + L * 128 + ((ch ^ (L & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-    }
+    // A P^T row holds P (fp16, kept whole: no low part) in query columns 0-31, the first four
+    // 16-byte chunks of its 128-byte swizzled row; the P V MMA reads only those (N = 32).
     for (int i = 0; i < n; ++i, tw.next(a)) {
       if (i == 0 || tw.t == 0) {
         ++seg;

@@ -228,17 +228,6 @@ __device__ __forceinline__ uint32_t pack_p(float p0, float p1) {
   return pack_bf16(p0, p1);
 }
 
-// tcgen05.mma with A from tensor memory: D[tmem] (+)= A[tmem] * B[smem desc]^T.  A 16-bit A
-// operand keeps row m in TMEM lane m and elements 2i, 2i+1 of its K dimension in the low and
-// high half of column i.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -363,7 +352,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         const uint32_t v_s = smem_u32(sV(j % kVStages));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tO[w], tS[w] + 8 * kk, tc05::smem_desc_sw128(v_s + kk * 2048, kHalf, 1024), idO,
+          tc05::mma_ts(tO[w], tS[w] + 8 * kk, tc05::smem_desc_sw128(v_s + kk * 2048, kHalf, 1024), idO,
                  (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_bar(&bars.q_full, 0, abort) && wait_bar(&bars.k_full[0], 0, abort);

@@ -247,6 +247,38 @@ void order_items_for_tc(const Geo& g, wam::FrameLists& fl, int sms) {
   memo.in = in;
   memo.out.assign(fl.item, fl.item + n);
 }
+// Cross-frame pairing of a one-wave call.  When every CTA of a call is resident at once, its
+// time is that of the longest CTA, and a CTA normally takes two query tiles of one frame: the
+// frames with the most key frames set the time while the others finish early.  Paired, a CTA
+// takes the same query tile of two frames of one episode, one with the most key frames and
+// one with the fewest (items 2i and 2i + 1, fl.paired = 1): the second frame's keys are the
+// first entries of the first one's, so the two tiles share every key tile up to the end of
+// the shorter list, and only the rest runs for one tile.  Same number of CTAs; needs an even
+// number of 128-row query tiles per frame and of items per episode, and unequal key counts.
+void pair_items_for_tc(const Geo& g, wam::FrameLists& fl, int sms) {
+  fl.paired = 0;
+  const int QT = g.T / 128;
+  if (QT % 2 || sms <= 0 || fl.n_items < 2) return;
+  if (int64_t(fl.n_items) * (QT / 2) * g.H > sms) return;  // several waves: keep the order
+  std::vector<std::vector<uint32_t>> per(g.B);
+  for (int i = 0; i < fl.n_items; ++i) per[wam::item_b(fl.item[i])].push_back(fl.item[i]);
+  bool unequal = false;
+  for (auto& v : per) {
+    if (v.size() % 2) return;
+    std::stable_sort(v.begin(), v.end(),
+                     [](uint32_t x, uint32_t y) { return wam::item_nk(x) > wam::item_nk(y); });
+    if (!v.empty() && wam::item_nk(v.front()) != wam::item_nk(v.back())) unequal = true;
+  }
+  if (!unequal) return;
+  int k = 0;
+  for (auto& v : per)
+    for (size_t i = 0; i < v.size() / 2; ++i) {
+      fl.item[k++] = v[i];
+      fl.item[k++] = v[v.size() - 1 - i];
+    }
+  fl.paired = 1;
+}
+
 bool tc_action_ok(const Geo& g, wam_dtype dt, int n_act) {
   return dt == WAM_BF16 && g.D == 128 && g.T % 64 == 0 && n_act <= 32;
 }
@@ -426,6 +458,7 @@ wam_status wam_video_prefill_kv(const wam_video_layout* layout, wam_dtype dt, in
   const bool bf16 = dt == WAM_BF16;
   if (tc_video_ok(g, dt)) {
     order_items_for_tc(g, a.fl, sm_count());
+    pair_items_for_tc(g, a.fl, sm_count());
     cudaError_t e = wam::launch_prefill_tc(a, s);
     if (e != cudaErrorNotSupported) return cuda_status(e, "wam_video_prefill_kv (tensor cores)");
   }
@@ -657,7 +690,7 @@ wam_status wam_debug_action_plan(const wam_video_layout* layout, int32_t n_sms, 
 
 wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
                                    int32_t n_sms, int32_t* episode, int32_t* frame,
-                                   int32_t* n_key_frames, int32_t* n_items) {
+                                   int32_t* n_key_frames, int32_t* n_items, int32_t* paired) {
   Geo g;
   WAM_CHECK(check_layout(layout, g));
   WAM_CHECK(check_range(g, f_begin, f_end));
@@ -670,6 +703,8 @@ wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_beg
   fill_vlists(g, a.fl);
   fill_items(g, f_begin, f_end, a.fl);
   order_items_for_tc(g, a.fl, n_sms);
+  pair_items_for_tc(g, a.fl, n_sms);
+  if (paired) *paired = a.fl.paired;
   for (int i = 0; i < a.fl.n_items; ++i) {
     episode[i] = wam::item_b(a.fl.item[i]);
     frame[i] = wam::item_f(a.fl.item[i]);

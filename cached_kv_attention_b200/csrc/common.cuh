@@ -29,6 +29,7 @@ __host__ __device__ inline int item_nk(uint32_t it) { return int(it >> 21); }
 
 struct FrameLists {
   int32_t n_items;                               // prefill / store: valid query frames
+  int32_t paired;                                // tensor-core prefill: items (2i, 2i + 1) share CTAs
   uint32_t item[WAM_MAX_EPISODE_FRAMES];         // launch order (order_items_for_tc in api.cu)
   uint16_t vlist[WAM_MAX_EPISODE_FRAMES];        // valid frames of episode b at [b*F, ...)
   uint16_t nvalid[WAM_MAX_EPISODE_FRAMES];       // number of valid frames of episode b

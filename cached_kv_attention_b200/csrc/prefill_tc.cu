@@ -3,7 +3,8 @@
 //
 // One CTA computes up to 256 query tokens (two 128-row tiles Q0, Q1) of one (episode, frame,
 // head) against every key tile the block-causal predicate allows ("Long-WAM: Scaling the
-// Context of World-Action Models | Summary" §3.1-3.2).  T is a multiple of 128, so every
+// Context of World-Action Models | Summary" §3.1-3.2); or, when the host pairs the items of a
+// one-wave call, the same query tile of two frames of one episode, Q1's keys a prefix of Q0's.  T is a multiple of 128, so every
 // 128 x 128 tile is wholly visible or wholly masked: the host work list holds only visible key
 // frames and no element mask is applied.  Keys of frames below f_begin come from the layer's
 // cache, the others from the call's new K/V.  Each K/V tile loaded feeds both query tiles.
@@ -146,22 +147,25 @@ __device__ __forceinline__ void store_fuse_unit(const PrefillArgs& a, const void
 // time through a shared-memory counter by whole warps: the helper warps from the start, each
 // softmax warp once its output is written, so a CTA with few key tiles does not wait on two
 // warps for its epilogue.  `rows` (a multiple of 8) own tokens from row_in / row_out.
-__device__ __forceinline__ void store_fuse_pool(const PrefillArgs& a, int* next, int rows,
-                                                int64_t row_in, int64_t row_out, int h,
-                                                int lane) {
+__device__ __forceinline__ void store_fuse_pool(const PrefillArgs& a, int* next, int nq,
+                                                int64_t in0, int64_t in1, int64_t out0,
+                                                int64_t out1, int h, int lane) {
   if (a.k_store == nullptr && !a.fuse_on) return;
-  const int per = rows / 8;
+  constexpr int kPerTile = kBM / 8;  // units of one query tile's rows, of K or of V
+  const int per = nq * kPerTile;
   for (;;) {
     int u = 0;
     if (lane == 0) u = atomicAdd(next, 1);
     u = __shfl_sync(0xffffffffu, u, 0);
     if (u >= 2 * per) break;
-    if (u < per)
-      store_fuse_unit(a, a.k_new, a.k_store, a.acc_k, a.fused_k, row_in + 8 * u,
-                      row_out + 8 * u, h, lane);
+    const bool is_v = u >= per;
+    const int uu = is_v ? u - per : u, r0 = 8 * (uu % kPerTile);
+    const bool t1 = uu >= kPerTile;  // rows of query tile 1
+    const int64_t ri = (t1 ? in1 : in0) + r0, ro = (t1 ? out1 : out0) + r0;
+    if (!is_v)
+      store_fuse_unit(a, a.k_new, a.k_store, a.acc_k, a.fused_k, ri, ro, h, lane);
     else
-      store_fuse_unit(a, a.v_new, a.v_store, a.acc_v, a.fused_v, row_in + 8 * (u - per),
-                      row_out + 8 * (u - per), h, lane);
+      store_fuse_unit(a, a.v_new, a.v_store, a.acc_v, a.fused_v, ri, ro, h, lane);
   }
 }
 
@@ -247,17 +251,38 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   Bars& bars = *reinterpret_cast<Bars*>(base + (2 + kKStages + kVStages) * kTile);
   volatile int* abort = &bars.abort;
 
-  // ---- work item: query tiles 2 qp and 2 qp + 1 of frame f (the second may not exist)
+  // ---- work item: query tiles 2 qp and 2 qp + 1 of frame f (the second may not exist), or,
+  // with a.fl.paired, query tile qt of both frames of the item pair (2 i, 2 i + 1) of one
+  // episode: the first reads nk_0 key frames, the second nk_1 <= nk_0, the first nk_1 of the
+  // same list, so every key tile loaded feeds both tiles until the second one's keys end.
   const int QT = a.T / kBM, QP = (QT + 1) / 2;
   const int h = int(blockIdx.x % a.H);
   const int rest = int(blockIdx.x / a.H);
-  const int qp = rest % QP;
-  const uint32_t it = a.fl.item[rest / QP];
-  const int b = item_b(it), f = item_f(it), nk = item_nk(it);
-  const int nq = (2 * qp + 1 < QT) ? 2 : 1;            // query tiles in this CTA
   const int tpf = a.T / kBN;
-  const int n = nk * tpf;                               // key tiles
-  const int qtok0 = (f - a.f_begin) * a.T + qp * 2 * kBM;
+  // (scalars per query tile, selected by w: no local-memory arrays)
+  int b, f0, f1, nk0, nk1, qt0, qt1, nq;
+  if (a.fl.paired) {
+    const uint32_t i0 = a.fl.item[2 * (rest / QT)], i1 = a.fl.item[2 * (rest / QT) + 1];
+    b = item_b(i0);
+    f0 = item_f(i0), f1 = item_f(i1);
+    nk0 = item_nk(i0), nk1 = item_nk(i1);
+    qt0 = qt1 = rest % QT;
+    nq = 2;
+  } else {
+    const int qp = rest % QP;
+    const uint32_t it = a.fl.item[rest / QP];
+    b = item_b(it);
+    f0 = f1 = item_f(it);
+    nk0 = nk1 = item_nk(it);
+    qt0 = 2 * qp, qt1 = 2 * qp + 1;
+    nq = (2 * qp + 1 < QT) ? 2 : 1;                     // query tiles in this CTA
+  }
+  const int n = nk0 * tpf;                              // key tiles (of the first query tile)
+  auto nw = [&](int w) { return (w ? nk1 : nk0) * tpf; };  // key tiles of query tile w
+  auto fw = [&](int w) { return w ? f1 : f0; };
+  auto qtw = [&](int w) { return w ? qt1 : qt0; };
+  // first token of query tile w among the call's query tokens
+  auto qtokw = [&](int w) { return (fw(w) - a.f_begin) * a.T + qtw(w) * kBM; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   auto key_tile = [&](int j, bool& old, int& tok) {
@@ -305,8 +330,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       int k_issued = 0, v_issued = 0;
       mbar_arrive_expect_tx(&bars.q_full, nq * kTile);
       for (int w = 0; w < nq; ++w) {
-        tma_load_4d(sQ(w), &maps.q, &bars.q_full, 0, h, qtok0 + w * kBM, b);
-        tma_load_4d(sQ(w) + kHalf, &maps.q, &bars.q_full, 64, h, qtok0 + w * kBM, b);
+        tma_load_4d(sQ(w), &maps.q, &bars.q_full, 0, h, qtokw(w), b);
+        tma_load_4d(sQ(w) + kHalf, &maps.q, &bars.q_full, 64, h, qtokw(w), b);
       }
       for (int j = 0; j < n; ++j) {
         bool old;
@@ -370,11 +395,12 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         if (more && !wait_bar(&bars.k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, abort)) break;
         bool fail = false;
         for (int w = 0; w < nq; ++w) {
+          if (j >= nw(w)) continue;  // this query tile's keys have ended
           if (!wait_bar(&bars.p_full[w], j & 1, abort)) { fail = true; break; }
           tc05::fence_after_sync();
           issue_PV(w, j);
-          if (j == n - 1) tc05::mma_commit(&bars.o_full[w]);
-          if (more) {
+          if (j == nw(w) - 1) tc05::mma_commit(&bars.o_full[w]);
+          if (j + 1 < nw(w)) {
             issue_S(w, j + 1);
             tc05::mma_commit(&bars.s_full[w]);
           }
@@ -398,7 +424,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       const float c = a.scale_log2;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < n; ++j) {
+      const int n_own = nw(w);
+      for (int j = 0; j < n_own; ++j) {
         ok = __all_sync(FULL, ok && wait_bar(&bars.s_full[w], j & 1, abort));
         if (!ok) continue;
         tc05::fence_after_sync();
@@ -500,7 +527,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         tc05::fence_after_sync();
         const float inv = 1.f / l;
         const int64_t qtok = int64_t(a.f_end - a.f_begin) * a.T;
-        const int64_t row = int64_t(b) * qtok + qtok0 + w * kBM + r;
+        const int64_t row = int64_t(b) * qtok + qtokw(w) + r;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
@@ -534,10 +561,11 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     // The CTA's own tokens, read from the call's new K/V: the helper warps start at once, while
     // the attention loop runs; each softmax warp joins once its output is written (converged:
     // every branch in the softmax is warp-uniform).
-    // first own token row in the call's new K/V and in the layer's cache
-    const int64_t own_in = int64_t(b) * (int64_t(a.f_end - a.f_begin) * a.T) + qtok0;
-    const int64_t own_out = int64_t(b) * (int64_t(a.F) * a.T) + int64_t(f) * a.T + qp * 2 * kBM;
-    store_fuse_pool(a, &bars.unit_next, nq * kBM, own_in, own_out, h, lane);
+    // first own token row of query tile w in the call's new K/V and in the layer's cache
+    const int64_t in0 = int64_t(b) * (int64_t(a.f_end - a.f_begin) * a.T);
+    const int64_t out0 = int64_t(b) * (int64_t(a.F) * a.T);
+    store_fuse_pool(a, &bars.unit_next, nq, in0 + qtokw(0), in0 + qtokw(1),
+                    out0 + int64_t(f0) * a.T + qt0 * kBM, out0 + int64_t(f1) * a.T + qt1 * kBM, h, lane);
   }
 
   // ------------------------------------------------------------ teardown
@@ -573,8 +601,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   // go stale across devices, threads or a device reset.
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int QP = (a.T / kBM + 1) / 2;
-  const int64_t grid = int64_t(a.fl.n_items) * QP * a.H;
+  const int QT = a.T / kBM, QP = (QT + 1) / 2;
+  const int64_t grid = a.fl.paired ? int64_t(a.fl.n_items / 2) * QT * a.H : int64_t(a.fl.n_items) * QP * a.H;
   return launch_pdl(prefill_tc_kernel, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);
 }
 

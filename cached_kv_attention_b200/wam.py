@@ -70,7 +70,7 @@ def _load() -> ctypes.CDLL:
         "wam_fuse_weights": [i32, ctypes.POINTER(f32), ctypes.POINTER(f32)],
         "wam_debug_video_mask": [lay, i32, i32, vp, vp],
         "wam_debug_prefill_order": [lay, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
-                                    ctypes.POINTER(i32), ctypes.POINTER(i32)],
+                                    ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "wam_device_error": [i32],
         "wam_debug_wait_timeout": [i32, vp],
         "wam_debug_action_plan": [lay, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
@@ -284,16 +284,21 @@ def debug_video_mask(layout: VideoLayout, f_begin: int, f_end: int, stream=None)
     return mask
 
 
-def debug_prefill_order(layout: VideoLayout, f_begin: int, f_end: int, n_sms: int):
+def debug_prefill_order(layout: VideoLayout, f_begin: int, f_end: int, n_sms: int,
+                        with_pairing: bool = False):
     """Work items of a tensor-core prefill call over [f_begin, f_end) in launch order for a
-    device of n_sms SMs (host only): int32 arrays (episode, frame, n_key_frames)."""
+    device of n_sms SMs (host only): int32 arrays (episode, frame, n_key_frames), and with
+    with_pairing also whether items (2i, 2i + 1) share CTAs."""
     cap = max(layout.B * (f_end - f_begin), 1)
     ep, fr, nk = (np.zeros(cap, dtype=np.int32) for _ in range(3))
     n = ctypes.c_int32(0)
+    paired = ctypes.c_int32(0)
     P = ctypes.POINTER(ctypes.c_int32)
     check(lib.wam_debug_prefill_order(layout.ref, f_begin, f_end, n_sms, ep.ctypes.data_as(P),
-                                      fr.ctypes.data_as(P), nk.ctypes.data_as(P), ctypes.byref(n)))
-    return ep[:n.value], fr[:n.value], nk[:n.value]
+                                      fr.ctypes.data_as(P), nk.ctypes.data_as(P), ctypes.byref(n),
+                                      ctypes.byref(paired)))
+    out = ep[:n.value], fr[:n.value], nk[:n.value]
+    return out + (bool(paired.value),) if with_pairing else out
 
 
 def nvfp4_workspace_size(n: int) -> int:

@@ -329,13 +329,18 @@ wam_status wam_debug_video_mask(const wam_video_layout* layout, int32_t f_begin,
  * The order starts from longest first; each class of equal key-frame count is also tried right
  * behind the longest class and at the end, every candidate is scored by replaying in-order
  * dispatch of its CTAs onto n_sms SMs (cost per CTA: key tiles + 5), and the cheapest is
- * kept (longest first on ties; n_sms <= 0, or a single wave, keeps longest first).
+ * kept (longest first on ties; n_sms <= 0, or a single wave, keeps longest first).  A single
+ * wave whose frames hold an even number of 128-row query tiles, and whose episodes each hold
+ * an even number of items of unequal key-frame counts, is instead paired: within each
+ * episode the items with most and fewest key frames become items 2i and 2i + 1, and each CTA
+ * of a pair takes the same query tile of both frames (T / 128 x H CTAs per pair).
  *   episode, frame, n_key_frames: host int32 arrays with room for B * (f_end - f_begin);
- *   *n_items receives the number of items written.
+ *   *n_items receives the number of items written; *paired (may be NULL) receives 1 for a
+ *   paired order, else 0.
  */
 wam_status wam_debug_prefill_order(const wam_video_layout* layout, int32_t f_begin, int32_t f_end,
                                    int32_t n_sms, int32_t* episode, int32_t* frame,
-                                   int32_t* n_key_frames, int32_t* n_items);
+                                   int32_t* n_key_frames, int32_t* n_items, int32_t* paired);
 
 /*
  * Failure-detection check: launches one warp that waits on a shared-memory mbarrier nothing

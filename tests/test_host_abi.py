@@ -170,13 +170,17 @@ def test_debug_prefill_order_rejects_bad_arguments():
     lay = _lay(B=1, H=2, D=128, T=256, F=4)
     out = [(ctypes.c_int32 * 8)() for _ in range(3)]
     n = ctypes.c_int32(-1)
-    call = lambda f0=0, f1=4, ep=out[0], fr=out[1], nk=out[2], cnt=ctypes.byref(n): \
-        L.wam_debug_prefill_order(lay.ref, f0, f1, 148, ep, fr, nk, cnt)
+    paired = ctypes.c_int32(-1)
+    call = lambda f0=0, f1=4, ep=out[0], fr=out[1], nk=out[2], cnt=ctypes.byref(n), pr=None: \
+        L.wam_debug_prefill_order(lay.ref, f0, f1, 148, ep, fr, nk, cnt, pr)
     assert call(f0=2, f1=2) == 1 and "frame range" in _msg()
     assert call(ep=None) == 1 and "NULL" in _msg()
     assert call(cnt=None) == 1 and "NULL" in _msg()
     bad_t = _lay(B=1, H=2, D=128, T=64, F=4)
     assert L.wam_debug_prefill_order(bad_t.ref, 0, 4, 148, out[0], out[1], out[2],
-                                     ctypes.byref(n)) == 1 and "multiple of 128" in _msg()
-    assert call() == 0 and n.value == 4             # host only: valid without a GPU
-    assert list(out[2])[:4] == [4, 3, 2, 1] and list(out[1])[:4] == [3, 2, 1, 0]
+                                     ctypes.byref(n), None) == 1 and "multiple of 128" in _msg()
+    # host only: valid without a GPU.  8 CTAs on 148 SMs, 2 query tiles per frame, 4 items of
+    # 4, 3, 2 and 1 key frames: paired, most with fewest
+    assert call(pr=ctypes.byref(paired)) == 0 and n.value == 4 and paired.value == 1
+    assert list(out[2])[:4] == [4, 1, 3, 2] and list(out[1])[:4] == [3, 0, 2, 1]
+    assert call() == 0 and n.value == 4             # the pairing flag is optional

@@ -120,3 +120,80 @@ def test_repeated_and_alternating_calls_give_the_same_orders():
             assert got == first[(name, sms)]
             again = [a.tolist() for a in wam.debug_prefill_order(lay, f0, w.F_h, sms)]
             assert again == got
+
+
+# ---- cross-frame pairing of one-wave calls
+
+
+def test_one_wave_imagination_pass_pairs_its_two_frames():
+    # 19.2 s: the 2 imagined frames read 7 and 6 key frames; 2 items x 3 CTAs x 24 heads = 144
+    # CTAs fit on 148 SMs, so each CTA takes the same query tile of both frames
+    w, lay = layout_of("ctx19.2s_bf16")
+    ep, fr, nk, paired = wam.debug_prefill_order(lay, w.F_h, w.F, B200_SMS, with_pairing=True)
+    assert paired
+    assert list(ep) == [0, 0] and list(fr) == [w.F_h + 1, w.F_h] and list(nk) == [7, 6]
+
+
+def test_multi_wave_calls_are_not_paired():
+    w, lay = layout_of("ctx19.2s_bf16")
+    assert not wam.debug_prefill_order(lay, 0, w.F_h, B200_SMS, with_pairing=True)[3]  # 360 CTAs
+    assert not wam.debug_prefill_order(lay, w.F_h, w.F, 16, with_pairing=True)[3]      # 16 SMs
+    assert not wam.debug_prefill_order(lay, w.F_h, w.F, 0, with_pairing=True)[3]
+
+
+def _expected_pairing(ep, nk, T, H, sms):
+    """The pairing rule restated: a one-wave call (all CTAs resident), an even number of
+    128-row query tiles per frame, an even number of items in every episode, and some episode
+    whose items read unequal numbers of key frames."""
+    QT = T // 128
+    n = len(ep)
+    if QT % 2 or sms <= 0 or n < 2 or n * (QT // 2) * H > sms:
+        return False
+    per = {}
+    for b, k in zip(ep.tolist(), nk.tolist()):
+        per.setdefault(b, []).append(k)
+    if any(len(v) % 2 for v in per.values()):
+        return False
+    return any(max(v) != min(v) for v in per.values())
+
+
+def _random_call(seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 4))
+    H = int(rng.choice([1, 2, 4, 24]))
+    T = int(rng.choice([128, 256, 384, 512, 768]))
+    F = int(rng.integers(2, 9))
+    pad = (rng.random((B, F)) < 0.3).astype(np.uint8)
+    pad[:, -1] = 0
+    lay = wam.VideoLayout(B, H, 128, T, F, pad)
+    f0 = int(rng.integers(0, F - 1))
+    sms = int(rng.choice([0, 16, B200_SMS, 1000, 1000]))
+    return lay, f0, F, sms, T, H
+
+
+@pytest.mark.parametrize("seed", range(48))
+def test_pairing_rule_and_pairs(seed):
+    lay, f0, F, sms, T, H = _random_call(seed)
+    ep, fr, nk, paired = wam.debug_prefill_order(lay, f0, F, sms, with_pairing=True)
+    ep0, fr0, nk0 = wam.debug_prefill_order(lay, f0, F, 0)
+    assert paired == _expected_pairing(ep0, nk0, T, H, sms)
+    # always a permutation of the longest-first items
+    assert sorted(zip(ep.tolist(), fr.tolist(), nk.tolist())) == \
+        sorted(zip(ep0.tolist(), fr0.tolist(), nk0.tolist()))
+    if not paired:
+        return
+    # pairs (2i, 2i + 1): one episode, the first reading at least the second's key frames; in
+    # each episode the i-th most with the i-th fewest
+    per = {}
+    for i in range(0, len(ep), 2):
+        assert ep[i] == ep[i + 1] and nk[i] >= nk[i + 1]
+        per.setdefault(int(ep[i]), []).append((int(nk[i]), int(nk[i + 1])))
+    for b, pairs in per.items():
+        ks = sorted((int(k) for e, k in zip(ep0, nk0) if e == b), reverse=True)
+        assert sorted(pairs, reverse=True) == [(ks[i], ks[-1 - i]) for i in range(len(ks) // 2)]
+
+
+def test_pairing_cases_are_exercised():
+    # the random calls above include paired and unpaired ones
+    flags = [wam.debug_prefill_order(*_random_call(s)[:4], with_pairing=True)[3] for s in range(48)]
+    assert 5 <= sum(flags) <= 43

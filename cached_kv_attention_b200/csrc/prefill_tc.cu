@@ -147,12 +147,31 @@ __device__ __forceinline__ void store_fuse_unit(const PrefillArgs& a, const void
 // time through a shared-memory counter by whole warps: the helper warps from the start, each
 // softmax warp once its output is written, so a CTA with few key tiles does not wait on two
 // warps for its epilogue.  `rows` (a multiple of 8) own tokens from row_in / row_out.
-__device__ __forceinline__ void store_fuse_pool(const PrefillArgs& a, int* next, int nq,
-                                                int64_t in0, int64_t in1, int64_t out0,
-                                                int64_t out1, int h, int lane) {
+__device__ __forceinline__ void store_fuse_pool(const PrefillArgs& a, int* next, int rows,
+                                                int64_t row_in, int64_t row_out, int h,
+                                                int lane) {
+  if (a.k_store == nullptr && !a.fuse_on) return;
+  const int per = rows / 8;
+  for (;;) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(next, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= 2 * per) break;
+    if (u < per)
+      store_fuse_unit(a, a.k_new, a.k_store, a.acc_k, a.fused_k, row_in + 8 * u,
+                      row_out + 8 * u, h, lane);
+    else
+      store_fuse_unit(a, a.v_new, a.v_store, a.acc_v, a.fused_v, row_in + 8 * (u - per),
+                      row_out + 8 * (u - per), h, lane);
+  }
+}
+// The same for a cross-frame pair: the rows of the two query tiles are not contiguous.
+__device__ __forceinline__ void store_fuse_pool_pair(const PrefillArgs& a, int* next,
+                                                     int64_t in0, int64_t in1, int64_t out0,
+                                                     int64_t out1, int h, int lane) {
   if (a.k_store == nullptr && !a.fuse_on) return;
   constexpr int kPerTile = kBM / 8;  // units of one query tile's rows, of K or of V
-  const int per = nq * kPerTile;
+  const int per = 2 * kPerTile;
   for (;;) {
     int u = 0;
     if (lane == 0) u = atomicAdd(next, 1);
@@ -234,6 +253,9 @@ __device__ __forceinline__ uint32_t pack_p(float p0, float p1) {
 
 
 
+// kPaired: the call's items are cross-frame pairs (a.fl.paired); a separate instantiation, so
+// that the per-tile key counts and token offsets of a pair cost nothing in unpaired calls.
+template <bool kPaired>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   // the tensor maps' descriptors first, hidden behind the set-up below (parameter space: the
@@ -261,7 +283,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const int tpf = a.T / kBN;
   // (scalars per query tile, selected by w: no local-memory arrays)
   int b, f0, f1, nk0, nk1, qt0, qt1, nq;
-  if (a.fl.paired) {
+  if constexpr (kPaired) {
     const uint32_t i0 = a.fl.item[2 * (rest / QT)], i1 = a.fl.item[2 * (rest / QT) + 1];
     b = item_b(i0);
     f0 = item_f(i0), f1 = item_f(i1);
@@ -278,11 +300,15 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     nq = (2 * qp + 1 < QT) ? 2 : 1;                     // query tiles in this CTA
   }
   const int n = nk0 * tpf;                              // key tiles (of the first query tile)
-  auto nw = [&](int w) { return (w ? nk1 : nk0) * tpf; };  // key tiles of query tile w
-  auto fw = [&](int w) { return w ? f1 : f0; };
-  auto qtw = [&](int w) { return w ? qt1 : qt0; };
-  // first token of query tile w among the call's query tokens
-  auto qtokw = [&](int w) { return (fw(w) - a.f_begin) * a.T + qtw(w) * kBM; };
+  // key tiles of query tile w, and its first token among the call's query tokens
+  auto nw = [&](int w) {
+    if constexpr (kPaired) return (w ? nk1 : nk0) * tpf;
+    else return n;
+  };
+  auto qtokw = [&](int w) {
+    if constexpr (kPaired) return ((w ? f1 : f0) - a.f_begin) * a.T + (w ? qt1 : qt0) * kBM;
+    else return (f0 - a.f_begin) * a.T + (qt0 + w) * kBM;
+  };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   auto key_tile = [&](int j, bool& old, int& tok) {
@@ -564,8 +590,12 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     // first own token row of query tile w in the call's new K/V and in the layer's cache
     const int64_t in0 = int64_t(b) * (int64_t(a.f_end - a.f_begin) * a.T);
     const int64_t out0 = int64_t(b) * (int64_t(a.F) * a.T);
-    store_fuse_pool(a, &bars.unit_next, nq, in0 + qtokw(0), in0 + qtokw(1),
-                    out0 + int64_t(f0) * a.T + qt0 * kBM, out0 + int64_t(f1) * a.T + qt1 * kBM, h, lane);
+    if constexpr (kPaired)
+      store_fuse_pool_pair(a, &bars.unit_next, in0 + qtokw(0), in0 + qtokw(1),
+                           out0 + int64_t(f0) * a.T + qt0 * kBM, out0 + int64_t(f1) * a.T + qt1 * kBM, h, lane);
+    else
+      store_fuse_pool(a, &bars.unit_next, nq * kBM, in0 + qtokw(0), out0 + int64_t(f0) * a.T + qt0 * kBM, h,
+                      lane);
   }
 
   // ------------------------------------------------------------ teardown
@@ -599,11 +629,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   }
   // Set on every call (a host-side attribute write, no device work): nothing cached here can
   // go stale across devices, threads or a device reset.
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int QT = a.T / kBM, QP = (QT + 1) / 2;
   const int64_t grid = a.fl.paired ? int64_t(a.fl.n_items / 2) * QT * a.H : int64_t(a.fl.n_items) * QP * a.H;
-  return launch_pdl(prefill_tc_kernel, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);
+  if (a.fl.paired)
+    return launch_pdl(prefill_tc_kernel<true>, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);
+  return launch_pdl(prefill_tc_kernel<false>, dim3(unsigned(grid)), dim3(kThreads), kSmemBytes, s, 0, a, maps);
 }
 
 }  // namespace wam

@@ -459,21 +459,22 @@ action_tc_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__ A
 //   O^T += V^T P^T M = D = 128, N = 64 (32 query columns of P_hi, 32 of P_lo), K = 128 keys;
 //                  V^T is the MN-major view of the V tile as TMA wrote it, P^T a tile of
 //                  128-byte rows.
-// S^T (two buffers) and O^T live in tensor memory.  One softmax thread per key reads its 32
-// scores; each query keeps one reference max, shared by all threads, that moves (with O^T and
-// the row sums rescaled) only when a tile exceeds it by more than 2^16, which one OR-reduction
-// barrier per tile detects.
+// S^T (two buffers) and O^T live in tensor memory.  Two softmax warpgroups: a thread takes one
+// key (its TMEM lane) and the 16 queries of its group; each query keeps one reference max,
+// shared by all threads, that moves (with O^T and the row sums rescaled) only when a tile
+// exceeds it by more than 2^16, which one OR-reduction barrier per tile detects.
 //
 // Work split: one thread-block cluster of k <= 8 CTAs per (episode, head); CTA r of the
 // cluster streams the r-th of k contiguous slices of the (episode, head)'s tiles (the action
 // tile first, then the valid frames' tiles).  The k partials (O, m, l) meet in distributed
-// shared memory and never leave the chip: CTA r owns query rows [r n_act / k, (r+1) n_act / k).
-// Once its MMAs are done its K/V stage buffers are free, and it tells its peers so (a release
-// arrive on each peer's barrier); every CTA then writes its partial rows straight into their
-// owners' stage buffers (shared::cluster stores, released by one arrive per owner) and merges
-// its own rows from local memory.  One one-way hop follows the slowest slice, and no CTA waits
-// on another before leaving.
-// Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-5 softmax (TMEM lane quarters 2, 3, 0, 1).
+// shared memory and never leave the chip: CTA r owns query rows [r n_act / k, (r+1) n_act / k)
+// and keeps a receive region for them, whose barrier it arms at start with every byte its
+// peers will send.  After its loop a CTA sends each partial row to its owner with st.async
+// stores counted on that barrier (its own rows are copied locally), then waits for its rows
+// from every peer and merges them.  One one-way hop follows the slowest slice, and no CTA
+// waits on another before leaving.
+// Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-9 softmax (warp w: TMEM lane quarter
+// w % 4, query group (w - 2) / 4).
 namespace um {
 constexpr int kKeys = 128;
 constexpr int kTile = kKeys * 128 * 2;   // one of K or V: 32 KB

@@ -1038,46 +1038,45 @@ action_umma_kernel(const __grid_constant__ ActionArgs a, const __grid_constant__
       }
       wait_cluster(&bars.rx_full, 0, abort);  // every peer's rows for this CTA have landed
       softmax8_sync();                        // and this CTA's own copies
-      // merge rows [r0, r1): half-warp hw = 2 wr + lane / 16 takes rows hw, hw + 16, ... (one
-      // round for rows <= 16), its lane the columns 8 (lane % 16) .. + 7
+      // merge rows [r0, r1): warp wr takes rows wr, wr + 8, ... (one round for rows <= 8), lane l
+      // the columns 4 l .. 4 l + 3; lane p < k loads slot p's (m, l) pair and the warp shares
+      // its weight, so each thread loads one 16-byte chunk per slot and takes one exponential
       const int r0 = rank * a.n_act / k, r1 = (rank + 1) * a.n_act / k, rows = r1 - r0;
       const float* rxo = reinterpret_cast<const float*>(rx);
       const float* rml = reinterpret_cast<const float*>(rx + k * rows * 512);
-      const int hw = 2 * wr + (lane >> 4), c0 = 8 * (lane & 15);
       // (the merge and the sends above run once per CTA, from a cold instruction cache: their
       // loops stay rolled)
-      for (int j = hw; j < rows; j += 16) {
-        float M = -INFINITY;
-#pragma unroll 1
-        for (int p = 0; p < k; ++p) M = fmaxf(M, rml[2 * (p * rows + j)]);
+      for (int j = wr; j < rows; j += 8) {
+        const float2 ml = lane < k ? *reinterpret_cast<const float2*>(rml + 2 * (lane * rows + j))
+                                   : make_float2(-INFINITY, 0.f);
+        float M = ml.x;  // max over lanes 0 .. 7 (k <= 8), then lane 0's to all
+        M = fmaxf(M, __shfl_xor_sync(FULL, M, 1));
+        M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
+        M = fmaxf(M, __shfl_xor_sync(FULL, M, 4));
+        M = __shfl_sync(FULL, M, 0);
         const float Mu = M == -INFINITY ? 0.f : M;
-        float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
+        const float wl = lane < k ? tc05::fast_exp2(ml.x - Mu) : 0.f;  // slot `lane`'s weight
+        float den = wl * ml.y;
+        den += __shfl_xor_sync(FULL, den, 1);
+        den += __shfl_xor_sync(FULL, den, 2);
+        den += __shfl_xor_sync(FULL, den, 4);
+        den = __shfl_sync(FULL, den, 0);
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
         for (int p = 0; p < k; ++p) {
-          const float2 ml = *reinterpret_cast<const float2*>(rml + 2 * (p * rows + j));
-          const float4 pa = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0);
-          const float4 pb = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + c0 + 4);
-          const float wgt = tc05::fast_exp2(ml.x - Mu);
-          den = fmaf(wgt, ml.y, den);
-          num[0] = fmaf(wgt, pa.x, num[0]), num[1] = fmaf(wgt, pa.y, num[1]);
-          num[2] = fmaf(wgt, pa.z, num[2]), num[3] = fmaf(wgt, pa.w, num[3]);
-          num[4] = fmaf(wgt, pb.x, num[4]), num[5] = fmaf(wgt, pb.y, num[5]);
-          num[6] = fmaf(wgt, pb.z, num[6]), num[7] = fmaf(wgt, pb.w, num[7]);
+          const float wgt = __shfl_sync(FULL, wl, p);
+          const float4 x = *reinterpret_cast<const float4*>(rxo + (p * rows + j) * 128 + 4 * lane);
+          num.x = fmaf(wgt, x.x, num.x), num.y = fmaf(wgt, x.y, num.y);
+          num.z = fmaf(wgt, x.z, num.z), num.w = fmaf(wgt, x.w, num.w);
         }
         const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
-        float val[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) val[e] = num[e] * inv;
-        const int64_t off = ((int64_t(b) * a.n_act + r0 + j) * a.H + h) * 128 + c0;
-        if (a.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + off);
-          dst[0] = make_float4(val[0], val[1], val[2], val[3]);
-          dst[1] = make_float4(val[4], val[5], val[6], val[7]);
-        } else {
-          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + off) =
-              make_uint4(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]), pack_bf16(val[4], val[5]),
-                         pack_bf16(val[6], val[7]));
-        }
+        const int64_t off = ((int64_t(b) * a.n_act + r0 + j) * a.H + h) * 128 + 4 * lane;
+        if (a.o_f32)
+          *reinterpret_cast<float4*>(static_cast<float*>(a.o) + off) =
+              make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+        else
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + off) =
+              make_uint2(pack_bf16(num.x * inv, num.y * inv), pack_bf16(num.z * inv, num.w * inv));
       }
     }
   }

@@ -391,7 +391,7 @@ IMAG_TRAFFIC_BYTES = {"ctx19.2s_bf16": 80.47e6}
 # The same for one fused-cache action read (`bench.py --profile-call action`, and
 # `--workload nvfp4_ctx19.2s_bf16 --profile-call action_nvfp4` for the NVFP4 read); the stride
 # variants issue the identical bf16 read.
-ACTION_TRAFFIC_BYTES = {"ctx19.2s_bf16": 67.74e6, "nvfp4_ctx19.2s_bf16": 19.27e6}
+ACTION_TRAFFIC_BYTES = {"ctx19.2s_bf16": 67.70e6, "nvfp4_ctx19.2s_bf16": 19.27e6}
 
 
 def time_fused_read(runner, stream, n=20) -> float:

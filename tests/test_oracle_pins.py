@@ -393,90 +393,151 @@ def _bf_attend(q, keys, vals):
     return [sum(e[j] * vals[j][d] for j in range(len(keys))) / z for d in range(len(vals[0]))]
 
 
-def _bf_chunk(inp, pad, L, S, T, Fh, Ff, Nv, Ne, sigma_star):
-    """One chunk restated from the readings with loops and math.exp, calling nothing of the
-    oracle: the history pass over frames [0, Fh) (a query of frame f reads every non-padded
-    frame <= f, R2-R3; padded query frames stay 0), its K/V stored for non-padded frames; Nv
-    imagination passes over the stored history and their own future K/V, each followed by an
-    Euler step of -(1 - sigma*) / Nv on the future latents (R1, R7); the final pass, its K/V
-    stored (R6); intervals I_m = {S m, ..}, fused pair m = sum of w_m,j x cache_j (R5); Ne action
-    steps where layer max(I_m) reads the non-padded frames of fused pair m before the action keys
-    and other layers read the action keys only (R5, R9), each followed by an Euler step of
-    -1 / Ne."""
-    F = Fh + Ff
+def _bf_video(q, kn, vn, kc, vc, f0, f1, pad, T):
+    """A video pass over query frames [f0, f1): a query of frame f reads every non-padded frame
+    <= f (R2-R3), from the cache below f0 and from the call's own K/V from f0 on; padded query
+    frames stay 0."""
+    B, _, H, _ = np.shape(q)
+    o = np.zeros(np.shape(q))
+    for b in range(B):
+        for f in range(f0, f1):
+            if pad[b][f]:
+                continue
+            src = [(g, t) for g in range(f + 1) if not pad[b][g] for t in range(T)]
+            for h in range(H):
+                keys = [list(kc[b, g * T + t, h]) if g < f0 else list(kn[b, (g - f0) * T + t, h]) for g, t in src]
+                vals = [list(vc[b, g * T + t, h]) if g < f0 else list(vn[b, (g - f0) * T + t, h]) for g, t in src]
+                for t in range(T):
+                    row = (f - f0) * T + t
+                    o[b, row, h] = _bf_attend(list(q[b, row, h]), keys, vals)
+    return o
+
+
+def _bf_store(cache, new, f0, f1, pad, T):
+    """The cache with frames [f0, f1) that are not padding taken from the call's K or V."""
+    c = np.array(cache, dtype=np.float64)
+    for b in range(c.shape[0]):
+        for f in range(f0, f1):
+            if not pad[b][f]:
+                c[b, f * T:(f + 1) * T] = new[b, (f - f0) * T:(f - f0 + 1) * T]
+    return c
+
+
+def _bf_action(qa, ka, va, fk, fv, pad, T, F):
+    """Action queries over the non-padded frames of a fused pair (when the layer reads one,
+    R9) followed by the action keys."""
+    B, n, H, _ = np.shape(qa)
+    o = np.zeros(np.shape(qa))
+    for b in range(B):
+        for h in range(H):
+            keys, vals = [], []
+            if fk is not None:
+                for g in range(F):
+                    if not pad[b][g]:
+                        keys += [list(fk[b, g * T + t, h]) for t in range(T)]
+                        vals += [list(fv[b, g * T + t, h]) for t in range(T)]
+            keys += [list(ka[b, j, h]) for j in range(n)]
+            vals += [list(va[b, j, h]) for j in range(n)]
+            for r in range(n):
+                o[b, r, h] = _bf_attend(list(qa[b, r, h]), keys, vals)
+    return o
+
+
+def _bf_intervals(L, S):
+    """I_m = {S m, .., min(S m + S, L) - 1}; the interaction layer of I_m is its last (R5)."""
+    iv = [list(range(S * m, min(S * m + S, L))) for m in range(-(-L // S))]
+    return iv, {I[-1]: m for m, I in enumerate(iv)}
+
+
+def _bf_history(inp, pad, L, T, Fh, F):
     B, _, H, D = np.shape(inp["hist_q"][0])
-    n = np.shape(inp["act_q"][0][0])[1]
-    ok = lambda b, f: not pad[b][f]
-
-    def video(q, kn, vn, kc, vc, f0, f1):
-        o = np.zeros(np.shape(q))
-        for b in range(B):
-            for f in range(f0, f1):
-                if not ok(b, f):
-                    continue
-                src = [(g, t) for g in range(f + 1) if ok(b, g) for t in range(T)]
-                for h in range(H):
-                    keys = [list(kc[b, g * T + t, h]) if g < f0 else list(kn[b, (g - f0) * T + t, h])
-                            for g, t in src]
-                    vals = [list(vc[b, g * T + t, h]) if g < f0 else list(vn[b, (g - f0) * T + t, h])
-                            for g, t in src]
-                    for t in range(T):
-                        row = (f - f0) * T + t
-                        o[b, row, h] = _bf_attend(list(q[b, row, h]), keys, vals)
-        return o
-
-    def store(cache, new, f0, f1):
-        c = cache.copy()
-        for b in range(B):
-            for f in range(f0, f1):
-                if ok(b, f):
-                    c[b, f * T:(f + 1) * T] = new[b, (f - f0) * T:(f - f0 + 1) * T]
-        return c
-
-    out = {"hist_o": [], "imag_o": [], "final_o": [], "act_o": []}
     kc = [np.zeros((B, F * T, H, D)) for _ in range(L)]
     vc = [np.zeros((B, F * T, H, D)) for _ in range(L)]
+    outs = []
     for l in range(L):
-        out["hist_o"].append(video(inp["hist_q"][l], inp["hist_k"][l], inp["hist_v"][l], kc[l], vc[l], 0, Fh))
-        kc[l], vc[l] = store(kc[l], inp["hist_k"][l], 0, Fh), store(vc[l], inp["hist_v"][l], 0, Fh)
+        outs.append(_bf_video(inp["hist_q"][l], inp["hist_k"][l], inp["hist_v"][l], kc[l], vc[l], 0, Fh, pad, T))
+        kc[l], vc[l] = _bf_store(kc[l], inp["hist_k"][l], 0, Fh, pad, T), _bf_store(vc[l], inp["hist_v"][l], 0, Fh, pad, T)
+    return outs, kc, vc
+
+
+def _bf_chunk(inp, pad, L, S, T, Fh, Ff, Nv, Ne, sigma_star):
+    """One chunk restated from the readings with loops and math.exp, calling nothing of the
+    oracle: the history pass over frames [0, Fh), its K/V stored for non-padded frames; Nv
+    imagination passes over the stored history and their own future K/V, each followed by an
+    Euler step of -(1 - sigma*) / Nv on the future latents (R1, R7); the final pass, its K/V
+    stored (R6); fused pair m = sum of w_m,j x cache_j over I_m (R5); Ne action steps where
+    layer max(I_m) reads fused pair m and the other layers the action keys only, each followed
+    by an Euler step of -1 / Ne."""
+    F = Fh + Ff
+    out = {"imag_o": [], "final_o": [], "act_o": []}
+    out["hist_o"], kc, vc = _bf_history(inp, pad, L, T, Fh, F)
     x = np.array(inp["x_future"], dtype=np.float64)
     for s in range(Nv):
-        out["imag_o"].append([video(inp["imag_q"][s][l], inp["imag_k"][s][l], inp["imag_v"][s][l],
-                                    kc[l], vc[l], Fh, F) for l in range(L)])
+        out["imag_o"].append([_bf_video(inp["imag_q"][s][l], inp["imag_k"][s][l], inp["imag_v"][s][l],
+                                        kc[l], vc[l], Fh, F, pad, T) for l in range(L)])
         x = x - (1.0 - sigma_star) / Nv * np.asarray(inp["v_future"][s])
     out["x_future"] = x
     for l in range(L):
-        out["final_o"].append(video(inp["final_q"][l], inp["final_k"][l], inp["final_v"][l], kc[l], vc[l], Fh, F))
-        kc[l], vc[l] = store(kc[l], inp["final_k"][l], Fh, F), store(vc[l], inp["final_v"][l], Fh, F)
+        out["final_o"].append(_bf_video(inp["final_q"][l], inp["final_k"][l], inp["final_v"][l], kc[l], vc[l],
+                                        Fh, F, pad, T))
+        kc[l], vc[l] = _bf_store(kc[l], inp["final_k"][l], Fh, F, pad, T), _bf_store(vc[l], inp["final_v"][l], Fh, F, pad, T)
     out["k_cache"], out["v_cache"] = kc, vc
-    intervals = [list(range(S * m, min(S * m + S, L))) for m in range(-(-L // S))]
-    out["fused_k"] = [sum(w * kc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(intervals)]
-    out["fused_v"] = [sum(w * vc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(intervals)]
-    reader = {I[-1]: m for m, I in enumerate(intervals)}
+    iv, reader = _bf_intervals(L, S)
+    out["fused_k"] = [sum(w * kc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(iv)]
+    out["fused_v"] = [sum(w * vc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(iv)]
     xa = np.array(inp["x_act"], dtype=np.float64)
     for i in range(Ne):
-        outs = []
-        for l in range(L):
-            qa, ka, va = inp["act_q"][i][l], inp["act_k"][i][l], inp["act_v"][i][l]
-            o = np.zeros(np.shape(qa))
-            for b in range(B):
-                for h in range(H):
-                    keys, vals = [], []
-                    if l in reader:
-                        fk, fv = out["fused_k"][reader[l]], out["fused_v"][reader[l]]
-                        for g in range(F):
-                            if ok(b, g):
-                                keys += [list(fk[b, g * T + t, h]) for t in range(T)]
-                                vals += [list(fv[b, g * T + t, h]) for t in range(T)]
-                    keys += [list(ka[b, j, h]) for j in range(n)]
-                    vals += [list(va[b, j, h]) for j in range(n)]
-                    for r in range(n):
-                        o[b, r, h] = _bf_attend(list(qa[b, r, h]), keys, vals)
-            outs.append(o)
-        out["act_o"].append(outs)
+        out["act_o"].append([_bf_action(inp["act_q"][i][l], inp["act_k"][i][l], inp["act_v"][i][l],
+                                        out["fused_k"][reader[l]] if l in reader else None,
+                                        out["fused_v"][reader[l]] if l in reader else None, pad, T, F)
+                             for l in range(L)])
         xa = xa - 1.0 / Ne * np.asarray(inp["v_act"][i])
     out["x_act"] = xa
     return out
+
+
+def _bf_chunk_joint(inp, pad, L, S, T, Fh, Ff, N):
+    """The co-denoising chunk restated (R10): the history pass once; at joint step i every layer
+    passes the future frames with that step's Q/K/V and stores their K/V, the fused pairs are
+    formed from the caches, every action layer reads, and both latents take an Euler step of
+    -1 / N."""
+    F = Fh + Ff
+    out = {"joint_o": [], "act_o": []}
+    out["hist_o"], kc, vc = _bf_history(inp, pad, L, T, Fh, F)
+    iv, reader = _bf_intervals(L, S)
+    x = np.array(inp["x_future"], dtype=np.float64)
+    xa = np.array(inp["x_act"], dtype=np.float64)
+    for i in range(N):
+        outs = []
+        for l in range(L):
+            outs.append(_bf_video(inp["joint_q"][i][l], inp["joint_k"][i][l], inp["joint_v"][i][l], kc[l], vc[l],
+                                  Fh, F, pad, T))
+            kc[l] = _bf_store(kc[l], inp["joint_k"][i][l], Fh, F, pad, T)
+            vc[l] = _bf_store(vc[l], inp["joint_v"][i][l], Fh, F, pad, T)
+        out["joint_o"].append(outs)
+        fk = [sum(w * kc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(iv)]
+        fv = [sum(w * vc[j] for w, j in zip(inp["fuse_weights"][m], I)) for m, I in enumerate(iv)]
+        out["act_o"].append([_bf_action(inp["act_q"][i][l], inp["act_k"][i][l], inp["act_v"][i][l],
+                                        fk[reader[l]] if l in reader else None,
+                                        fv[reader[l]] if l in reader else None, pad, T, F) for l in range(L)])
+        x = x - 1.0 / N * np.asarray(inp["v_future"][i])
+        xa = xa - 1.0 / N * np.asarray(inp["v_act"][i])
+    out.update(k_cache=kc, v_cache=vc, fused_k=fk, fused_v=fv, x_future=x, x_act=xa)
+    return out
+
+
+def _assert_same_chunk(got, want, lists, nested):
+    for key in lists:
+        assert len(got[key]) == len(want[key])
+        for a, b in zip(got[key], want[key]):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    for key in nested:
+        assert len(got[key]) == len(want[key])
+        for ra, rb in zip(got[key], want[key]):
+            for a, b in zip(ra, rb):
+                np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["x_future"], want["x_future"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(got["x_act"], want["x_act"], rtol=0, atol=1e-13)
 
 
 @pytest.mark.parametrize("pad_row", [[1, 0, 0, 0], [0, 0, 0, 0]])
@@ -486,17 +547,8 @@ def test_chunk_matches_a_brute_force_restatement(pad_row):
     got = O.chunk(inp, pad=pad, **kw)
     want = _bf_chunk(inp, pad, kw["L"], kw["S"], kw["T"], kw["F_h"], kw["F_f"], kw["n_video_steps"],
                      kw["n_euler_steps"], kw["sigma_star"])
-    for key in ("hist_o", "final_o", "k_cache", "v_cache", "fused_k", "fused_v"):
-        assert len(got[key]) == len(want[key])
-        for a, b in zip(got[key], want[key]):
-            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
-    for key in ("imag_o", "act_o"):
-        assert len(got[key]) == len(want[key])
-        for ra, rb in zip(got[key], want[key]):
-            for a, b in zip(ra, rb):
-                np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
-    np.testing.assert_allclose(got["x_future"], want["x_future"], rtol=0, atol=1e-13)
-    np.testing.assert_allclose(got["x_act"], want["x_act"], rtol=0, atol=1e-13)
+    _assert_same_chunk(got, want, ("hist_o", "final_o", "k_cache", "v_cache", "fused_k", "fused_v"),
+                       ("imag_o", "act_o"))
 
 
 def test_action_never_changes_video_outputs():
@@ -522,6 +574,15 @@ def _joint_inputs(N=3, **kw):
     inp["joint_q"], inp["joint_k"], inp["joint_v"] = inp["imag_q"], inp["imag_k"], inp["imag_v"]
     jkw = {k: ckw[k] for k in ("L", "S", "T", "F_h", "F_f")}
     return inp, jkw, N
+
+
+@pytest.mark.parametrize("pad_row", [[1, 0, 0, 0], [0, 0, 0, 0]])
+def test_joint_chunk_matches_a_brute_force_restatement(pad_row):
+    inp, jkw, N = _joint_inputs(N=3)
+    pad = np.array([pad_row], np.uint8)
+    got = O.chunk_joint(inp, n_steps=N, pad=pad, **jkw)
+    want = _bf_chunk_joint(inp, pad, jkw["L"], jkw["S"], jkw["T"], jkw["F_h"], jkw["F_f"], N)
+    _assert_same_chunk(got, want, ("hist_o", "k_cache", "v_cache", "fused_k", "fused_v"), ("joint_o", "act_o"))
 
 
 def test_joint_chunk_of_one_step_is_the_one_shot_chunk():

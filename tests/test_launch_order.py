@@ -197,3 +197,17 @@ def test_pairing_cases_are_exercised():
     # the random calls above include paired and unpaired ones
     flags = [wam.debug_prefill_order(*_random_call(s)[:4], with_pairing=True)[3] for s in range(48)]
     assert 5 <= sum(flags) <= 43
+
+
+def test_grouped_future_frames_are_not_paired():
+    # the two imagined frames in one attention block read the same key frames: equal counts,
+    # nothing to balance, so the call keeps one frame per CTA pair of tiles
+    w = synth.WORKLOADS["ctx19.2s_bf16"]
+    pad = synth.pad_mask(w).numpy()
+    block = list(range(w.F_h)) + [w.F_h] * w.F_f
+    lay = wam.VideoLayout(w.B, w.H, w.D, w.T, w.F, pad, block)
+    ep, fr, nk, paired = wam.debug_prefill_order(lay, w.F_h, w.F, B200_SMS, with_pairing=True)
+    assert not paired and list(nk) == [7, 7]
+    # one frame per block (the default layout) pairs them
+    lay1 = wam.VideoLayout(w.B, w.H, w.D, w.T, w.F, pad)
+    assert wam.debug_prefill_order(lay1, w.F_h, w.F, B200_SMS, with_pairing=True)[3]
